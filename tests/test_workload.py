@@ -1,0 +1,37 @@
+"""The synthetic decode workload reproduces the pages' cache behaviour: with
+16 LFU slots per layer the hit rate sits in the 60-70% band the pages report
+("Show HN: Motor de codigo abierto que ejecuta Gemma 4 26B en 2 GB de RAM",
+section "Enfoque tecnico"), using the oracle's router and LFU plan on the
+seeded hidden states and Zipf(s=1.1) popularity bias."""
+import numpy as np
+
+import oracle
+from expert_streaming_decode_b200 import synth
+
+
+def test_zipf_hit_rate_band():
+    O = oracle.get()
+    d = synth.GEMMA4_26B
+    wq, ws = synth.router_weights(0, 0, d.E, d.D)
+    bias = synth.zipf_bias(0, 0, d.E, s=1.1, lam=0.75)
+    st = oracle.LfuState(d.E, 16)
+    hits = total = 0
+    for t in range(700):
+        lg = O.router_logits(synth.hidden(0, t, 0, d.D), wq, ws, bias, d.E, d.D, d.G)
+        r = O.lfu_plan(st, O.topk(lg, d.K)[None], t)
+        if t >= 100:
+            hits += int(r["hit"].sum())
+            total += d.K
+    assert 0.60 <= hits / total <= 0.70, hits / total
+
+
+def test_blob_sizes():
+    """Expert blob sizes follow from the shapes: 3 matrices of 4-bit weights
+    plus a binary16 (scale, bias) pair per group of 64.  30 layers x 128
+    experts is the ~12.9 GB expert store the pages quote ("El milagro de la IA
+    de 2GB en Apple Silicon", section "Mas inteligente que tu RAM")."""
+    O = oracle.get()
+    routed = O.blob_bytes(2816, 704)
+    assert routed == 3 * 704 * 2816 // 2 + 3 * 704 * 2816 // 64 * 4 == synth.blob_bytes(2816, 704)
+    assert O.blob_bytes(2816, 2112) == 3 * routed
+    assert abs(30 * 128 * routed / 1e9 - 12.9) < 0.06
