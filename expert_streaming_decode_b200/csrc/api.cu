@@ -1,0 +1,595 @@
+// api.cu -- the C ABI of libmoe.so (declared and documented in moe.h): the
+// context, argument checking, and the host orchestration of the layer:
+// router -> cache plan -> (miss copies on the side stream || shared expert)
+// -> routed experts -> combine.
+//
+// Host I/O design ("TurboFieldfare: motor open source ...", section "Proceso
+// de generacion de tokens": the CPU turns the router's ids into a fetch plan
+// against the layer's cache, issues the reads of missing experts, and the GPU
+// runs the resident shared-expert branch while they are in flight).  Here the
+// plan itself is computed on the GPU; the host learns it through a pinned
+// mapped mailbox (one poll per layer, bounded), issues one cudaMemcpyAsync per
+// missed expert blob from pinned host memory on a side stream, and makes the
+// compute stream wait on an event.  The shared expert's kernels are already
+// queued before the host polls, so they overlap the copies.
+#include <atomic>
+#include <chrono>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "common.cuh"
+#include "ffn.cuh"
+#include "plan.cuh"
+
+namespace moe {
+cudaError_t launch_router(const uint16_t* x, const int8_t* wq, const uint16_t* ws, const float* bias, int E, int D,
+                          int K, int T, int32_t* ids, float* gate_w, int* status, cudaStream_t s);
+cudaError_t launch_residual_rmsnorm(float* r, const float* y, uint16_t* x_next, int T, int D, cudaStream_t s);
+cudaError_t launch_bf16_to_f32(const uint16_t* x, float* out, size_t n, cudaStream_t s);
+}  // namespace moe
+
+using namespace moe;
+
+struct moe_ctx {
+    moe_dims d;
+    int device = 0;
+    int sms = 0;
+    cudaStream_t side = nullptr;
+    cudaEvent_t ev_plan = nullptr, ev_fill = nullptr, ev_wave = nullptr;
+    PlanMailbox* mbox_host = nullptr;
+    PlanMailbox* mbox_dev = nullptr;
+    uint32_t seq = 0;
+    int* status = nullptr;  // device status word
+    // scratch (device)
+    WorkList* wl = nullptr;
+    FfnEntry* entries = nullptr;
+    FfnRow* rows = nullptr;
+    float* h = nullptr;
+    int h_shared_off = 0;
+    float* partials_gu = nullptr;
+    int* counters_gu = nullptr;
+    float* partials_dn = nullptr;
+    int* counters_dn = nullptr;
+    int32_t* ids = nullptr;
+    float* gate_w = nullptr;
+    int32_t* pair_slot = nullptr;
+    int32_t* pair_wave = nullptr;
+    GemvShapes shapes{};
+    uint64_t launches = 0;
+    size_t blob_routed = 0;
+    // instrumentation (moe_ctx_profile)
+    struct Rec {
+        int kind;
+        cudaEvent_t a, b;
+    };
+    bool prof = false;
+    std::vector<cudaEvent_t> pool;
+    std::vector<Rec> recs;
+    cudaEvent_t open[MOE_PROF_KINDS] = {};
+};
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+bool dims_ok(const moe_dims* d) {
+    if (!d) return false;
+    auto ff_ok = [](int F) { return F > 0 && F % 64 == 0 && (F <= 704 || F % 704 == 0); };
+    if (d->d_model <= 0 || d->d_model % 256 || d->d_model > 16384) return false;
+    if (d->group != 64) return false;
+    if (d->n_experts <= 0 || d->n_experts > 1024 || d->n_experts % 8) return false;
+    if (d->top_k <= 0 || d->top_k > 16 || d->top_k > d->n_experts) return false;
+    if (!ff_ok(d->d_ff) || d->d_ff > 3 * 704) return false;
+    if (d->d_ff_shared != 0 && (!ff_ok(d->d_ff_shared) || d->d_ff_shared > 3 * 704)) return false;
+    if (d->n_slots < d->top_k || d->n_slots > d->n_experts) return false;
+    if (d->max_tokens < 1 || d->max_tokens > 1024) return false;
+    return true;
+}
+
+template <typename T>
+cudaError_t dalloc(T** p, size_t n) {
+    return cudaMalloc(reinterpret_cast<void**>(p), n * sizeof(T) + 16);
+}
+
+void free_ctx(moe_ctx* c) {
+    if (!c) return;
+    for (auto& r : c->recs) {
+        cudaEventDestroy(r.a);
+        cudaEventDestroy(r.b);
+    }
+    for (auto e : c->pool) cudaEventDestroy(e);
+    cudaFree(c->status);
+    cudaFree(c->wl);
+    cudaFree(c->entries);
+    cudaFree(c->rows);
+    cudaFree(c->h);
+    cudaFree(c->partials_gu);
+    cudaFree(c->counters_gu);
+    cudaFree(c->partials_dn);
+    cudaFree(c->counters_dn);
+    cudaFree(c->ids);
+    cudaFree(c->gate_w);
+    cudaFree(c->pair_slot);
+    cudaFree(c->pair_wave);
+    if (c->mbox_host) cudaFreeHost(c->mbox_host);
+    if (c->ev_plan) cudaEventDestroy(c->ev_plan);
+    if (c->ev_fill) cudaEventDestroy(c->ev_fill);
+    if (c->ev_wave) cudaEventDestroy(c->ev_wave);
+    if (c->side) cudaStreamDestroy(c->side);
+    delete c;
+}
+
+// Records an instrumentation event on `s` opening (begin) or closing an
+// interval of `kind`; no-op unless profiling is enabled.
+void prof_mark(moe_ctx* c, int kind, bool begin, cudaStream_t s) {
+    if (!c->prof) return;
+    cudaEvent_t ev = nullptr;
+    if (!c->pool.empty()) {
+        ev = c->pool.back();
+        c->pool.pop_back();
+    } else if (cudaEventCreate(&ev) != cudaSuccess) {
+        c->prof = false;
+        return;
+    }
+    cudaEventRecord(ev, s);
+    if (begin) {
+        if (c->open[kind]) c->pool.push_back(c->open[kind]);
+        c->open[kind] = ev;
+    } else if (c->open[kind]) {
+        c->recs.push_back({kind, c->open[kind], ev});
+        c->open[kind] = nullptr;
+    } else {
+        c->pool.push_back(ev);
+    }
+}
+
+struct FfnHookArg {
+    moe_ctx* c;
+    cudaStream_t s;
+};
+void ffn_hook(void* p, int where) {
+    auto* h = static_cast<FfnHookArg*>(p);
+    if (where == 0) prof_mark(h->c, MOE_PROF_GATE_UP, true, h->s);
+    if (where == 1) {
+        prof_mark(h->c, MOE_PROF_GATE_UP, false, h->s);
+        prof_mark(h->c, MOE_PROF_DOWN, true, h->s);
+    }
+    if (where == 2) prof_mark(h->c, MOE_PROF_DOWN, false, h->s);
+}
+
+int max_entries(const moe_dims& d) {
+    const int pairs = d.max_tokens * d.top_k;
+    return (d.max_tokens + kMaxRows - 1) / kMaxRows + (pairs < 1024 ? pairs : 1024) + (pairs + kMaxRows - 1) / kMaxRows;
+}
+
+// Runs the expert kernels over one work list: builds it on the device, then
+// K3 (gate/up) and K4 (down + combine).
+int run_ffn(moe_ctx* c, const WorkListArgs& wa, const uint16_t* x, int T, const float* y_in, float* y,
+            uint16_t* y_bf16, cudaStream_t s) {
+    prof_mark(c, MOE_PROF_WORKLIST, true, s);
+    cudaError_t e = launch_build_worklist(wa, s);
+    prof_mark(c, MOE_PROF_WORKLIST, false, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    GemvLaunch L;
+    L.wl = c->wl;
+    L.entries = c->entries;
+    L.rows = c->rows;
+    L.x = x;
+    L.h = c->h;
+    L.y_in = y_in;
+    L.y = y;
+    L.y_bf16 = y_bf16;
+    L.partials_gu = c->partials_gu;
+    L.counters_gu = c->counters_gu;
+    L.partials_dn = c->partials_dn;
+    L.counters_dn = c->counters_dn;
+    L.D = c->d.d_model;
+    L.rmax = (T == 1) ? 1 : kMaxRows;
+    L.shapes = &c->shapes;
+    L.status = c->status;
+    FfnHookArg ha{c, s};
+    e = launch_ffn(L, s, c->prof ? ffn_hook : nullptr, &ha);
+    c->launches += 3;
+    return cuda_status(e);
+}
+
+WorkListArgs worklist_args(moe_ctx* c, int T, int K, const int32_t* pair_slot, const float* gate_w,
+                           const uint8_t* slot_base, size_t stride, int n_slot_range, int F,
+                           const uint8_t* shared_blob) {
+    WorkListArgs a;
+    a.T = T;
+    a.K = K;
+    a.pair_slot = pair_slot;
+    a.pair_wave = nullptr;
+    a.wave = 0;
+    a.gate_w = gate_w;
+    a.slot_base = slot_base;
+    a.slot_stride = stride;
+    a.n_slot_range = n_slot_range;
+    a.F = F;
+    a.shared_blob = shared_blob;
+    a.FS = c->d.d_ff_shared;
+    a.h_shared_off = c->h_shared_off;
+    a.D = c->d.d_model;
+    a.wl = c->wl;
+    a.entries = c->entries;
+    a.rows = c->rows;
+    a.status = c->status;
+    return a;
+}
+
+// Waits (bounded) until the plan kernel of call `seq` has published its
+// mailbox.  Also watches the plan event so a failed launch is an error, not a
+// time-out.
+int wait_mailbox(moe_ctx* c, uint32_t seq, int timeout_ms) {
+    const auto t0 = std::chrono::steady_clock::now();
+    volatile uint32_t* p = &c->mbox_host->seq;
+    for (uint64_t it = 0;; ++it) {
+        if (*p == seq) {
+            std::atomic_thread_fence(std::memory_order_acquire);
+            return MOE_OK;
+        }
+        if ((it & 1023) == 1023) {
+            const cudaError_t q = cudaEventQuery(c->ev_plan);
+            if (q != cudaSuccess && q != cudaErrorNotReady) return MOE_ERR_CUDA;
+            if (q == cudaSuccess && *p != seq) {
+                // the kernel finished: its system-scope writes are visible now
+                if (*p == seq) return MOE_OK;
+                return MOE_ERR_STATE;
+            }
+            const auto ms = std::chrono::duration_cast<std::chrono::milliseconds>(std::chrono::steady_clock::now() - t0);
+            if (ms.count() > timeout_ms) return MOE_ERR_TIMEOUT;
+        }
+    }
+}
+
+void copy_trace(const PlanMailbox* mb, moe_plan_trace* tr, size_t blob, uint64_t h2d) {
+    if (!tr) return;
+    tr->n_distinct = mb->n_distinct;
+    tr->n_waves = mb->n_waves;
+    tr->n_misses = mb->n_misses;
+    tr->h2d_bytes = h2d;
+    const int n = mb->n_distinct < tr->capacity ? mb->n_distinct : tr->capacity;
+    for (int i = 0; i < n; ++i) {
+        if (tr->expert) tr->expert[i] = mb->expert[i];
+        if (tr->slot) tr->slot[i] = mb->slot[i];
+        if (tr->hit) tr->hit[i] = mb->hit[i];
+        if (tr->victim) tr->victim[i] = mb->victim[i];
+        if (tr->wave) tr->wave[i] = mb->wave[i];
+    }
+    (void)blob;
+}
+
+// Issues the copies of wave `w`'s misses on the side stream after `after`
+// (an event on the compute stream), then makes `s` wait for them.
+int fill_wave(moe_ctx* c, const moe_slot_cache* cache, int w, cudaEvent_t after, cudaStream_t s, uint64_t* bytes) {
+    const PlanMailbox* mb = c->mbox_host;
+    const size_t nb = c->blob_routed;
+    if (cudaStreamWaitEvent(c->side, after, 0) != cudaSuccess) return MOE_ERR_CUDA;
+    prof_mark(c, MOE_PROF_H2D, true, c->side);
+    for (int i = 0; i < mb->n_distinct; ++i) {
+        if (mb->wave[i] != w || mb->hit[i]) continue;
+        const int e = mb->expert[i], sl = mb->slot[i];
+        if (e < 0 || e >= c->d.n_experts || sl < 0 || sl >= c->d.n_slots) return MOE_ERR_RANGE;
+        if (cudaMemcpyAsync(cache->slots + size_t(sl) * cache->slot_stride, cache->store + size_t(e) * cache->store_stride,
+                            nb, cudaMemcpyHostToDevice, c->side) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        *bytes += nb;
+    }
+    prof_mark(c, MOE_PROF_H2D, false, c->side);
+    if (cudaEventRecord(c->ev_fill, c->side) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaStreamWaitEvent(s, c->ev_fill, 0) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+int check_cache(const moe_ctx* c, const moe_slot_cache* cache) {
+    if (!cache || !cache->slots || !cache->state) return MOE_ERR_ARG;
+    if (!aligned(cache->slots, 256) || cache->slot_stride % 256 || cache->slot_stride < c->blob_routed) return MOE_ERR_ARG;
+    if (!aligned(cache->state, 16)) return MOE_ERR_ARG;
+    if (cache->store && cache->store_stride < c->blob_routed) return MOE_ERR_ARG;
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_blob_bytes(int d_model, int d_ff) {
+    if (d_model <= 0 || d_model % 256 || d_ff <= 0 || d_ff % 64 || (d_ff > 704 && d_ff % 704)) return 0;
+    return blob_bytes(d_model, d_ff);
+}
+
+size_t moe_cache_state_words(const moe_dims* d) { return d ? size_t(3) * d->n_experts + d->n_slots : 0; }
+
+const char* moe_status_str(int s) {
+    switch (s) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_ARG: return "invalid argument";
+        case MOE_ERR_CUDA: return "CUDA error";
+        case MOE_ERR_TIMEOUT: return "timed out";
+        case MOE_ERR_STATE: return "invalid state";
+        case MOE_ERR_NAN: return "NaN router logit";
+        case MOE_ERR_RANGE: return "index out of range";
+        default: return "unknown status";
+    }
+}
+
+int moe_ctx_create(const moe_dims* dims, int device, moe_ctx** out) {
+    if (!out) return MOE_ERR_ARG;
+    *out = nullptr;
+    if (!dims_ok(dims)) return MOE_ERR_ARG;
+    if (cudaSetDevice(device) != cudaSuccess) return MOE_ERR_CUDA;
+    moe_ctx* c = new (std::nothrow) moe_ctx();
+    if (!c) return MOE_ERR_CUDA;
+    c->d = *dims;
+    c->device = device;
+    c->blob_routed = blob_bytes(dims->d_model, dims->d_ff);
+    const moe_dims& d = c->d;
+    bool ok = cudaDeviceGetAttribute(&c->sms, cudaDevAttrMultiProcessorCount, device) == cudaSuccess;
+    ok = ok && cudaStreamCreateWithFlags(&c->side, cudaStreamNonBlocking) == cudaSuccess;
+    ok = ok && cudaEventCreateWithFlags(&c->ev_plan, cudaEventDisableTiming) == cudaSuccess;
+    ok = ok && cudaEventCreateWithFlags(&c->ev_fill, cudaEventDisableTiming) == cudaSuccess;
+    ok = ok && cudaEventCreateWithFlags(&c->ev_wave, cudaEventDisableTiming) == cudaSuccess;
+    ok = ok && cudaHostAlloc(reinterpret_cast<void**>(&c->mbox_host), sizeof(PlanMailbox), cudaHostAllocMapped) == cudaSuccess;
+    ok = ok && cudaHostGetDevicePointer(reinterpret_cast<void**>(&c->mbox_dev), c->mbox_host, 0) == cudaSuccess;
+    if (ok) std::memset(c->mbox_host, 0, sizeof(PlanMailbox));
+    const int T = d.max_tokens, pairs = T * d.top_k;
+    const int fmax = d.d_ff > d.d_ff_shared ? d.d_ff : d.d_ff_shared;
+    ok = ok && ffn_prepare(d.d_model, fmax, T, c->sms, &c->shapes) == cudaSuccess;
+    const int ment = max_entries(d);
+    const size_t h_floats = size_t(pairs) * d.d_ff + size_t(T) * d.d_ff_shared;
+    c->h_shared_off = pairs * d.d_ff;
+    int grid_gu = c->shapes.gu[0].grid > c->shapes.gu[1].grid ? c->shapes.gu[0].grid : c->shapes.gu[1].grid;
+    const size_t tiles_gu = size_t(ment) * (fmax / 16);
+    const int ns_dn_max = fmax / down_ks(fmax);
+    const size_t units_dn = size_t(ment) * (d.d_model / kChunkRows) * ns_dn_max;
+    ok = ok && dalloc(&c->status, 1) == cudaSuccess;
+    ok = ok && dalloc(&c->wl, 1) == cudaSuccess;
+    ok = ok && dalloc(&c->entries, ment) == cudaSuccess;
+    ok = ok && dalloc(&c->rows, size_t(T) + pairs) == cudaSuccess;
+    ok = ok && dalloc(&c->h, h_floats) == cudaSuccess;
+    ok = ok && dalloc(&c->partials_gu, size_t(2) * grid_gu * kMaxRows * 32) == cudaSuccess;
+    ok = ok && dalloc(&c->counters_gu, tiles_gu) == cudaSuccess;
+    ok = ok && dalloc(&c->partials_dn, units_dn * kMaxRows * 32) == cudaSuccess;
+    ok = ok && dalloc(&c->counters_dn, size_t(d.d_model / kChunkRows)) == cudaSuccess;
+    ok = ok && dalloc(&c->ids, pairs) == cudaSuccess;
+    ok = ok && dalloc(&c->gate_w, pairs) == cudaSuccess;
+    ok = ok && dalloc(&c->pair_slot, pairs) == cudaSuccess;
+    ok = ok && dalloc(&c->pair_wave, pairs) == cudaSuccess;
+    ok = ok && cudaMemset(c->status, 0, sizeof(int)) == cudaSuccess;
+    ok = ok && cudaMemset(c->counters_gu, 0, tiles_gu * sizeof(int)) == cudaSuccess;
+    ok = ok && cudaMemset(c->counters_dn, 0, size_t(d.d_model / kChunkRows) * sizeof(int)) == cudaSuccess;
+    ok = ok && cudaDeviceSynchronize() == cudaSuccess;
+    if (!ok) {
+        cudaGetLastError();
+        free_ctx(c);
+        return MOE_ERR_CUDA;
+    }
+    *out = c;
+    return MOE_OK;
+}
+
+int moe_ctx_destroy(moe_ctx* c) {
+    if (!c) return MOE_OK;
+    cudaSetDevice(c->device);
+    const auto t0 = std::chrono::steady_clock::now();
+    while (cudaStreamQuery(c->side) == cudaErrorNotReady &&
+           std::chrono::steady_clock::now() - t0 < std::chrono::seconds(10)) {
+    }
+    free_ctx(c);
+    return MOE_OK;
+}
+
+uint64_t moe_ctx_launches(const moe_ctx* c) { return c ? c->launches : 0; }
+
+int moe_ctx_profile(moe_ctx* c, int enable) {
+    if (!c) return MOE_ERR_ARG;
+    c->prof = enable != 0;
+    return MOE_OK;
+}
+
+int moe_ctx_profile_read(moe_ctx* c, double* total_ms, uint64_t* count) {
+    if (!c || !total_ms || !count) return MOE_ERR_ARG;
+    for (int k = 0; k < MOE_PROF_KINDS; ++k) {
+        total_ms[k] = 0.0;
+        count[k] = 0;
+    }
+    int rc = MOE_OK;
+    for (auto& r : c->recs) {
+        float ms = 0.f;
+        if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess)
+            rc = MOE_ERR_CUDA;
+        total_ms[r.kind] += ms;
+        count[r.kind] += 1;
+        c->pool.push_back(r.a);
+        c->pool.push_back(r.b);
+    }
+    c->recs.clear();
+    return rc;
+}
+
+int moe_ctx_sync(moe_ctx* c, cudaStream_t s, int timeout_ms) {
+    if (!c) return MOE_ERR_ARG;
+    const auto t0 = std::chrono::steady_clock::now();
+    for (;;) {
+        const cudaError_t a = cudaStreamQuery(s), b = cudaStreamQuery(c->side);
+        if ((a != cudaSuccess && a != cudaErrorNotReady) || (b != cudaSuccess && b != cudaErrorNotReady))
+            return MOE_ERR_CUDA;
+        if (a == cudaSuccess && b == cudaSuccess) break;
+        const auto ms = std::chrono::duration_cast<std::chrono::milliseconds>(std::chrono::steady_clock::now() - t0);
+        if (ms.count() > timeout_ms) return MOE_ERR_TIMEOUT;
+    }
+    int st = 0;
+    if (cudaMemcpy(&st, c->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+    if (st != 0 && cudaMemset(c->status, 0, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+    return st;
+}
+
+int moe_router_topk(moe_ctx* c, const uint16_t* x, const int8_t* wq, const uint16_t* ws, const float* bias, int T,
+                    int32_t* ids, float* gate_w, cudaStream_t s) {
+    if (!c || !x || !wq || !ws || !ids || !gate_w) return MOE_ERR_ARG;
+    if (T < 1 || T > c->d.max_tokens) return MOE_ERR_ARG;
+    if (!aligned(x, 16) || !aligned(wq, 16) || !aligned(ws, 4) || !aligned(ids, 4) || !aligned(gate_w, 4))
+        return MOE_ERR_ARG;
+    prof_mark(c, MOE_PROF_ROUTER, true, s);
+    const cudaError_t e = launch_router(x, wq, ws, bias, c->d.n_experts, c->d.d_model, c->d.top_k, T, ids, gate_w,
+                                        c->status, s);
+    prof_mark(c, MOE_PROF_ROUTER, false, s);
+    c->launches += 1;
+    return cuda_status(e);
+}
+
+int moe_cache_reset(moe_ctx* c, moe_slot_cache* cache, cudaStream_t s) {
+    if (!c || !cache || !cache->state) return MOE_ERR_ARG;
+    c->launches += 1;
+    return cuda_status(launch_cache_reset(cache->state, c->d.n_experts, c->d.n_slots, s));
+}
+
+// Plans the call; when the host needs the plan (store or trace) waits for the
+// mailbox.  *waves receives the wave count (0 when not waited for).
+static int plan_call(moe_ctx* c, moe_slot_cache* cache, const int32_t* ids, int T, uint32_t step, int32_t* pair_slot,
+                     bool need_host, int* waves, cudaStream_t s) {
+    const uint32_t seq = ++c->seq;
+    prof_mark(c, MOE_PROF_PLAN, true, s);
+    cudaError_t e = launch_plan(ids, T * c->d.top_k, c->d.n_experts, c->d.n_slots, cache->state, step, pair_slot,
+                                c->pair_wave, need_host ? c->mbox_dev : nullptr, seq, c->status, s);
+    prof_mark(c, MOE_PROF_PLAN, false, s);
+    c->launches += 1;
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaEventRecord(c->ev_plan, s) != cudaSuccess) return MOE_ERR_CUDA;
+    *waves = 0;
+    if (!need_host) return MOE_OK;
+    const int r = wait_mailbox(c, seq, 10000);
+    if (r != MOE_OK) return r;
+    *waves = c->mbox_host->n_waves;
+    return MOE_OK;
+}
+
+int moe_cache_plan(moe_ctx* c, moe_slot_cache* cache, const int32_t* ids, int T, uint32_t step, int32_t* pair_slot,
+                   moe_plan_trace* trace, cudaStream_t s) {
+    if (!c || !ids || !pair_slot) return MOE_ERR_ARG;
+    if (T < 1 || T > c->d.max_tokens) return MOE_ERR_ARG;
+    int r = check_cache(c, cache);
+    if (r != MOE_OK) return r;
+    const bool need_host = cache->store || trace;
+    int waves = 0;
+    r = plan_call(c, cache, ids, T, step, pair_slot, need_host, &waves, s);
+    if (r != MOE_OK) return r;
+    uint64_t bytes = 0;
+    if (cache->store && waves == 1) {
+        r = fill_wave(c, cache, 0, c->ev_plan, s, &bytes);
+        if (r != MOE_OK) return r;
+    }
+    if (need_host) copy_trace(c->mbox_host, trace, c->blob_routed, bytes);
+    return MOE_OK;
+}
+
+int moe_expert_ffn(moe_ctx* c, const uint16_t* x, int T, int top_k, const int32_t* pair_slot, const float* gate_w,
+                   const uint8_t* slot_base, size_t slot_stride, int n_slot_range, int d_ff, const float* y_in,
+                   float* y, uint16_t* y_bf16, cudaStream_t s) {
+    if (!c || !x || !pair_slot || !gate_w || !slot_base || !y) return MOE_ERR_ARG;
+    if (T < 1 || T > 32 || T > c->d.max_tokens || top_k < 1 || top_k > c->d.top_k) return MOE_ERR_ARG;
+    if (n_slot_range < 1 || n_slot_range > 1024) return MOE_ERR_ARG;
+    if (d_ff <= 0 || (d_ff != c->d.d_ff && d_ff != c->d.d_ff_shared)) return MOE_ERR_ARG;
+    if (!aligned(x, 16) || !aligned(slot_base, 256) || slot_stride % 256 || !aligned(y, 16)) return MOE_ERR_ARG;
+    if (y_in && !aligned(y_in, 16)) return MOE_ERR_ARG;
+    if (slot_stride < blob_bytes(c->d.d_model, d_ff) && n_slot_range > 1) return MOE_ERR_ARG;
+    WorkListArgs wa = worklist_args(c, T, top_k, pair_slot, gate_w, slot_base, slot_stride, n_slot_range, d_ff, nullptr);
+    if (d_ff != c->d.d_ff) {
+        // the shared-width expert through the routed interface: its rows live
+        // in the shared part of the activation buffer
+        if (T * top_k * d_ff > c->h_shared_off + T * c->d.d_ff_shared) return MOE_ERR_ARG;
+    }
+    return run_ffn(c, wa, x, T, y_in, y, y_bf16, s);
+}
+
+int moe_layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache* cache, const uint16_t* x, int T,
+                      uint32_t step, const float* bias, float* y, uint16_t* y_bf16, int32_t* ids, float* gate_w,
+                      moe_plan_trace* trace, cudaStream_t s) {
+    if (!c || !W || !W->router_q || !W->router_s || !x || !y) return MOE_ERR_ARG;
+    if (T < 1 || T > c->d.max_tokens) return MOE_ERR_ARG;
+    if (!aligned(x, 16) || !aligned(y, 16)) return MOE_ERR_ARG;
+    if (W->shared_blob && (!aligned(W->shared_blob, 256) || c->d.d_ff_shared == 0)) return MOE_ERR_ARG;
+    if (!cache && (!W->experts || !aligned(W->experts, 256) || W->expert_stride % 256 ||
+                   W->expert_stride < c->blob_routed))
+        return MOE_ERR_ARG;
+    if (cache) {
+        const int r = check_cache(c, cache);
+        if (r != MOE_OK) return r;
+    }
+    int32_t* id = ids ? ids : c->ids;
+    float* gw = gate_w ? gate_w : c->gate_w;
+    int r = moe_router_topk(c, x, W->router_q, W->router_s, bias, T, id, gw, s);
+    if (r != MOE_OK) return r;
+    const int K = c->d.top_k;
+    if (!cache) {
+        // resident: expert e's blob is W->experts + e * stride, one pass
+        WorkListArgs wa = worklist_args(c, T, K, id, gw, W->experts, W->expert_stride, c->d.n_experts, c->d.d_ff,
+                                        W->shared_blob);
+        return run_ffn(c, wa, x, T, nullptr, y, y_bf16, s);
+    }
+    // streaming: plan, then the shared expert (queued before the host waits,
+    // so it runs during the copies), then the routed experts wave by wave
+    const uint32_t seq = ++c->seq;
+    prof_mark(c, MOE_PROF_PLAN, true, s);
+    cudaError_t e = launch_plan(id, T * K, c->d.n_experts, c->d.n_slots, cache->state, step, c->pair_slot,
+                                c->pair_wave, c->mbox_dev, seq, c->status, s);
+    prof_mark(c, MOE_PROF_PLAN, false, s);
+    c->launches += 1;
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaEventRecord(c->ev_plan, s) != cudaSuccess) return MOE_ERR_CUDA;
+    bool have_y = false;
+    if (W->shared_blob) {
+        WorkListArgs wa = worklist_args(c, T, 0, c->pair_slot, gw, cache->slots, cache->slot_stride, c->d.n_slots,
+                                        c->d.d_ff, W->shared_blob);
+        r = run_ffn(c, wa, x, T, nullptr, y, nullptr, s);
+        if (r != MOE_OK) return r;
+        have_y = true;
+    }
+    r = wait_mailbox(c, seq, 10000);
+    if (r != MOE_OK) return r;
+    const int waves = c->mbox_host->n_waves;
+    uint64_t bytes = 0;
+    for (int w = 0; w < waves; ++w) {
+        if (cache->store) {
+            // wave w's victims may be slots wave w-1 still reads: copy after it
+            cudaEvent_t after = c->ev_plan;
+            if (w > 0) {
+                if (cudaEventRecord(c->ev_wave, s) != cudaSuccess) return MOE_ERR_CUDA;
+                after = c->ev_wave;
+            }
+            r = fill_wave(c, cache, w, after, s, &bytes);
+            if (r != MOE_OK) return r;
+        }
+        WorkListArgs wa = worklist_args(c, T, K, c->pair_slot, gw, cache->slots, cache->slot_stride, c->d.n_slots,
+                                        c->d.d_ff, nullptr);
+        wa.pair_wave = c->pair_wave;
+        wa.wave = w;
+        r = run_ffn(c, wa, x, T, have_y ? y : nullptr, y, (w + 1 == waves) ? y_bf16 : nullptr, s);
+        if (r != MOE_OK) return r;
+        have_y = true;
+    }
+    copy_trace(c->mbox_host, trace, c->blob_routed, bytes);
+    return MOE_OK;
+}
+
+int moe_residual_rmsnorm(moe_ctx* c, float* r, const float* y, uint16_t* x_next, int T, cudaStream_t s) {
+    if (!c || !r || !y || !x_next || T < 1) return MOE_ERR_ARG;
+    c->launches += 1;
+    prof_mark(c, MOE_PROF_HARNESS, true, s);
+    const cudaError_t e = launch_residual_rmsnorm(r, y, x_next, T, c->d.d_model, s);
+    prof_mark(c, MOE_PROF_HARNESS, false, s);
+    return cuda_status(e);
+}
+
+int moe_bf16_to_f32(moe_ctx* c, const uint16_t* x, float* out, size_t n, cudaStream_t s) {
+    if (!c || !x || !out) return MOE_ERR_ARG;
+    c->launches += 1;
+    return cuda_status(launch_bf16_to_f32(x, out, n, s));
+}
+
+}  // extern "C"

@@ -1,0 +1,62 @@
+// ffn.cuh -- host-side interface of the expert GEMV kernels (ffn.cu).
+#pragma once
+#include "common.cuh"
+
+namespace moe {
+
+struct GemvShape {
+    int grid;       // persistent CTAs (SMs x resident CTAs per SM)
+    size_t smem;    // dynamic shared memory per CTA
+};
+struct GemvShapes {
+    GemvShape gu[2];   // [0]: one token row per entry, [1]: up to kMaxRows
+    GemvShape dn[2];
+    int vstride_gu, vstride_dn;
+};
+
+struct GemvLaunch {
+    const WorkList* wl;
+    const FfnEntry* entries;
+    const FfnRow* rows;
+    const uint16_t* x;
+    float* h;
+    const float* y_in;
+    float* y;
+    uint16_t* y_bf16;
+    float* partials_gu;
+    int* counters_gu;
+    float* partials_dn;
+    int* counters_dn;
+    int D;
+    int rmax;      // 1 when every entry has one row (T == 1), else kMaxRows
+    const GemvShapes* shapes;
+    int* status;
+};
+
+struct WorkListArgs {
+    int T, K;                   // tokens, selections per token in this call (K may be 0)
+    const int32_t* pair_slot;   // [T*K]
+    const int32_t* pair_wave;   // [T*K] or null: keep only pairs with pair_wave == wave
+    int wave;
+    const float* gate_w;        // [T*K]
+    const uint8_t* slot_base;
+    size_t slot_stride;
+    int n_slot_range;
+    int F;
+    const uint8_t* shared_blob; // or null
+    int FS;
+    int h_shared_off;           // float offset of the shared rows in the h buffer
+    int D;
+    WorkList* wl;
+    FfnEntry* entries;
+    FfnRow* rows;
+    int* status;
+};
+
+cudaError_t ffn_prepare(int D, int Fmax, int T, int sms, GemvShapes* shapes);
+// Launches K3 (gate/up) then K4 (down); `between` (may be null) is called
+// after K3's launch and `after` after K4's (used for timing events).
+cudaError_t launch_ffn(const GemvLaunch& L, cudaStream_t s, void (*hook)(void*, int), void* hook_arg);
+cudaError_t launch_build_worklist(const WorkListArgs& a, cudaStream_t s);
+
+}  // namespace moe

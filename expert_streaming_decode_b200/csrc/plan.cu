@@ -1,0 +1,213 @@
+// plan.cu -- K2: per-layer LFU expert-cache plan on the device.
+//
+// Method ("El milagro de la IA de 2GB en Apple Silicon", section "Mas
+// inteligente que tu RAM": each layer keeps 16 of its 128 experts in an LFU
+// cache and a miss replaces the least frequently used resident expert;
+// "TurboFieldfare: motor open source ...", section "Proceso de generacion de
+// tokens": the top-8 ids are checked against the layer's cache and the misses
+// become a fetch plan).  Readings where the pages are silent: frequency = all
+// selections so far (kept across evictions); ties by older last use, then
+// lower id; the experts of the current wave are never evicted; empty slots
+// fill lowest first; distinct experts are planned in ascending id, in waves of
+// at most S; last_use = step + 1 after a wave.
+//
+// One CTA per call.  State is staged in shared memory, counts are gathered
+// with shared atomics, and a single warp walks the distinct experts in order;
+// each miss picks its slot with a ballot (empty slot) or a shuffle arg-min
+// over the resident slots (victim).  Results: pair -> slot map and pair ->
+// wave map in device memory, and the per-expert plan in the pinned mapped
+// mailbox for the host, published by writing `seq` last.
+#include "common.cuh"
+#include "plan.cuh"
+
+namespace moe {
+
+constexpr int kPlanThreads = 256;
+
+__global__ void __launch_bounds__(kPlanThreads) cache_plan_kernel(
+    const int32_t* __restrict__ ids, int npairs, int E, int S, int32_t* __restrict__ state, uint32_t step,
+    int32_t* __restrict__ pair_slot, int32_t* __restrict__ pair_wave, PlanMailbox* mailbox, uint32_t seq,
+    int* status) {
+    extern __shared__ int32_t psm[];
+    uint32_t* mult = reinterpret_cast<uint32_t*>(psm);   // [E] selections in this call
+    uint32_t* count = mult + E;                           // [E]
+    uint32_t* last = count + E;                           // [E]
+    int32_t* slot_of = reinterpret_cast<int32_t*>(last + E);  // [E]
+    int32_t* expert_in = slot_of + E;                     // [S]
+    int32_t* uslot = expert_in + S;                       // [E] slot of expert in its wave
+    int32_t* uwave = uslot + E;                           // [E]
+    uint8_t* inwave = reinterpret_cast<uint8_t*>(uwave + E);  // [E]
+    __shared__ int32_t ulist[1024];
+
+    uint32_t* g_count = reinterpret_cast<uint32_t*>(state);
+    uint32_t* g_last = g_count + E;
+    int32_t* g_slot_of = state + 2 * E;
+    int32_t* g_expert_in = state + 3 * E;
+
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        mult[e] = 0;
+        count[e] = g_count[e];
+        last[e] = g_last[e];
+        slot_of[e] = g_slot_of[e];
+        uslot[e] = -1;
+        uwave[e] = -1;
+        inwave[e] = 0;
+    }
+    for (int s = threadIdx.x; s < S; s += blockDim.x) expert_in[s] = g_expert_in[s];
+    __syncthreads();
+    bool bad = false;
+    for (int p = threadIdx.x; p < npairs; p += blockDim.x) {
+        int e = ids[p];
+        if (e < 0 || e >= E) { bad = true; e = 0; }
+        atomicAdd(&mult[e], 1u);
+    }
+    if (bad) set_status(status, MOE_ERR_RANGE);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) count[e] += mult[e];
+    __syncthreads();
+
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        // distinct experts, ascending id (ballot compaction)
+        int n = 0;
+        for (int base = 0; base < E; base += 32) {
+            const int e = base + lane;
+            const bool f = e < E && mult[e] > 0;
+            const uint32_t b = __ballot_sync(0xffffffffu, f);
+            if (f) ulist[n + __popc(b & ((1u << lane) - 1u))] = e;
+            n += __popc(b);
+        }
+        __syncwarp();
+        int n_miss = 0;
+        const int waves = (n + S - 1) / S;
+        for (int w = 0; w < waves; ++w) {
+            const int lo = w * S, hi = min(n, (w + 1) * S);
+            for (int i = lo + lane; i < hi; i += 32) inwave[ulist[i]] = 1;
+            __syncwarp();
+            for (int i = lo; i < hi; ++i) {
+                const int e = ulist[i];
+                int victim = -1, slot = slot_of[e];
+                if (slot >= S) {  // corrupted state: treat as not resident, report
+                    if (lane == 0) set_status(status, MOE_ERR_STATE);
+                    slot = -1;
+                }
+                const bool hit = slot >= 0;
+                if (!hit) {
+                    // lowest empty slot
+                    slot = -1;
+                    for (int base = 0; base < S && slot < 0; base += 32) {
+                        const int s = base + lane;
+                        const uint32_t b = __ballot_sync(0xffffffffu, s < S && expert_in[s] < 0);
+                        if (b) slot = base + __ffs(b) - 1;
+                    }
+                    if (slot < 0) {
+                        // victim: smallest (count, last_use, id) among resident, not in this wave
+                        uint32_t bc = 0xffffffffu, bl = 0xffffffffu;
+                        int br = 0x7fffffff;
+                        for (int s = lane; s < S; s += 32) {
+                            const int r = expert_in[s];
+                            if (r < 0 || r >= E || inwave[r]) continue;
+                            if (count[r] < bc || (count[r] == bc && (last[r] < bl || (last[r] == bl && r < br)))) {
+                                bc = count[r]; bl = last[r]; br = r;
+                            }
+                        }
+#pragma unroll
+                        for (int off = 16; off > 0; off >>= 1) {
+                            const uint32_t oc = __shfl_xor_sync(0xffffffffu, bc, off);
+                            const uint32_t ol = __shfl_xor_sync(0xffffffffu, bl, off);
+                            const int orr = __shfl_xor_sync(0xffffffffu, br, off);
+                            if (oc < bc || (oc == bc && (ol < bl || (ol == bl && orr < br)))) {
+                                bc = oc; bl = ol; br = orr;
+                            }
+                        }
+                        if (br < E) {  // S >= wave size guarantees one exists in a valid state
+                            victim = br;
+                            slot = slot_of[victim];
+                        }
+                        if (slot < 0 || slot >= S) {  // corrupted state: stay in bounds, report
+                            if (lane == 0) set_status(status, MOE_ERR_STATE);
+                            victim = -1;
+                            slot = 0;
+                        }
+                    }
+                    __syncwarp();
+                    if (lane == 0) {
+                        if (victim >= 0) slot_of[victim] = -1;
+                        const int prev = expert_in[slot];
+                        if (prev >= 0 && prev < E && prev != victim) slot_of[prev] = -1;
+                        slot_of[e] = slot;
+                        expert_in[slot] = e;
+                    }
+                    ++n_miss;
+                }
+                if (lane == 0) {
+                    uslot[e] = slot;
+                    uwave[e] = w;
+                    if (mailbox) {
+                        mailbox->expert[i] = e;
+                        mailbox->slot[i] = slot;
+                        mailbox->hit[i] = hit ? 1 : 0;
+                        mailbox->victim[i] = victim;
+                        mailbox->wave[i] = w;
+                    }
+                }
+                __syncwarp();
+            }
+            for (int i = lo + lane; i < hi; i += 32) {
+                last[ulist[i]] = step + 1u;
+                inwave[ulist[i]] = 0;
+            }
+            __syncwarp();
+        }
+        if (lane == 0) {
+            if (mailbox) {
+                mailbox->n_distinct = n;
+                mailbox->n_waves = waves;
+                mailbox->n_misses = n_miss;
+            }
+        }
+    }
+    __syncthreads();
+    for (int p = threadIdx.x; p < npairs; p += blockDim.x) {
+        int e = ids[p];
+        if (e < 0 || e >= E) e = 0;
+        pair_slot[p] = uslot[e];
+        if (pair_wave) pair_wave[p] = uwave[e];
+    }
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        g_count[e] = count[e];
+        g_last[e] = last[e];
+        g_slot_of[e] = slot_of[e];
+    }
+    for (int s = threadIdx.x; s < S; s += blockDim.x) g_expert_in[s] = expert_in[s];
+    if (mailbox) {
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            __threadfence_system();
+            *reinterpret_cast<volatile uint32_t*>(&mailbox->seq) = seq;
+            __threadfence_system();
+        }
+    }
+}
+
+size_t plan_smem_bytes(int E, int S) { return size_t(E) * 4 * 6 + size_t(S) * 4 + size_t(E) + 16; }
+
+cudaError_t launch_plan(const int32_t* ids, int npairs, int E, int S, int32_t* state, uint32_t step,
+                        int32_t* pair_slot, int32_t* pair_wave, PlanMailbox* mailbox, uint32_t seq, int* status,
+                        cudaStream_t s) {
+    cache_plan_kernel<<<1, kPlanThreads, plan_smem_bytes(E, S), s>>>(ids, npairs, E, S, state, step, pair_slot,
+                                                                     pair_wave, mailbox, seq, status);
+    return cudaGetLastError();
+}
+
+__global__ void cache_reset_kernel(int32_t* state, int E, int S) {
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < 3 * E + S; i += gridDim.x * blockDim.x)
+        state[i] = (i < 2 * E) ? 0 : -1;
+}
+
+cudaError_t launch_cache_reset(int32_t* state, int E, int S, cudaStream_t s) {
+    cache_reset_kernel<<<4, 256, 0, s>>>(state, E, S);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

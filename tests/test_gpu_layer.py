@@ -1,0 +1,184 @@
+"""GPU parity of the whole layer (moe_layer_forward) against the CPU oracle on
+the workloads of the pages' model shape: decode with every expert resident,
+decode streaming from a pinned host store through the 16-slot LFU cache,
+batched decode, and a 128-token prefill chunk with cold caches.
+
+Inputs are seeded generator hidden states for every (token, layer), so the
+oracle and the GPU see identical inputs; ids and cache traces must match bit
+for bit, outputs within max|y - r| <= 2e-3 * max|r|."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from expert_streaming_decode_b200 import moe, synth
+from gpu_data import GATE_TOL, TOL, Layer, bf16_tensor, rel_err
+
+pytestmark = pytest.mark.gpu
+
+FULL = synth.GEMMA4_26B
+TINY = synth.TINY
+
+
+@pytest.fixture(scope="module")
+def O():
+    return oracle.get()
+
+
+def _check_token(O, L, xb, ids, gw, y):
+    want_ids, want_w, _, want_y = L.oracle_token(O, xb)
+    assert np.array_equal(ids, want_ids), (ids, want_ids)
+    assert np.max(np.abs(gw - want_w)) <= GATE_TOL
+    err = rel_err(y, want_y)
+    assert err <= TOL, err
+    return err
+
+
+@pytest.mark.parametrize("d", [TINY, FULL], ids=["tiny", "full"])
+def test_decode_resident_single_layer(O, d):
+    """One layer, all experts resident, 16 sequential decode tokens."""
+    L = Layer(d, layer=0, seed=0, zipf_s=None)
+    ctx = moe.Ctx.from_dims(d, max_tokens=1)
+    W = L.weights()
+    y = torch.empty((1, d.D), dtype=torch.float32, device="cuda")
+    ids = torch.empty((1, d.K), dtype=torch.int32, device="cuda")
+    gw = torch.empty((1, d.K), dtype=torch.float32, device="cuda")
+    for t in range(16):
+        xb = synth.hidden(0, t, 0, d.D)
+        moe.layer_forward(ctx, W, None, bf16_tensor(xb[None]), 1, t, None, y, ids=ids, gate_w=gw)
+        ctx.sync()
+        _check_token(O, L, xb, ids.cpu().numpy()[0], gw.cpu().numpy()[0], y.cpu().numpy()[0])
+
+
+@pytest.mark.parametrize("d,T", [(TINY, 8), (FULL, 8), (FULL, 32)], ids=["tiny-8", "full-8", "full-32"])
+def test_batched_decode_resident(O, d, T):
+    L = Layer(d, layer=1, seed=2, zipf_s=None)
+    ctx = moe.Ctx.from_dims(d, max_tokens=T)
+    xb = synth.hidden_batch(2, range(T), 1, d.D)
+    y = torch.empty((T, d.D), dtype=torch.float32, device="cuda")
+    yb = torch.empty((T, d.D), dtype=torch.int16, device="cuda")
+    ids = torch.empty((T, d.K), dtype=torch.int32, device="cuda")
+    gw = torch.empty((T, d.K), dtype=torch.float32, device="cuda")
+    moe.layer_forward(ctx, L.weights(), None, bf16_tensor(xb), T, 0, None, y, yb, ids, gw)
+    ctx.sync()
+    ids_h, gw_h, y_h = ids.cpu().numpy(), gw.cpu().numpy(), y.cpu().numpy()
+    sample = range(T) if d is TINY else [0, 1, T // 2, T - 1]
+    for t in sample:
+        _check_token(O, L, xb[t], ids_h[t], gw_h[t], y_h[t])
+    assert np.array_equal(yb.cpu().numpy().view(np.uint16), synth.to_bf16_bits(y_h))
+
+
+def _streaming(O, d, layers, tokens, S, check_y_every=1, T=1):
+    Ls = [Layer(d, layer=l, seed=1, zipf_s=1.1, resident=False, pinned=True) for l in range(layers)]
+    ctx = moe.Ctx.from_dims(d, max_tokens=T, S=S)
+    caches, states, slotbufs = [], [], []
+    for L in Ls:
+        state = torch.empty(ctx.state_words(), dtype=torch.int32, device="cuda")
+        slots = torch.empty((S, L.stride), dtype=torch.uint8, device="cuda")
+        c = moe.slot_cache(slots, L.stride, state, L.store_t, L.stride)
+        moe.cache_reset(ctx, c)
+        caches.append(c)
+        states.append(state)
+        slotbufs.append(slots)
+    ost = [oracle.LfuState(d.E, S) for _ in Ls]
+    y = torch.empty((T, d.D), dtype=torch.float32, device="cuda")
+    ids = torch.empty((T, d.K), dtype=torch.int32, device="cuda")
+    gw = torch.empty((T, d.K), dtype=torch.float32, device="cuda")
+    tr = moe.Trace(d.E)
+    hits = misses = 0
+    for step in range(tokens):
+        for l, L in enumerate(Ls):
+            xb = synth.hidden_batch(1, range(step * T, step * T + T), l, d.D)
+            moe.layer_forward(ctx, L.weights(resident=False), caches[l], bf16_tensor(xb), T, step, L.bias_t, y,
+                              ids=ids, gate_w=gw, trace=tr)
+            ctx.sync()
+            got = tr.result()
+            ids_h = ids.cpu().numpy()
+            oids = np.stack([O.topk(O.router_logits(xb[t], L.wq, L.ws, L.bias, d.E, d.D, d.G), d.K)
+                             for t in range(T)])
+            assert np.array_equal(ids_h, oids), (step, l)
+            want = O.lfu_plan(ost[l], oids, step)
+            for key in ("expert", "slot", "hit", "victim", "wave"):
+                assert np.array_equal(got[key], want[key]), (step, l, key)
+            nmiss = int((want["hit"] == 0).sum())
+            assert got["misses"] == nmiss and got["h2d_bytes"] == nmiss * L.nb
+            hits += int(want["hit"].sum())
+            misses += nmiss
+            if step % check_y_every == 0:
+                for t in range(T):
+                    _check_token(O, L, xb[t], ids_h[t], gw.cpu().numpy()[t], y.cpu().numpy()[t])
+            # slot contents equal the store's blob of the expert the oracle placed there
+            if step % 7 == 0:
+                sl = slotbufs[l].cpu().numpy()
+                for s_, e_ in enumerate(ost[l].expert_in):
+                    if e_ >= 0:
+                        assert np.array_equal(sl[s_, :L.nb], L.blobs[e_]), (step, l, s_, e_)
+    return hits, misses
+
+
+def test_streaming_decode_tiny(O):
+    _streaming(O, TINY, layers=3, tokens=40, S=6)
+
+
+def test_streaming_decode_full(O):
+    """Three layers of the real shape, 24 tokens, 16 slots, Zipf(1.1) router
+    bias: traces bit-exact every token, outputs checked every 4th token."""
+    h, m = _streaming(O, FULL, layers=3, tokens=24, S=16, check_y_every=4)
+    assert h + m == 3 * 24 * 8
+
+
+def test_streaming_batched_decode(O):
+    _streaming(O, FULL, layers=1, tokens=4, S=16, check_y_every=2, T=4)
+
+
+@pytest.mark.parametrize("S", [16, 8])
+def test_prefill_chunk_cold_cache(O, S):
+    """A 128-token chunk through a cold 16-slot (and 8-slot) cache: the
+    distinct experts exceed the slots, so the plan runs in waves; traces must
+    match and sampled tokens' outputs too."""
+    d, T = FULL, 128
+    L = Layer(d, layer=2, seed=5, zipf_s=1.1, resident=False, pinned=True)
+    ctx = moe.Ctx.from_dims(d, max_tokens=T, S=S)
+    state = torch.empty(ctx.state_words(), dtype=torch.int32, device="cuda")
+    slots = torch.empty((S, L.stride), dtype=torch.uint8, device="cuda")
+    cache = moe.slot_cache(slots, L.stride, state, L.store_t, L.stride)
+    moe.cache_reset(ctx, cache)
+    xb = synth.hidden_batch(5, range(T), 2, d.D)
+    y = torch.empty((T, d.D), dtype=torch.float32, device="cuda")
+    ids = torch.empty((T, d.K), dtype=torch.int32, device="cuda")
+    gw = torch.empty((T, d.K), dtype=torch.float32, device="cuda")
+    tr = moe.Trace(d.E)
+    moe.layer_forward(ctx, L.weights(resident=False), cache, bf16_tensor(xb), T, 0, L.bias_t, y, ids=ids,
+                      gate_w=gw, trace=tr)
+    ctx.sync()
+    got = tr.result()
+    oids = np.stack([O.topk(O.router_logits(xb[t], L.wq, L.ws, L.bias, d.E, d.D, d.G), d.K) for t in range(T)])
+    assert np.array_equal(ids.cpu().numpy(), oids)
+    want = O.lfu_plan(oracle.LfuState(d.E, S), oids, 0)
+    for key in ("expert", "slot", "hit", "victim", "wave"):
+        assert np.array_equal(got[key], want[key]), key
+    assert got["waves"] == want["waves"] > 1
+    assert got["h2d_bytes"] == got["misses"] * L.nb == got["n_distinct"] * L.nb  # cold: every expert misses
+    for t in (0, 1, 63, 127):
+        _check_token(O, L, xb[t], ids.cpu().numpy()[t], gw.cpu().numpy()[t], y.cpu().numpy()[t])
+
+
+def test_resident_no_shared_expert(O):
+    d = TINY
+    L = Layer(d, layer=0, seed=9, zipf_s=None, shared=False)
+    L.shared = None
+    ctx = moe.Ctx.from_dims(d, max_tokens=2)
+    xb = synth.hidden_batch(9, range(2), 0, d.D)
+    y = torch.empty((2, d.D), dtype=torch.float32, device="cuda")
+    ids = torch.empty((2, d.K), dtype=torch.int32, device="cuda")
+    gw = torch.empty((2, d.K), dtype=torch.float32, device="cuda")
+    moe.layer_forward(ctx, L.weights(), None, bf16_tensor(xb), 2, 0, None, y, ids=ids, gate_w=gw)
+    ctx.sync()
+    for t in range(2):
+        _check_token(O, L, xb[t], ids.cpu().numpy()[t], gw.cpu().numpy()[t], y.cpu().numpy()[t])
+
+
+def test_minimum_slots_equal_top_k(O):
+    """S = K: every wave fills the whole cache; still bit-exact."""
+    d = TINY
+    _streaming(O, d, layers=1, tokens=30, S=d.K)
