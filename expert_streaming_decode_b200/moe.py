@@ -176,8 +176,12 @@ def router_topk(ctx: Ctx, x, wq, ws, bias, T, ids, gate_w, stream=None):
 
 
 def slot_cache(slots, slot_stride, state, store=None, store_stride=0) -> moe_slot_cache:
-    return moe_slot_cache(slots.data_ptr(), slot_stride, state.data_ptr(),
-                          None if store is None else store.data_ptr(), store_stride)
+    """moe_slot_cache for torch tensors.  The struct keeps references to the
+    tensors, so their memory lives at least as long as the struct."""
+    c = moe_slot_cache(slots.data_ptr(), slot_stride, state.data_ptr(),
+                       None if store is None else store.data_ptr(), store_stride)
+    c._keep = (slots, state, store)
+    return c
 
 
 def cache_reset(ctx: Ctx, cache: moe_slot_cache, stream=None):
@@ -215,9 +219,13 @@ def expert_ffn(ctx: Ctx, x, T, top_k, pair_slot, gate_w, slot_base, slot_stride,
 
 
 def layer_weights(router_q, router_s, shared_blob=None, experts=None, expert_stride=0) -> moe_layer_weights:
-    return moe_layer_weights(router_q.data_ptr(), router_s.data_ptr(),
-                             None if shared_blob is None else shared_blob.data_ptr(),
-                             None if experts is None else experts.data_ptr(), expert_stride)
+    """moe_layer_weights for torch tensors; keeps references to them (a struct
+    of raw pointers alone would let the allocator reuse their memory)."""
+    w = moe_layer_weights(router_q.data_ptr(), router_s.data_ptr(),
+                          None if shared_blob is None else shared_blob.data_ptr(),
+                          None if experts is None else experts.data_ptr(), expert_stride)
+    w._keep = (router_q, router_s, shared_blob, experts)
+    return w
 
 
 def layer_forward(ctx: Ctx, W: moe_layer_weights, cache: moe_slot_cache | None, x, T, step, bias, y, y_bf16=None,
