@@ -49,13 +49,18 @@ def parse_args():
     p.add_argument("--workload", default="decode_stream", choices=["decode_stream", "decode_resident", "prefill"])
     p.add_argument("--batch", type=int, default=1)
     p.add_argument("--slots", type=int, default=16)
-    p.add_argument("--zipf", type=float, default=1.1)
+    p.add_argument("--zipf", type=float, default=None,
+                   help="Zipf exponent of the router popularity bias (default 1.1; 0 = uniform router, "
+                        "the default for decode_resident)")
     p.add_argument("--layers", type=int, default=30)
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
     p.add_argument("--profile", action="store_true", help="short run for ncu: no clocks, e2e or cpu legs")
-    return p.parse_args()
+    a = p.parse_args()
+    if a.zipf is None:
+        a.zipf = 0.0 if a.workload == "decode_resident" else 1.1
+    return a
 
 
 # --------------------------------------------------------------- helpers

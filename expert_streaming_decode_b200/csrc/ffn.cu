@@ -424,6 +424,46 @@ cudaError_t ffn_prepare(int D, int Fmax, int T, int sms, GemvShapes* shapes) {
     return cudaSuccess;
 }
 
+template <int MODE>
+static cudaError_t raise_smem(size_t smem) {
+    auto kern = stream_gemv_kernel<MODE, 1>;
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return e;
+    if (size_t(fa.maxDynamicSharedSizeBytes) >= smem) return cudaSuccess;
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+}
+
+template <int MODE>
+static cudaError_t one_row_shape(int vstride, int T, int sms, GemvShape* out) {
+    const size_t smem = gemv_smem<MODE, 1>(vstride, T);
+    cudaError_t e = raise_smem<MODE>(smem);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, stream_gemv_kernel<MODE, 1>,
+                                                      (GemvCfg<MODE>::NW + 1) * 32, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    out->grid = sms * per_sm;
+    out->smem = smem;
+    return cudaSuccess;
+}
+
+cudaError_t ffn_shapes_one_row(int vstride_gu, int vstride_dn, int T, int sms, GemvShapes* shapes) {
+    *shapes = GemvShapes{};
+    shapes->vstride_gu = vstride_gu;
+    shapes->vstride_dn = vstride_dn;
+    cudaError_t e = one_row_shape<0>(vstride_gu, T, sms, &shapes->gu[0]);
+    if (e != cudaSuccess) return e;
+    return one_row_shape<1>(vstride_dn, T, sms, &shapes->dn[0]);
+}
+
+cudaError_t ffn_ensure_one_row_smem(const GemvShapes& shapes) {
+    cudaError_t e = raise_smem<0>(shapes.gu[0].smem);
+    if (e != cudaSuccess) return e;
+    return raise_smem<1>(shapes.dn[0].smem);
+}
+
 cudaError_t launch_ffn(const GemvLaunch& L, cudaStream_t s, void (*hook)(void*, int), void* hook_arg) {
     GemvArgs a;
     a.wl = L.wl;

@@ -54,6 +54,13 @@ struct WorkListArgs {
 };
 
 cudaError_t ffn_prepare(int D, int Fmax, int T, int sms, GemvShapes* shapes);
+// Launch shapes of the one-row variants (shapes->gu[0], dn[0]) for inputs up
+// to vstride_gu / vstride_dn wide and T tokens, raising (never lowering) each
+// kernel's dynamic shared-memory limit; the [1] entries are left zero.
+cudaError_t ffn_shapes_one_row(int vstride_gu, int vstride_dn, int T, int sms, GemvShapes* shapes);
+// Raises the one-row kernels' shared-memory limits back to what `shapes`
+// needs, should another user of the library have lowered them since.
+cudaError_t ffn_ensure_one_row_smem(const GemvShapes& shapes);
 // Launches K3 (gate/up) then K4 (down); `between` (may be null) is called
 // after K3's launch and `after` after K4's (used for timing events).
 cudaError_t launch_ffn(const GemvLaunch& L, cudaStream_t s, void (*hook)(void*, int), void* hook_arg);

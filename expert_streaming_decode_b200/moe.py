@@ -76,6 +76,8 @@ lib.moe_cache_plan.restype = _i
 lib.moe_cache_plan.argtypes = [_vp, C.POINTER(moe_slot_cache), _vp, _i, _u32, _vp, C.POINTER(moe_plan_trace), _vp]
 lib.moe_expert_ffn.restype = _i
 lib.moe_expert_ffn.argtypes = [_vp, _vp, _i, _i, _vp, _vp, _vp, _sz, _i, _i, _vp, _vp, _vp, _vp]
+lib.moe_expert_ffn_noalloc.restype = _i
+lib.moe_expert_ffn_noalloc.argtypes = [_i, _i, _i, _vp, _vp, _vp, _vp, _sz, _i, _vp, _vp, _vp, _vp]
 lib.moe_layer_forward.restype = _i
 lib.moe_layer_forward.argtypes = [_vp, C.POINTER(moe_layer_weights), C.POINTER(moe_slot_cache), _vp, _i, _u32,
                                   _vp, _vp, _vp, _vp, _vp, C.POINTER(moe_plan_trace), _vp]
@@ -216,6 +218,15 @@ def expert_ffn(ctx: Ctx, x, T, top_k, pair_slot, gate_w, slot_base, slot_stride,
     _check(lib.moe_expert_ffn(ctx.h, _ptr(x), T, top_k, _ptr(pair_slot), _ptr(gate_w), base, slot_stride,
                               n_slot_range, d_ff, _ptr(y_in), _ptr(y), _ptr(y_bf16), _stream(stream)),
            "moe_expert_ffn")
+
+
+def expert_ffn_noalloc(d_model, d_ff, top_k, x, pair_slot, gate_w, slot_base, slot_stride, n_slot_range, y_in, y,
+                       y_bf16=None, stream=None, slot_base_ptr=None):
+    """moe_expert_ffn_noalloc: one token, no context and no device allocation."""
+    base = C.c_void_p(slot_base_ptr) if slot_base_ptr is not None else _ptr(slot_base)
+    _check(lib.moe_expert_ffn_noalloc(d_model, d_ff, top_k, _ptr(x), _ptr(pair_slot), _ptr(gate_w), base,
+                                      slot_stride, n_slot_range, _ptr(y_in), _ptr(y), _ptr(y_bf16),
+                                      _stream(stream)), "moe_expert_ffn_noalloc")
 
 
 def layer_weights(router_q, router_s, shared_blob=None, experts=None, expert_stride=0) -> moe_layer_weights:

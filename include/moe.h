@@ -229,6 +229,36 @@ int moe_expert_ffn(moe_ctx *ctx, const uint16_t *x, int T, int top_k, const int3
                    int n_slot_range, int d_ff, const float *y_in, float *y, uint16_t *y_bf16,
                    cudaStream_t stream);
 
+/* Routed experts + combine for ONE token without any device allocation, for
+ * callers that may not allocate: code running inside another program's memory
+ * budget (an engine that gives each plugin a fixed workspace and owns every
+ * device allocation), or code on a latency-critical path where cudaMalloc and
+ * cudaFree can synchronise the device.  Such callers cannot create a moe_ctx,
+ * whose scratch is allocated; this entry point needs none.  (The pages have
+ * no counterpart: their runtime is a single process that owns its memory.)
+ * Computes, for T = 1,
+ *   y = (y_in ? y_in : 0) + sum_{k<top_k} gate_w[k] * FFN_{pair_slot[k]}(x)
+ * with the same kernels and arguments as moe_expert_ffn (x dev bf16 [d_model],
+ * pair_slot dev int32 [top_k], gate_w dev fp32 [top_k], slot_base/slot_stride/
+ * n_slot_range as there, y_in/y dev fp32 [d_model], y_bf16 dev bf16 or NULL).
+ * Limits of the fixed scratch: d_model <= 2816 (multiple of 256), d_ff <= 2112,
+ * top_k <= 8; larger sizes return MOE_ERR_ARG before any CUDA call.  Slots of
+ * one token must be distinct.
+ * Scratch: a 4 MiB file-scope device array inside libmoe.so, present on every
+ * GPU that loads the library until the process exits.  The FIRST call on each
+ * device sets up that device (looks up the array's device address and the
+ * kernels' launch shapes, with the device current); make that first call
+ * before any stream capture.  Every call shares the array and it keeps the
+ * last call's contents: calls whose work overlaps on the GPU race, so issue
+ * them on one stream (or order them).  Errors: MOE_ERR_ARG (sizes, pointers),
+ * MOE_ERR_CUDA (a launch or the set-up failed), MOE_ERR_STATE (the GPU has
+ * more SMs than the scratch covers).  Slot indices out of range are clamped;
+ * there is no status word to read back. */
+int moe_expert_ffn_noalloc(int d_model, int d_ff, int top_k, const uint16_t *x, const int32_t *pair_slot,
+                           const float *gate_w, const uint8_t *slot_base, size_t slot_stride,
+                           int n_slot_range, const float *y_in, float *y, uint16_t *y_bf16,
+                           cudaStream_t stream);
+
 /* ----------------------------------------------------------- whole layer
  * Resident weights of one layer. */
 typedef struct moe_layer_weights {
