@@ -22,12 +22,15 @@
 #include "common.cuh"
 #include "ffn.cuh"
 #include "plan.cuh"
+#include <cstdlib>
 
 namespace moe {
 cudaError_t launch_router(const uint16_t* x, const int8_t* wq, const uint16_t* ws, const float* bias, int E, int D,
-                          int K, int T, int32_t* ids, float* gate_w, int* status, cudaStream_t s);
-cudaError_t launch_residual_rmsnorm(float* r, const float* y, uint16_t* x_next, int T, int D, cudaStream_t s);
-cudaError_t launch_bf16_to_f32(const uint16_t* x, float* out, size_t n, cudaStream_t s);
+                          int K, int T, int32_t* ids, float* gate_w, int* status, const DecodeWLTarget& wlt,
+                          const uint8_t* pf_ptr, size_t pf_bytes, bool pdl, cudaStream_t s);
+cudaError_t launch_residual_rmsnorm(float* r, const float* y, uint16_t* x_next, int T, int D, bool pdl,
+                                    cudaStream_t s);
+cudaError_t launch_bf16_to_f32(const uint16_t* x, float* out, size_t n, bool pdl, cudaStream_t s);
 }  // namespace moe
 
 using namespace moe;
@@ -42,10 +45,15 @@ struct moe_ctx {
     PlanMailbox* mbox_dev = nullptr;
     uint32_t seq = 0;
     int* status = nullptr;  // device status word
-    // scratch (device)
+    bool pdl = true;  // programmatic dependent launch between this context's kernels
+    // scratch (device); the second work list holds the routed phase of a
+    // streamed one-token layer while the first holds its shared phase
     WorkList* wl = nullptr;
     FfnEntry* entries = nullptr;
     FfnRow* rows = nullptr;
+    WorkList* wl2 = nullptr;
+    FfnEntry* entries2 = nullptr;
+    FfnRow* rows2 = nullptr;
     float* h = nullptr;
     int h_shared_off = 0;
     float* partials_gu = nullptr;
@@ -59,6 +67,7 @@ struct moe_ctx {
     GemvShapes shapes{};
     uint64_t launches = 0;
     size_t blob_routed = 0;
+    size_t blob_shared = 0;
     // instrumentation (moe_ctx_profile)
     struct Rec {
         int kind;
@@ -106,6 +115,9 @@ void free_ctx(moe_ctx* c) {
     cudaFree(c->wl);
     cudaFree(c->entries);
     cudaFree(c->rows);
+    cudaFree(c->wl2);
+    cudaFree(c->entries2);
+    cudaFree(c->rows2);
     cudaFree(c->h);
     cudaFree(c->partials_gu);
     cudaFree(c->counters_gu);
@@ -166,18 +178,14 @@ int max_entries(const moe_dims& d) {
     return (d.max_tokens + kMaxRows - 1) / kMaxRows + (pairs < 1024 ? pairs : 1024) + (pairs + kMaxRows - 1) / kMaxRows;
 }
 
-// Runs the expert kernels over one work list: builds it on the device, then
-// K3 (gate/up) and K4 (down + combine).
-int run_ffn(moe_ctx* c, const WorkListArgs& wa, const uint16_t* x, int T, const float* y_in, float* y,
-            uint16_t* y_bf16, cudaStream_t s) {
-    prof_mark(c, MOE_PROF_WORKLIST, true, s);
-    cudaError_t e = launch_build_worklist(wa, s);
-    prof_mark(c, MOE_PROF_WORKLIST, false, s);
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
+// K3 (gate/up) and K4 (down + combine) over a work list already on the device.
+int run_ffn_list(moe_ctx* c, WorkList* wl, FfnEntry* entries, FfnRow* rows, const uint16_t* x, int T,
+                 const float* y_in, float* y, uint16_t* y_bf16, cudaStream_t s) {
+    cudaError_t e;
     GemvLaunch L;
-    L.wl = c->wl;
-    L.entries = c->entries;
-    L.rows = c->rows;
+    L.wl = wl;
+    L.entries = entries;
+    L.rows = rows;
     L.x = x;
     L.h = c->h;
     L.y_in = y_in;
@@ -191,10 +199,39 @@ int run_ffn(moe_ctx* c, const WorkListArgs& wa, const uint16_t* x, int T, const 
     L.rmax = (T == 1) ? 1 : kMaxRows;
     L.shapes = &c->shapes;
     L.status = c->status;
+    L.pdl = c->pdl;
     FfnHookArg ha{c, s};
     e = launch_ffn(L, s, c->prof ? ffn_hook : nullptr, &ha);
-    c->launches += 3;
+    c->launches += 2;
     return cuda_status(e);
+}
+
+// Builds the work list on the device, then K3 and K4.
+int run_ffn(moe_ctx* c, const WorkListArgs& wa, const uint16_t* x, int T, const float* y_in, float* y,
+            uint16_t* y_bf16, cudaStream_t s) {
+    prof_mark(c, MOE_PROF_WORKLIST, true, s);
+    cudaError_t e = launch_build_worklist(wa, c->pdl, s);
+    prof_mark(c, MOE_PROF_WORKLIST, false, s);
+    c->launches += 1;
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    return run_ffn_list(c, c->wl, c->entries, c->rows, x, T, y_in, y, y_bf16, s);
+}
+
+DecodeWLTarget decode_target(moe_ctx* c, WorkList* wl, FfnEntry* en, FfnRow* rows, const uint8_t* slot_base,
+                             size_t stride, const uint8_t* shared_blob) {
+    DecodeWLTarget t;
+    t.wl = wl;
+    t.entries = en;
+    t.rows = rows;
+    t.slot_base = slot_base;
+    t.slot_stride = stride;
+    t.shared_blob = shared_blob;
+    t.F = c->d.d_ff;
+    t.FS = c->d.d_ff_shared;
+    t.D = c->d.d_model;
+    t.h_shared_off = c->h_shared_off;
+    t.blob_bytes = c->blob_routed;
+    return t;
 }
 
 WorkListArgs worklist_args(moe_ctx* c, int T, int K, const int32_t* pair_slot, const float* gate_w,
@@ -328,6 +365,7 @@ int moe_ctx_create(const moe_dims* dims, int device, moe_ctx** out) {
     c->d = *dims;
     c->device = device;
     c->blob_routed = blob_bytes(dims->d_model, dims->d_ff);
+    c->blob_shared = dims->d_ff_shared > 0 ? blob_bytes(dims->d_model, dims->d_ff_shared) : 0;
     const moe_dims& d = c->d;
     bool ok = cudaDeviceGetAttribute(&c->sms, cudaDevAttrMultiProcessorCount, device) == cudaSuccess;
     ok = ok && cudaStreamCreateWithFlags(&c->side, cudaStreamNonBlocking) == cudaSuccess;
@@ -339,7 +377,7 @@ int moe_ctx_create(const moe_dims* dims, int device, moe_ctx** out) {
     if (ok) std::memset(c->mbox_host, 0, sizeof(PlanMailbox));
     const int T = d.max_tokens, pairs = T * d.top_k;
     const int fmax = d.d_ff > d.d_ff_shared ? d.d_ff : d.d_ff_shared;
-    ok = ok && ffn_prepare(d.d_model, fmax, T, c->sms, &c->shapes) == cudaSuccess;
+    ok = ok && ffn_prepare(d.d_model, d.d_ff, d.d_ff_shared, d.top_k, T, c->sms, &c->shapes) == cudaSuccess;
     const int ment = max_entries(d);
     const size_t h_floats = size_t(pairs) * d.d_ff + size_t(T) * d.d_ff_shared;
     c->h_shared_off = pairs * d.d_ff;
@@ -351,6 +389,10 @@ int moe_ctx_create(const moe_dims* dims, int device, moe_ctx** out) {
     ok = ok && dalloc(&c->wl, 1) == cudaSuccess;
     ok = ok && dalloc(&c->entries, ment) == cudaSuccess;
     ok = ok && dalloc(&c->rows, size_t(T) + pairs) == cudaSuccess;
+    ok = ok && dalloc(&c->wl2, 1) == cudaSuccess;
+    ok = ok && dalloc(&c->entries2, ment) == cudaSuccess;
+    ok = ok && dalloc(&c->rows2, size_t(T) + pairs) == cudaSuccess;
+    if (const char* v = std::getenv("MOE_NO_PDL")) c->pdl = !(v[0] == '1');
     ok = ok && dalloc(&c->h, h_floats) == cudaSuccess;
     ok = ok && dalloc(&c->partials_gu, size_t(2) * grid_gu * kMaxRows * 32) == cudaSuccess;
     ok = ok && dalloc(&c->counters_gu, tiles_gu) == cudaSuccess;
@@ -437,7 +479,7 @@ int moe_router_topk(moe_ctx* c, const uint16_t* x, const int8_t* wq, const uint1
         return MOE_ERR_ARG;
     prof_mark(c, MOE_PROF_ROUTER, true, s);
     const cudaError_t e = launch_router(x, wq, ws, bias, c->d.n_experts, c->d.d_model, c->d.top_k, T, ids, gate_w,
-                                        c->status, s);
+                                        c->status, DecodeWLTarget{}, nullptr, 0, c->pdl, s);
     prof_mark(c, MOE_PROF_ROUTER, false, s);
     c->launches += 1;
     return cuda_status(e);
@@ -446,7 +488,7 @@ int moe_router_topk(moe_ctx* c, const uint16_t* x, const int8_t* wq, const uint1
 int moe_cache_reset(moe_ctx* c, moe_slot_cache* cache, cudaStream_t s) {
     if (!c || !cache || !cache->state) return MOE_ERR_ARG;
     c->launches += 1;
-    return cuda_status(launch_cache_reset(cache->state, c->d.n_experts, c->d.n_slots, s));
+    return cuda_status(launch_cache_reset(cache->state, c->d.n_experts, c->d.n_slots, c->pdl, s));
 }
 
 // Plans the call; when the host needs the plan (store or trace) waits for the
@@ -456,7 +498,8 @@ static int plan_call(moe_ctx* c, moe_slot_cache* cache, const int32_t* ids, int 
     const uint32_t seq = ++c->seq;
     prof_mark(c, MOE_PROF_PLAN, true, s);
     cudaError_t e = launch_plan(ids, T * c->d.top_k, c->d.n_experts, c->d.n_slots, cache->state, step, pair_slot,
-                                c->pair_wave, need_host ? c->mbox_dev : nullptr, seq, c->status, s);
+                                c->pair_wave, need_host ? c->mbox_dev : nullptr, seq, c->status, nullptr,
+                                DecodeWLTarget{}, DecodeWLTarget{}, c->pdl, s);
     prof_mark(c, MOE_PROF_PLAN, false, s);
     c->launches += 1;
     if (e != cudaSuccess) return MOE_ERR_CUDA;
@@ -523,9 +566,34 @@ int moe_layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache* ca
     }
     int32_t* id = ids ? ids : c->ids;
     float* gw = gate_w ? gate_w : c->gate_w;
-    int r = moe_router_topk(c, x, W->router_q, W->router_s, bias, T, id, gw, s);
-    if (r != MOE_OK) return r;
     const int K = c->d.top_k;
+    int r;
+    if (T == 1 && !cache) {
+        // one token, resident: the router writes the work list itself
+        const DecodeWLTarget t = decode_target(c, c->wl, c->entries, c->rows, W->experts, W->expert_stride,
+                                               W->shared_blob);
+        prof_mark(c, MOE_PROF_ROUTER, true, s);
+        const cudaError_t e = launch_router(x, W->router_q, W->router_s, bias, c->d.n_experts, c->d.d_model, K, 1,
+                                            id, gw, c->status, t, W->shared_blob, c->blob_shared, c->pdl, s);
+        prof_mark(c, MOE_PROF_ROUTER, false, s);
+        c->launches += 1;
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        return run_ffn_list(c, c->wl, c->entries, c->rows, x, 1, nullptr, y, y_bf16, s);
+    }
+    if (T == 1 && W->shared_blob) {
+        // one streamed token: the router also starts the shared expert's L2 prefetch
+        if (!aligned(x, 16) || !aligned(id, 4) || !aligned(gw, 4)) return MOE_ERR_ARG;
+        prof_mark(c, MOE_PROF_ROUTER, true, s);
+        const cudaError_t e = launch_router(x, W->router_q, W->router_s, bias, c->d.n_experts, c->d.d_model, K, 1,
+                                            id, gw, c->status, DecodeWLTarget{}, W->shared_blob, c->blob_shared,
+                                            c->pdl, s);
+        prof_mark(c, MOE_PROF_ROUTER, false, s);
+        c->launches += 1;
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+    } else {
+        r = moe_router_topk(c, x, W->router_q, W->router_s, bias, T, id, gw, s);
+        if (r != MOE_OK) return r;
+    }
     if (!cache) {
         // resident: expert e's blob is W->experts + e * stride, one pass
         WorkListArgs wa = worklist_args(c, T, K, id, gw, W->experts, W->expert_stride, c->d.n_experts, c->d.d_ff,
@@ -535,18 +603,37 @@ int moe_layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache* ca
     // streaming: plan, then the shared expert (queued before the host waits,
     // so it runs during the copies), then the routed experts wave by wave
     const uint32_t seq = ++c->seq;
+    // one token: the plan kernel also writes both work lists
+    const bool one = (T == 1);
+    // list A: shared expert + hits (no copy needed); list B: misses
+    const DecodeWLTarget t_sh = one ? decode_target(c, c->wl, c->entries, c->rows, cache->slots, cache->slot_stride,
+                                                    W->shared_blob)
+                                    : DecodeWLTarget{};
+    const DecodeWLTarget t_rt = one ? decode_target(c, c->wl2, c->entries2, c->rows2, cache->slots,
+                                                    cache->slot_stride, nullptr)
+                                    : DecodeWLTarget{};
     prof_mark(c, MOE_PROF_PLAN, true, s);
     cudaError_t e = launch_plan(id, T * K, c->d.n_experts, c->d.n_slots, cache->state, step, c->pair_slot,
-                                c->pair_wave, c->mbox_dev, seq, c->status, s);
+                                c->pair_wave, c->mbox_dev, seq, c->status, gw, t_sh, t_rt, c->pdl, s);
     prof_mark(c, MOE_PROF_PLAN, false, s);
     c->launches += 1;
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     if (cudaEventRecord(c->ev_plan, s) != cudaSuccess) return MOE_ERR_CUDA;
     bool have_y = false;
-    if (W->shared_blob) {
-        WorkListArgs wa = worklist_args(c, T, 0, c->pair_slot, gw, cache->slots, cache->slot_stride, c->d.n_slots,
-                                        c->d.d_ff, W->shared_blob);
-        r = run_ffn(c, wa, x, T, nullptr, y, nullptr, s);
+    if (one) {
+        // list A runs now, during the copies; without a shared expert it may be
+        // empty, so y starts from zero and both lists accumulate into it
+        if (!W->shared_blob && cudaMemsetAsync(y, 0, sizeof(float) * c->d.d_model, s) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        r = run_ffn_list(c, c->wl, c->entries, c->rows, x, 1, W->shared_blob ? nullptr : y, y, y_bf16, s);
+        if (r != MOE_OK) return r;
+        have_y = true;
+    } else if (W->shared_blob) {
+        {
+            WorkListArgs wa = worklist_args(c, T, 0, c->pair_slot, gw, cache->slots, cache->slot_stride, c->d.n_slots,
+                                            c->d.d_ff, W->shared_blob);
+            r = run_ffn(c, wa, x, T, nullptr, y, nullptr, s);
+        }
         if (r != MOE_OK) return r;
         have_y = true;
     }
@@ -555,6 +642,7 @@ int moe_layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache* ca
     const int waves = c->mbox_host->n_waves;
     uint64_t bytes = 0;
     for (int w = 0; w < waves; ++w) {
+        if (one && c->mbox_host->n_misses == 0) break;  // everything hit: list A was the whole layer
         if (cache->store) {
             // wave w's victims may be slots wave w-1 still reads: copy after it
             cudaEvent_t after = c->ev_plan;
@@ -565,11 +653,15 @@ int moe_layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache* ca
             r = fill_wave(c, cache, w, after, s, &bytes);
             if (r != MOE_OK) return r;
         }
-        WorkListArgs wa = worklist_args(c, T, K, c->pair_slot, gw, cache->slots, cache->slot_stride, c->d.n_slots,
-                                        c->d.d_ff, nullptr);
-        wa.pair_wave = c->pair_wave;
-        wa.wave = w;
-        r = run_ffn(c, wa, x, T, have_y ? y : nullptr, y, (w + 1 == waves) ? y_bf16 : nullptr, s);
+        if (one) {
+            r = run_ffn_list(c, c->wl2, c->entries2, c->rows2, x, 1, have_y ? y : nullptr, y, y_bf16, s);
+        } else {
+            WorkListArgs wa = worklist_args(c, T, K, c->pair_slot, gw, cache->slots, cache->slot_stride,
+                                            c->d.n_slots, c->d.d_ff, nullptr);
+            wa.pair_wave = c->pair_wave;
+            wa.wave = w;
+            r = run_ffn(c, wa, x, T, have_y ? y : nullptr, y, (w + 1 == waves) ? y_bf16 : nullptr, s);
+        }
         if (r != MOE_OK) return r;
         have_y = true;
     }
@@ -581,7 +673,7 @@ int moe_residual_rmsnorm(moe_ctx* c, float* r, const float* y, uint16_t* x_next,
     if (!c || !r || !y || !x_next || T < 1) return MOE_ERR_ARG;
     c->launches += 1;
     prof_mark(c, MOE_PROF_HARNESS, true, s);
-    const cudaError_t e = launch_residual_rmsnorm(r, y, x_next, T, c->d.d_model, s);
+    const cudaError_t e = launch_residual_rmsnorm(r, y, x_next, T, c->d.d_model, c->pdl, s);
     prof_mark(c, MOE_PROF_HARNESS, false, s);
     return cuda_status(e);
 }
@@ -589,7 +681,7 @@ int moe_residual_rmsnorm(moe_ctx* c, float* r, const float* y, uint16_t* x_next,
 int moe_bf16_to_f32(moe_ctx* c, const uint16_t* x, float* out, size_t n, cudaStream_t s) {
     if (!c || !x || !out) return MOE_ERR_ARG;
     c->launches += 1;
-    return cuda_status(launch_bf16_to_f32(x, out, n, s));
+    return cuda_status(launch_bf16_to_f32(x, out, n, c->pdl, s));
 }
 
 }  // extern "C"

@@ -86,12 +86,36 @@ __device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gsrc, uint3
         "l"(gsrc), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
         : "memory");
 }
+// Bulk prefetch of [p, p + bytes) into L2 (no destination, no completion to
+// wait for), spread over the calling threads: thread `i` of `n` issues pieces
+// i, i+n, ...  p 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* p, size_t bytes, int i, int n) {
+    constexpr size_t kPiece = 32768;
+    const char* c = static_cast<const char*>(p);
+    const size_t pieces = (bytes + kPiece - 1) / kPiece;
+    for (size_t k = size_t(i); k < pieces; k += size_t(n)) {
+        const size_t off = k * kPiece;
+        const uint32_t len = uint32_t(bytes - off < kPiece ? bytes - off : kPiece);
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(c + off), "r"(len) : "memory");
+    }
+}
+
 // L2 policy for weights streamed exactly once per launch.
 __device__ __forceinline__ uint64_t l2_evict_first() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
     return p;
 }
+
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while its predecessor in the stream is finishing.
+// Discipline used by every kernel here: before pdl_wait() a kernel only reads
+// immutable data (weights) or data produced two or more launches back; after
+// pdl_wait() (the predecessor has completed and its writes are visible) it may
+// read anything and write; pdl_trigger() comes after pdl_wait(), so when a
+// kernel starts, its predecessor's predecessor has completed.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // Named barrier over a subset of warps (ids 1..15; 0 is __syncthreads).
 __device__ __forceinline__ void named_sync(int id, int nthreads) {
@@ -135,6 +159,28 @@ struct WorkList {
     int T;            // tokens (rows of x and y)
     int units_per_tile_dn;  // down units per 32-row output tile
     int max_rows;     // largest n_rows of any entry
+    // entries are the shared expert's (width FS) first, then routed ones
+    // (width F): this is enough to map a unit to its entry in O(1)
+    int n_shared;     // shared entries
+    int ush_gu;       // gate/up units of one shared entry
+    int urt_gu;       // gate/up units of one routed entry
+    int ns_sh_dn;     // down slices per tile of a shared entry
+    int ns_rt_dn;     // down slices per tile of a routed entry
+    int F, FS;        // widths
+};
+
+// Where a one-token work list is written by the router or plan kernel (so no
+// separate builder launch is needed); wl == nullptr: not requested.
+struct DecodeWLTarget {
+    WorkList* wl;
+    FfnEntry* entries;
+    FfnRow* rows;
+    const uint8_t* slot_base;   // routed blob of slot s at slot_base + s*slot_stride
+    size_t slot_stride;
+    const uint8_t* shared_blob; // or null
+    int F, FS, D;
+    int h_shared_off;           // float offset of the shared row's activation
+    size_t blob_bytes;          // routed blob size (for L2 prefetch)
 };
 
 }  // namespace moe

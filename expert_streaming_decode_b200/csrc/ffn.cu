@@ -29,6 +29,7 @@
 //     32-row output tile sums y_in and every entry in list order.
 #include "common.cuh"
 #include "ffn.cuh"
+#include "launch.cuh"
 
 namespace moe {
 
@@ -47,6 +48,8 @@ struct GemvCfg<1> {  // down: KS <= 704, up to 11 groups per chunk, one per warp
     static constexpr int NSTAGES = 6;
 };
 
+constexpr int kCtaEntries = 24;  // work-list entries a CTA keeps in shared memory
+
 struct GemvArgs {
     const WorkList* wl;
     const FfnEntry* entries;
@@ -59,7 +62,7 @@ struct GemvArgs {
     float* partials;        // K3: [2*grid][kMaxRows][32]; K4: [units][kMaxRows][32]
     int* counters;          // K3: per (entry, tile); K4: per output tile
     int D;
-    int vstride;            // floats per staged input row (D for gate/up, max F for down)
+    int vstride;            // widest staged input row (D for gate/up, max F for down)
     int* status;
 };
 
@@ -78,47 +81,98 @@ __device__ __forceinline__ bool ring_wait(uint64_t* bar, uint32_t parity, int* s
     return false;
 }
 
-// Entry of global unit u (entries sorted by unit base; small linear scan from a hint).
-template <int MODE>
-__device__ __forceinline__ int find_entry(const FfnEntry* __restrict__ E, int n, int u, int hint) {
-    int e = hint;
-    while (e + 1 < n && (MODE == 0 ? E[e + 1].ubase_gu : E[e + 1].ubase_dn) <= u) ++e;
-    return e;
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {  // u8 x s8
+    int d;
+    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ uint32_t dp4a_uu(uint32_t a, uint32_t b, uint32_t c) {  // u8 x u8
+    uint32_t d;
+    asm("dp4a.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
 }
 
-// One group of 64 inputs for one lane (= one row): 8 words of nibbles from
-// the two word-quads qa, qb; accumulates A into a[m] for every token row m.
-template <int RMAX>
-__device__ __forceinline__ void group_dot(const uint4& qa, const uint4& qb, const float* __restrict__ vin, int vstride,
-                                          int k0, int nrows, float (&a0)[RMAX], float (&a1)[RMAX]) {
-    const uint32_t words[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+// Per-CTA view of the work list: the entries its unit range touches, staged
+// in shared memory (global fallback beyond kCtaEntries).
+struct EntryCache {
+    const FfnEntry* g;
+    const FfnEntry* s;
+    int e0, n_staged, n;
+    __device__ __forceinline__ const FfnEntry& at(int e) const {
+        const int i = e - e0;
+        return (i >= 0 && i < n_staged) ? s[i] : g[e];
+    }
+    template <int MODE>
+    __device__ __forceinline__ int base(int e) const {
+        return MODE == 0 ? at(e).ubase_gu : at(e).ubase_dn;
+    }
+    // entry of global unit u, scanning forward from `hint` (units ascend)
+    template <int MODE>
+    __device__ __forceinline__ int find(int u, int hint) const {
+        int e = hint;
+        while (e + 1 < n && base<MODE>(e + 1) <= u) ++e;
+        return e;
+    }
+};
+
+// Stages one input row for the integer dot products.  Per group of 64
+// inputs: s_x = max|v| / 32767 and v ~= s_x * (256*hi + lo) with hi a signed
+// byte and lo an unsigned byte (16-bit fixed point, error <= s_x/2).  The 16
+// bytes for 8 inputs k0..k0+7 hold (hi of even k, lo of even k, hi of odd k,
+// lo of odd k) as four byte-vectors, in the order the nibble extraction of the
+// weights produces (low nibbles = even k, high nibbles = odd k).  X = sum v.
+template <int MODE, int NCONS>
+__device__ __forceinline__ void stage_row(const void* src, int kin, uint4* xq, float* sx, float* X) {
+    const int tasks = kin / 8;
+    for (int base = 0; base < tasks; base += NCONS) {
+        const int i = base + int(threadIdx.x);
+        const bool ok = i < tasks;
+        float v[8];
+        if (MODE == 0) {
+            uint4 q = make_uint4(0, 0, 0, 0);
+            if (ok) q = reinterpret_cast<const uint4*>(src)[i];
+            const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const uint32_t lo = words[j] & 0x0F0F0F0Fu;
-        const uint32_t hi = (words[j] >> 4) & 0x0F0F0F0Fu;
-        // byte b of lo/hi -> 0.5 + q/256 (nibble in mantissa bits 16..19 of 0.5)
-        const float f0 = __uint_as_float(__byte_perm(lo, 0x3F000000u, 0x7044));
-        const float f1 = __uint_as_float(__byte_perm(hi, 0x3F000000u, 0x7044));
-        const float f2 = __uint_as_float(__byte_perm(lo, 0x3F000000u, 0x7144));
-        const float f3 = __uint_as_float(__byte_perm(hi, 0x3F000000u, 0x7144));
-        const float f4 = __uint_as_float(__byte_perm(lo, 0x3F000000u, 0x7244));
-        const float f5 = __uint_as_float(__byte_perm(hi, 0x3F000000u, 0x7244));
-        const float f6 = __uint_as_float(__byte_perm(lo, 0x3F000000u, 0x7344));
-        const float f7 = __uint_as_float(__byte_perm(hi, 0x3F000000u, 0x7344));
-#pragma unroll
-        for (int m = 0; m < RMAX; ++m) {
-            if (m < nrows) {
-                const float4 xa = *reinterpret_cast<const float4*>(vin + m * vstride + k0 + 8 * j);
-                const float4 xb = *reinterpret_cast<const float4*>(vin + m * vstride + k0 + 8 * j + 4);
-                a0[m] = fmaf(f0, xa.x, a0[m]);
-                a1[m] = fmaf(f1, xa.y, a1[m]);
-                a0[m] = fmaf(f2, xa.z, a0[m]);
-                a1[m] = fmaf(f3, xa.w, a1[m]);
-                a0[m] = fmaf(f4, xb.x, a0[m]);
-                a1[m] = fmaf(f5, xb.y, a1[m]);
-                a0[m] = fmaf(f6, xb.z, a0[m]);
-                a1[m] = fmaf(f7, xb.w, a1[m]);
+            for (int j = 0; j < 4; ++j) {
+                v[2 * j] = __uint_as_float(w4[j] << 16);
+                v[2 * j + 1] = __uint_as_float(w4[j] & 0xFFFF0000u);
             }
+        } else {
+            float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+            if (ok) {
+                a = reinterpret_cast<const float4*>(src)[2 * i];
+                b = reinterpret_cast<const float4*>(src)[2 * i + 1];
+            }
+            v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+            v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+        }
+        float amax = 0.f, sum = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            amax = fmaxf(amax, fabsf(v[j]));
+            sum += v[j];
+        }
+#pragma unroll
+        for (int off = 1; off < 8; off <<= 1) {  // the 8 lanes of one group
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+            sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        }
+        if (!ok) continue;
+        const float inv = amax > 0.f ? 32767.f / amax : 0.f;
+        uint32_t hi_e = 0, lo_e = 0, hi_o = 0, lo_o = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            int qv = __float2int_rn(v[j] * inv);
+            qv = max(-32767, min(32767, qv));
+            const uint32_t hb = uint32_t(qv >> 8) & 0xFFu, lb = uint32_t(qv) & 0xFFu;
+            const int sh = 8 * (j >> 1);
+            if ((j & 1) == 0) { hi_e |= hb << sh; lo_e |= lb << sh; }
+            else { hi_o |= hb << sh; lo_o |= lb << sh; }
+        }
+        xq[i] = make_uint4(hi_e, lo_e, hi_o, lo_o);
+        if ((i & 7) == 0) {
+            sx[i >> 3] = amax / 32767.f;
+            X[i >> 3] = sum;
         }
     }
 }
@@ -129,6 +183,7 @@ __global__ void __launch_bounds__((GemvCfg<MODE>::NW + 1) * 32) stream_gemv_kern
     constexpr int STAGE = GemvCfg<MODE>::STAGE;
     constexpr int kStages = GemvCfg<MODE>::NSTAGES;
     constexpr int NCONS = NW * 32;
+    pdl_wait();  // the work list and the inputs come from the preceding launches
     const int D = A.D;
     const int n_entries = A.wl->n_entries;
     const int U = MODE == 0 ? A.wl->units_gu : A.wl->units_dn;
@@ -141,13 +196,16 @@ __global__ void __launch_bounds__((GemvCfg<MODE>::NW + 1) * 32) stream_gemv_kern
     uint8_t* ring = smem;
     uint64_t* full = reinterpret_cast<uint64_t*>(ring + kStages * STAGE);
     uint64_t* empty = full + kStages;
-    float* red = reinterpret_cast<float*>(empty + kStages);      // [NW][RMAX][32]
-    const int vstride = A.vstride;                                // max input width per row
-    const int xs_stride = ((vstride / kGroup) + 3) & ~3;          // keeps vin 16-byte aligned
-    float* xsum = red + NW * RMAX * 32;                           // [RMAX][xs_stride]
-    float* vin = xsum + RMAX * xs_stride;                         // [RMAX][vstride]
-    float* yacc = vin + RMAX * vstride;                           // [T][32] (MODE 1 finalize)
-    __shared__ int s_abort;
+    FfnEntry* s_ent = reinterpret_cast<FfnEntry*>(empty + kStages);   // [kCtaEntries]
+    float* red = reinterpret_cast<float*>(s_ent + kCtaEntries);         // [NW][RMAX][32]
+    const int vstride = A.vstride;
+    const int ng_max = vstride / kGroup;
+    const int gs = (ng_max + 3) & ~3;                                    // keeps xq 16-byte aligned
+    float* sx = red + NW * RMAX * 32;                                    // [RMAX][gs]
+    float* Xs = sx + RMAX * gs;                                          // [RMAX][gs]
+    uint4* xq = reinterpret_cast<uint4*>(Xs + RMAX * gs);                // [RMAX][vstride/8]
+    float* yacc = reinterpret_cast<float*>(xq + RMAX * (vstride / 8));   // [T][32] (MODE 1 finalize)
+    __shared__ int s_abort, s_e0, s_n;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -157,20 +215,33 @@ __global__ void __launch_bounds__((GemvCfg<MODE>::NW + 1) * 32) stream_gemv_kern
             mbar_init(&empty[i], NW);
         }
         mbar_fence_init();
+        // first entry of the range: binary search on the unit bases
+        int lo = 0, hi = n_entries - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if ((MODE == 0 ? A.entries[mid].ubase_gu : A.entries[mid].ubase_dn) <= u_begin) lo = mid;
+            else hi = mid - 1;
+        }
+        s_e0 = lo;
+        s_n = min(kCtaEntries, n_entries - lo);
     }
     __syncthreads();
+    pdl_trigger();
     if (u_begin >= u_end) return;
+    for (int i = threadIdx.x; i < s_n; i += blockDim.x) s_ent[i] = A.entries[s_e0 + i];
+    __syncthreads();
+    EntryCache EC{A.entries, s_ent, s_e0, s_n, n_entries};
 
     if (warp == NW) {
         // ------------------------------------------------------ producer
         if (lane == 0) {
             const uint64_t pol = l2_evict_first();
-            int e = find_entry<MODE>(A.entries, n_entries, u_begin, 0);
+            int e = s_e0;
             int issued = 0;
             bool ok = true;
             for (int u = u_begin; u < u_end && ok; ++u, ++issued) {
-                e = find_entry<MODE>(A.entries, n_entries, u, e);
-                const FfnEntry& en = A.entries[e];
+                e = EC.find<MODE>(u, e);
+                const FfnEntry& en = EC.at(e);
                 const uint8_t* src;
                 uint32_t bytes;
                 if (MODE == 0) {
@@ -198,16 +269,16 @@ __global__ void __launch_bounds__((GemvCfg<MODE>::NW + 1) * 32) stream_gemv_kern
     float acc[RMAX];
 #pragma unroll
     for (int m = 0; m < RMAX; ++m) acc[m] = 0.f;
-    int e = -1, nrows = 0, ns = 1, ks = kGuSlice;
+    int e = -1, nrows = 0, ns = 1, ks = kGuSlice, ubase = 0;
     int seg_start = u_begin;
     for (int u = u_begin; u < u_end; ++u) {
         const int i = u - u_begin;
         const int st = i % kStages;
-        const int ne = find_entry<MODE>(A.entries, n_entries, u, e < 0 ? 0 : e);
+        const int ne = EC.find<MODE>(u, e < 0 ? s_e0 : e);
         if (ne != e) {
-            // new entry: stage its input rows (fp32) and their group sums
+            // new entry: stage its input rows as 16-bit fixed point per group
             e = ne;
-            const FfnEntry& en = A.entries[e];
+            const FfnEntry& en = EC.at(e);
             nrows = en.n_rows;
             if (nrows > RMAX) {  // more rows than this variant stages: keep in bounds, report
                 if (threadIdx.x == 0) set_status(A.status, MOE_ERR_RANGE);
@@ -215,41 +286,19 @@ __global__ void __launch_bounds__((GemvCfg<MODE>::NW + 1) * 32) stream_gemv_kern
             }
             ks = MODE == 0 ? kGuSlice : down_ks(en.F);
             ns = MODE == 0 ? D / kGuSlice : en.F / ks;
+            ubase = MODE == 0 ? en.ubase_gu : en.ubase_dn;
             const int kin = MODE == 0 ? D : en.F;
             named_sync(1, NCONS);
             for (int m = 0; m < nrows; ++m) {
                 const FfnRow r = A.rows[en.row0 + m];
-                if (MODE == 0) {
-                    const uint4* src = reinterpret_cast<const uint4*>(A.x + size_t(r.x_row) * D);
-                    for (int v = threadIdx.x; v < kin / 8; v += NCONS) {
-                        const uint4 q = src[v];
-                        const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            vin[m * vstride + 8 * v + 2 * j] = __uint_as_float(w4[j] << 16);
-                            vin[m * vstride + 8 * v + 2 * j + 1] = __uint_as_float(w4[j] & 0xFFFF0000u);
-                        }
-                    }
-                } else {
-                    const float4* src = reinterpret_cast<const float4*>(A.h + r.h_off);
-                    for (int v = threadIdx.x; v < kin / 4; v += NCONS)
-                        *reinterpret_cast<float4*>(vin + m * vstride + 4 * v) = src[v];
-                }
-            }
-            named_sync(1, NCONS);
-            for (int gi = threadIdx.x; gi < nrows * (kin / kGroup); gi += NCONS) {
-                const int m = gi / (kin / kGroup), g = gi % (kin / kGroup);
-                const float* p = vin + m * vstride + g * kGroup;
-                float s = 0.f;
-#pragma unroll 8
-                for (int k = 0; k < kGroup; ++k) s += p[k];
-                xsum[m * xs_stride + g] = s;
+                const void* src = MODE == 0 ? static_cast<const void*>(A.x + size_t(r.x_row) * D)
+                                            : static_cast<const void*>(A.h + r.h_off);
+                stage_row<MODE, NCONS>(src, kin, xq + m * (vstride / 8), sx + m * gs, Xs + m * gs);
             }
             named_sync(1, NCONS);
         }
-        const FfnEntry& en = A.entries[e];
-        const int ul = u - (MODE == 0 ? en.ubase_gu : en.ubase_dn);
-        const int tile = ul / ns, slice = ul % ns;
+        const int ul = u - ubase;
+        const int tile = ul / ns, slice = ul - tile * ns;
 
         // on a time-out the warp skips the compute but keeps every barrier, so
         // no other warp waits on it; the status word carries the error
@@ -260,17 +309,34 @@ __global__ void __launch_bounds__((GemvCfg<MODE>::NW + 1) * 32) stream_gemv_kern
             const uint4 qb = lds128(chunk + ((2 * g + 1) * 32 + lane) * 16);
             const uint32_t sbw = *reinterpret_cast<const uint32_t*>(chunk + 16 * ks + (g * 32 + lane) * 4);
             const float s = f16_to_f32(uint16_t(sbw & 0xFFFF)), b = f16_to_f32(uint16_t(sbw >> 16));
-            const int k0 = slice * ks + g * kGroup;
-            float a0[RMAX], a1[RMAX];
+            const int G64 = (slice * ks) / kGroup + g;      // global group of the input row
+            const uint32_t words[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+            int shi[RMAX], shi2[RMAX];
+            uint32_t slo[RMAX], slo2[RMAX];
 #pragma unroll
-            for (int m = 0; m < RMAX; ++m) { a0[m] = 0.f; a1[m] = 0.f; }
-            group_dot<RMAX>(qa, qb, vin, vstride, k0, nrows, a0, a1);
+            for (int m = 0; m < RMAX; ++m) { shi[m] = 0; shi2[m] = 0; slo[m] = 0; slo2[m] = 0; }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const uint32_t lo = words[j] & 0x0F0F0F0Fu;          // even inputs, one per byte
+                const uint32_t hi = (words[j] >> 4) & 0x0F0F0F0Fu;   // odd inputs
+#pragma unroll
+                for (int m = 0; m < RMAX; ++m) {
+                    if (m < nrows) {
+                        const uint4 xv = xq[m * (vstride / 8) + G64 * 8 + j];
+                        shi[m] = dp4a_us(lo, xv.x, shi[m]);
+                        slo[m] = dp4a_uu(lo, xv.y, slo[m]);
+                        shi2[m] = dp4a_us(hi, xv.z, shi2[m]);
+                        slo2[m] = dp4a_uu(hi, xv.w, slo2[m]);
+                    }
+                }
+            }
 #pragma unroll
             for (int m = 0; m < RMAX; ++m) {
                 if (m < nrows) {
-                    const float X = xsum[m * xs_stride + k0 / kGroup];
-                    const float t = fmaf(256.f, a0[m] + a1[m], -128.f * X);
-                    acc[m] = fmaf(s, t, fmaf(b, X, acc[m]));
+                    // sum_k q_k x_k over the group, exact up to x's 16-bit image
+                    const int dot = 256 * (shi[m] + shi2[m]) + int(slo[m] + slo2[m]);
+                    const float qx = float(dot) * sx[m * gs + G64];
+                    acc[m] = fmaf(s, qx, fmaf(b, Xs[m * gs + G64], acc[m]));
                 }
             }
         }
@@ -280,7 +346,7 @@ __global__ void __launch_bounds__((GemvCfg<MODE>::NW + 1) * 32) stream_gemv_kern
         // segment end: next unit is another (entry, tile), or the range ends
         bool seg_end = (u + 1 == u_end);
         if (!seg_end) {
-            const int e2 = find_entry<MODE>(A.entries, n_entries, u + 1, e);
+            const int e2 = EC.find<MODE>(u + 1, e);
             seg_end = (e2 != e) || ((ul + 1) / ns != tile);
         }
         if (!seg_end) continue;
@@ -292,13 +358,14 @@ __global__ void __launch_bounds__((GemvCfg<MODE>::NW + 1) * 32) stream_gemv_kern
 #pragma unroll
         for (int m = 0; m < RMAX; ++m) acc[m] = 0.f;
         if (warp == 0) {
+            const FfnEntry& en = EC.at(e);
             float tot[RMAX];
 #pragma unroll
             for (int m = 0; m < RMAX; ++m) {
                 tot[m] = 0.f;
                 for (int w = 0; w < NW; ++w) tot[m] += red[(w * RMAX + m) * 32 + lane];
             }
-            const int tile_u0 = (MODE == 0 ? en.ubase_gu : en.ubase_dn) + tile * ns;  // first unit of (entry, tile)
+            const int tile_u0 = ubase + tile * ns;  // first unit of (entry, tile)
             if (MODE == 0) {
                 const bool whole = (seg_start == tile_u0) && (u + 1 == tile_u0 + ns);
                 bool last = whole;
@@ -360,7 +427,7 @@ __global__ void __launch_bounds__((GemvCfg<MODE>::NW + 1) * 32) stream_gemv_kern
                         yacc[t * 32 + lane] = A.y_in ? A.y_in[size_t(t) * D + 32 * tile + lane] : 0.f;
                     __syncwarp();
                     for (int e2 = 0; e2 < n_entries; ++e2) {
-                        const FfnEntry& f = A.entries[e2];
+                        const FfnEntry& f = EC.at(e2);
                         const int ks2 = down_ks(f.F), ns2 = f.F / ks2;
                         const int base = f.ubase_dn + tile * ns2;
                         for (int s2 = 0; s2 < ns2; ++s2) {
@@ -385,26 +452,349 @@ __global__ void __launch_bounds__((GemvCfg<MODE>::NW + 1) * 32) stream_gemv_kern
     }
 }
 
+// ---------------------------------------------------------------------------
+// One-token (decode) variant.  Every entry has one row, so each CTA stages its
+// inputs once, before its first unit: the token's x (gate/up) or the h rows of
+// all entries (down).  Units are entry-major for gate/up (a segment is an
+// (entry, 16-output tile)) and tile-major for down (a segment is a 32-row
+// output tile across all entries: the CTA sums w_e * dot_e in registers), so a
+// segment split across CTAs is reconciled from at most a few per-CTA partials.
+// Units map to entries in O(1): shared entries first, then routed ones.
+struct DecodeMap {
+    int nsh, ush_gu, urt_gu, ns_sh, ns_rt, upt, F, FS, D;
+    __device__ __forceinline__ int gu_entry(int u) const {
+        const int sh = nsh * ush_gu;
+        return u < sh ? u / ush_gu : nsh + (u - sh) / urt_gu;
+    }
+    __device__ __forceinline__ int gu_base(int e) const {
+        return e < nsh ? e * ush_gu : nsh * ush_gu + (e - nsh) * urt_gu;
+    }
+    // down unit u -> (entry, tile, slice); tiles are 32 output rows
+    __device__ __forceinline__ void dn_unit(int u, int& e, int& tile, int& slice) const {
+        tile = u / upt;
+        const int o = u - tile * upt, sh = nsh * ns_sh;
+        if (o < sh) { e = o / ns_sh; slice = o - e * ns_sh; }
+        else { const int o2 = o - sh; e = nsh + o2 / ns_rt; slice = o2 - (e - nsh) * ns_rt; }
+    }
+    __device__ __forceinline__ int width(int e) const { return e < nsh ? FS : F; }
+    // first staged 8-input chunk of entry e's h row (down) and of its groups
+    __device__ __forceinline__ int stage_chunk0(int e) const {
+        return e < nsh ? e * (FS / 8) : nsh * (FS / 8) + (e - nsh) * (F / 8);
+    }
+};
+
+// One 8-input task of the fixed-point staging (see stage_row).  All 32 lanes
+// must call it (shuffles); `ok` marks lanes with a real task.
+__device__ __forceinline__ void stage_task(const float (&v)[8], bool ok, int chunk, uint4* xq, float* sx, float* X) {
+    float amax = 0.f, sum = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        amax = fmaxf(amax, fabsf(v[j]));
+        sum += v[j];
+    }
+#pragma unroll
+    for (int off = 1; off < 8; off <<= 1) {
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    }
+    if (!ok) return;
+    const float inv = amax > 0.f ? 32767.f / amax : 0.f;
+    uint32_t hi_e = 0, lo_e = 0, hi_o = 0, lo_o = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        int qv = __float2int_rn(v[j] * inv);
+        qv = max(-32767, min(32767, qv));
+        const uint32_t hb = uint32_t(qv >> 8) & 0xFFu, lb = uint32_t(qv) & 0xFFu;
+        const int sh = 8 * (j >> 1);
+        if ((j & 1) == 0) { hi_e |= hb << sh; lo_e |= lb << sh; }
+        else { hi_o |= hb << sh; lo_o |= lb << sh; }
+    }
+    xq[chunk] = make_uint4(hi_e, lo_e, hi_o, lo_o);
+    if ((chunk & 7) == 0) {
+        sx[chunk >> 3] = amax / 32767.f;
+        X[chunk >> 3] = sum;
+    }
+}
+
+template <int MODE>
+__global__ void __launch_bounds__((GemvCfg<MODE>::NW + 1) * 32) gemv_decode_kernel(GemvArgs A) {
+    constexpr int NW = GemvCfg<MODE>::NW;
+    constexpr int STAGE = GemvCfg<MODE>::STAGE;
+    constexpr int kStages = GemvCfg<MODE>::NSTAGES;
+    constexpr int NCONS = NW * 32;
+    // gate/up: the work list is the previous launch's output, so wait before
+    // reading it.  down: the work list is two launches back (written before
+    // the gate/up kernel), so weights stream while gate/up finishes; only the
+    // consumers wait, before staging h.
+    if (MODE == 0) {
+        pdl_wait();
+        pdl_trigger();
+    }
+    const WorkList W = *A.wl;
+    const int D = A.D;
+    const int U = MODE == 0 ? W.units_gu : W.units_dn;
+    const int G = gridDim.x, c = blockIdx.x;
+    const int u_begin = range_start(c, U, G), u_end = range_start(c + 1, U, G);
+    const DecodeMap M{W.n_shared, W.ush_gu, W.urt_gu, W.ns_sh_dn, W.ns_rt_dn, W.units_per_tile_dn, W.F, W.FS, D};
+    const int n_ent = min(W.n_entries, kCtaEntries);
+    const int NSg = D / kGuSlice;
+
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint8_t* ring = smem;
+    uint64_t* full = reinterpret_cast<uint64_t*>(ring + kStages * STAGE);
+    uint64_t* empty = full + kStages;
+    FfnEntry* s_ent = reinterpret_cast<FfnEntry*>(empty + kStages);     // [kCtaEntries]
+    FfnRow* s_row = reinterpret_cast<FfnRow*>(s_ent + kCtaEntries);     // [kCtaEntries]
+    float* red = reinterpret_cast<float*>(s_row + kCtaEntries);          // [NW][32]
+    const int gs = ((A.vstride / kGroup) + 3) & ~3;
+    float* sx = red + NW * 32;                                           // [gs]
+    float* Xs = sx + gs;                                                 // [gs]
+    uint4* xq = reinterpret_cast<uint4*>(Xs + gs);                       // [vstride / 8]
+    __shared__ int s_abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], NW);
+        }
+        mbar_fence_init();
+    }
+    if (threadIdx.x < n_ent) {
+        const FfnEntry en = A.entries[threadIdx.x];
+        s_ent[threadIdx.x] = en;
+        s_row[threadIdx.x] = A.rows[en.row0];
+    }
+    __syncthreads();
+    if (u_begin >= u_end) return;
+    {
+        const int need = MODE == 0 ? D : M.stage_chunk0(W.n_entries) * 8;  // staged input values
+        if (W.n_entries > kCtaEntries || W.max_rows > 1 || need > A.vstride) {  // not a one-token list
+            if (threadIdx.x == 0) set_status(A.status, MOE_ERR_STATE);
+            return;
+        }
+    }
+
+    if (warp == NW) {
+        // ------------------------------------------------------ producer
+        if (lane == 0) {
+            const uint64_t pol = l2_evict_first();
+            int issued = 0;
+            bool ok = true;
+            for (int u = u_begin; u < u_end && ok; ++u, ++issued) {
+                const uint8_t* src;
+                uint32_t bytes;
+                if (MODE == 0) {
+                    const int e = M.gu_entry(u);
+                    src = s_ent[e].blob + size_t(u - M.gu_base(e)) * (18 * kGuSlice);
+                    bytes = 18 * kGuSlice;
+                } else {
+                    int e, tile, slice;
+                    M.dn_unit(u, e, tile, slice);
+                    const int F = M.width(e), ks = down_ks(F);
+                    src = s_ent[e].blob + gu_section_bytes(D, F) + size_t(tile * (F / ks) + slice) * (18u * ks);
+                    bytes = 18u * ks;
+                }
+                const int st = issued % kStages;
+                if (issued >= kStages) ok = ring_wait(&empty[st], ((issued / kStages) - 1) & 1, A.status, &s_abort);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&full[st], bytes);
+                bulk_g2s(ring + size_t(st) * STAGE, src, bytes, &full[st], pol);
+            }
+            const int first = issued > kStages ? issued - kStages : 0;
+            for (int i = first; i < issued; ++i) mbar_wait(&full[i % kStages], (i / kStages) & 1, A.status);
+        }
+        return;
+    }
+
+    // ----------------------------------------- consumers: stage the inputs once
+    if (MODE == 1) {
+        pdl_wait();  // h is the gate/up kernel's output
+        pdl_trigger();
+    }
+    {
+        const int tasks = MODE == 0 ? D / 8 : M.stage_chunk0(W.n_entries);
+        constexpr int kBatch = 3;  // tasks per thread per round trip
+        for (int base = 0; base < tasks; base += kBatch * NCONS) {
+            float v[kBatch][8];
+#pragma unroll
+            for (int r = 0; r < kBatch; ++r) {  // all loads first: one round trip
+                const int t = base + r * NCONS + int(threadIdx.x);
+                if (t < tasks) {
+                    if (MODE == 0) {
+                        const uint4 q = reinterpret_cast<const uint4*>(A.x + size_t(s_row[0].x_row) * D)[t];
+                        const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            v[r][2 * j] = __uint_as_float(w4[j] << 16);
+                            v[r][2 * j + 1] = __uint_as_float(w4[j] & 0xFFFF0000u);
+                        }
+                    } else {
+                        const int shc = M.nsh * (M.FS / 8);
+                        const int ee = t < shc ? t / (M.FS / 8) : M.nsh + (t - shc) / (M.F / 8);
+                        const float* h = A.h + s_row[ee].h_off + 8 * (t - M.stage_chunk0(ee));
+                        const float4 a4 = reinterpret_cast<const float4*>(h)[0];
+                        const float4 b4 = reinterpret_cast<const float4*>(h)[1];
+                        v[r][0] = a4.x; v[r][1] = a4.y; v[r][2] = a4.z; v[r][3] = a4.w;
+                        v[r][4] = b4.x; v[r][5] = b4.y; v[r][6] = b4.z; v[r][7] = b4.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) v[r][j] = 0.f;
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < kBatch; ++r) {
+                const int t = base + r * NCONS + int(threadIdx.x);
+                stage_task(v[r], t < tasks, t, xq, sx, Xs);
+            }
+        }
+        named_sync(1, NCONS);
+    }
+
+    // -------------------------------------------------- consumers: the units
+    float acc = 0.f;
+    int seg_start = u_begin;
+    for (int u = u_begin; u < u_end; ++u) {
+        const int i = u - u_begin, st = i % kStages;
+        int e, tile, slice, key_u0, key_len;
+        if (MODE == 0) {
+            e = M.gu_entry(u);
+            const int ul = u - M.gu_base(e);
+            tile = ul / NSg;
+            slice = ul - tile * NSg;
+            key_u0 = M.gu_base(e) + tile * NSg;
+            key_len = NSg;
+        } else {
+            M.dn_unit(u, e, tile, slice);
+            key_u0 = tile * M.upt;
+            key_len = M.upt;
+        }
+        const int ks = MODE == 0 ? kGuSlice : down_ks(M.width(e));
+        const int g_in0 = MODE == 0 ? slice * (kGuSlice / kGroup) : M.stage_chunk0(e) / 8 + slice * (ks / kGroup);
+        const float w = MODE == 0 ? 1.f : s_row[e].w;
+
+        const bool have = ring_wait(&full[st], (i / kStages) & 1, A.status, &s_abort);
+        const uint8_t* chunk = ring + size_t(st) * STAGE;
+        for (int g = warp; have && g < ks / kGroup; g += NW) {
+            const uint4 qa = lds128(chunk + ((2 * g) * 32 + lane) * 16);
+            const uint4 qb = lds128(chunk + ((2 * g + 1) * 32 + lane) * 16);
+            const uint32_t sbw = *reinterpret_cast<const uint32_t*>(chunk + 16 * ks + (g * 32 + lane) * 4);
+            const float s = f16_to_f32(uint16_t(sbw & 0xFFFF)), b = f16_to_f32(uint16_t(sbw >> 16));
+            const int gi = g_in0 + g;  // staged group of the input
+            const uint32_t words[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+            int shi = 0, shi2 = 0;
+            uint32_t slo = 0, slo2 = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const uint32_t lo = words[j] & 0x0F0F0F0Fu;
+                const uint32_t hi = (words[j] >> 4) & 0x0F0F0F0Fu;
+                const uint4 xv = xq[gi * 8 + j];
+                shi = dp4a_us(lo, xv.x, shi);
+                slo = dp4a_uu(lo, xv.y, slo);
+                shi2 = dp4a_us(hi, xv.z, shi2);
+                slo2 = dp4a_uu(hi, xv.w, slo2);
+            }
+            const int dot = 256 * (shi + shi2) + int(slo + slo2);
+            const float part = fmaf(s, float(dot) * sx[gi], b * Xs[gi]);
+            acc = fmaf(w, part, acc);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
+
+        const bool seg_end = (u + 1 == u_end) || (u + 1 == key_u0 + key_len);
+        if (!seg_end) continue;
+
+        named_sync(1, NCONS);
+        red[warp * 32 + lane] = acc;
+        named_sync(1, NCONS);
+        acc = 0.f;
+        if (warp == 0) {
+            float tot = 0.f;
+            for (int ww = 0; ww < NW; ++ww) tot += red[ww * 32 + lane];
+            const bool whole = (seg_start == key_u0) && (u + 1 == key_u0 + key_len);
+            bool last = whole;
+            const int cidx = MODE == 0 ? key_u0 / NSg : tile;
+            if (!whole) {
+                const int slot = (seg_start == u_begin) ? 0 : 1;
+                A.partials[size_t(2 * c + slot) * 32 + lane] = tot;
+                __threadfence();
+                __syncwarp();
+                int old = 0;
+                if (lane == 0) old = atomicAdd(&A.counters[cidx], u + 1 - seg_start);
+                old = __shfl_sync(0xffffffffu, old, 0);
+                last = (old + (u + 1 - seg_start) == key_len);
+                if (last) {
+                    __threadfence();
+                    // the segment's partials in CTA order (independent loads)
+                    tot = 0.f;
+                    const int c0 = cta_of(key_u0, U, G), c1 = cta_of(key_u0 + key_len - 1, U, G);
+                    for (int cc = c0; cc <= c1; ++cc) {
+                        const int rs = range_start(cc, U, G);
+                        if (rs >= range_start(cc + 1, U, G)) continue;
+                        tot += __ldcg(A.partials + size_t(2 * cc + (rs >= key_u0 ? 0 : 1)) * 32 + lane);
+                    }
+                    if (lane == 0) A.counters[cidx] = 0;
+                }
+            }
+            if (last) {
+                if (MODE == 0) {
+                    // lanes 0..15 gate rows, 16..31 up rows of outputs 16*tile + lane
+                    const float up = __shfl_down_sync(0xffffffffu, tot, 16);
+                    if (lane < 16) A.h[s_row[e].h_off + 16 * tile + lane] = gelu_tanh(tot) * up;
+                } else {
+                    const int r = 32 * tile + lane;
+                    const float yv = (A.y_in ? A.y_in[r] : 0.f) + tot;
+                    A.y[r] = yv;
+                    if (A.y_bf16) A.y_bf16[r] = f32_to_bf16_rn(yv);
+                }
+            }
+        }
+        seg_start = u + 1;
+    }
+}
+
 // ------------------------------------------------------------ host side
 template <int MODE, int RMAX>
 static size_t gemv_smem(int vstride, int T) {
     constexpr int NW = GemvCfg<MODE>::NW;
     size_t b = size_t(GemvCfg<MODE>::NSTAGES) * GemvCfg<MODE>::STAGE + 2 * GemvCfg<MODE>::NSTAGES * sizeof(uint64_t);
+    b += sizeof(FfnEntry) * kCtaEntries;             // staged work-list entries
     b += size_t(NW) * RMAX * 32 * 4;                 // red
-    b += size_t(RMAX) * (((vstride / kGroup) + 3) & ~3) * 4;  // xsum
-    b += size_t(RMAX) * vstride * 4;                 // vin
+    b += size_t(RMAX) * (((vstride / kGroup) + 3) & ~3) * 4 * 2;  // per-group scale and sum
+    b += size_t(RMAX) * vstride * 2;                 // 16-bit fixed-point image of the inputs
     if (MODE == 1) b += size_t(T) * 32 * 4;          // yacc
     return b;
 }
 
-template <int MODE, int RMAX>
-static cudaError_t prepare_one(int vstride, int T, int sms, GemvShape* out) {
-    const size_t smem = gemv_smem<MODE, RMAX>(vstride, T);
-    auto kern = stream_gemv_kernel<MODE, RMAX>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+// Decode kernel: entries + their rows, red, per-group scale/sum, staged image.
+template <int MODE>
+static size_t decode_smem(int vstride) {
+    constexpr int NW = GemvCfg<MODE>::NW;
+    size_t b = size_t(GemvCfg<MODE>::NSTAGES) * GemvCfg<MODE>::STAGE + 2 * GemvCfg<MODE>::NSTAGES * sizeof(uint64_t);
+    b += (sizeof(FfnEntry) + sizeof(FfnRow)) * kCtaEntries;
+    b += size_t(NW) * 32 * 4;
+    b += size_t(((vstride / kGroup) + 3) & ~3) * 4 * 2;
+    b += size_t(vstride) * 2;
+    return b;
+}
+
+template <typename K>
+static cudaError_t shape_of(K kern, int threads, size_t smem, int sms, bool raise_only, GemvShape* out) {
+    cudaError_t e;
+    if (raise_only) {
+        cudaFuncAttributes fa;
+        e = cudaFuncGetAttributes(&fa, kern);
+        if (e != cudaSuccess) return e;
+        if (size_t(fa.maxDynamicSharedSizeBytes) < smem)
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    } else {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    }
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, (GemvCfg<MODE>::NW + 1) * 32, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     out->grid = sms * per_sm;
@@ -412,56 +802,46 @@ static cudaError_t prepare_one(int vstride, int T, int sms, GemvShape* out) {
     return cudaSuccess;
 }
 
-cudaError_t ffn_prepare(int D, int Fmax, int T, int sms, GemvShapes* shapes) {
+cudaError_t ffn_prepare(int D, int F, int FS, int K, int T, int sms, GemvShapes* shapes) {
     cudaError_t e;
-    const int vdn = ((Fmax + kGroup - 1) / kGroup) * kGroup;
+    const int fmax = F > FS ? F : FS;
+    const int vdn = ((fmax + kGroup - 1) / kGroup) * kGroup;
     shapes->vstride_gu = D;
     shapes->vstride_dn = vdn;
-    if ((e = prepare_one<0, 1>(D, T, sms, &shapes->gu[0])) != cudaSuccess) return e;
-    if ((e = prepare_one<0, kMaxRows>(D, T, sms, &shapes->gu[1])) != cudaSuccess) return e;
-    if ((e = prepare_one<1, 1>(vdn, T, sms, &shapes->dn[0])) != cudaSuccess) return e;
-    if ((e = prepare_one<1, kMaxRows>(vdn, T, sms, &shapes->dn[1])) != cudaSuccess) return e;
+    shapes->stage_dn_decode = K * F + FS;
+    if ((e = shape_of(gemv_decode_kernel<0>, (GemvCfg<0>::NW + 1) * 32, decode_smem<0>(D), sms, false,
+                      &shapes->gu[0])) != cudaSuccess)
+        return e;
+    if ((e = shape_of(stream_gemv_kernel<0, kMaxRows>, (GemvCfg<0>::NW + 1) * 32, gemv_smem<0, kMaxRows>(D, T), sms,
+                      false, &shapes->gu[1])) != cudaSuccess)
+        return e;
+    if ((e = shape_of(gemv_decode_kernel<1>, (GemvCfg<1>::NW + 1) * 32, decode_smem<1>(shapes->stage_dn_decode), sms,
+                      false, &shapes->dn[0])) != cudaSuccess)
+        return e;
+    if ((e = shape_of(stream_gemv_kernel<1, kMaxRows>, (GemvCfg<1>::NW + 1) * 32, gemv_smem<1, kMaxRows>(vdn, T), sms,
+                      false, &shapes->dn[1])) != cudaSuccess)
+        return e;
     return cudaSuccess;
 }
 
-template <int MODE>
-static cudaError_t raise_smem(size_t smem) {
-    auto kern = stream_gemv_kernel<MODE, 1>;
-    cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, kern);
-    if (e != cudaSuccess) return e;
-    if (size_t(fa.maxDynamicSharedSizeBytes) >= smem) return cudaSuccess;
-    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-}
-
-template <int MODE>
-static cudaError_t one_row_shape(int vstride, int T, int sms, GemvShape* out) {
-    const size_t smem = gemv_smem<MODE, 1>(vstride, T);
-    cudaError_t e = raise_smem<MODE>(smem);
-    if (e != cudaSuccess) return e;
-    int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, stream_gemv_kernel<MODE, 1>,
-                                                      (GemvCfg<MODE>::NW + 1) * 32, smem);
-    if (e != cudaSuccess) return e;
-    if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    out->grid = sms * per_sm;
-    out->smem = smem;
-    return cudaSuccess;
-}
-
-cudaError_t ffn_shapes_one_row(int vstride_gu, int vstride_dn, int T, int sms, GemvShapes* shapes) {
+cudaError_t ffn_shapes_one_row(int vstride_gu, int stage_dn, int T, int sms, GemvShapes* shapes) {
+    (void)T;
     *shapes = GemvShapes{};
     shapes->vstride_gu = vstride_gu;
-    shapes->vstride_dn = vstride_dn;
-    cudaError_t e = one_row_shape<0>(vstride_gu, T, sms, &shapes->gu[0]);
+    shapes->stage_dn_decode = stage_dn;
+    cudaError_t e = shape_of(gemv_decode_kernel<0>, (GemvCfg<0>::NW + 1) * 32, decode_smem<0>(vstride_gu), sms, true,
+                             &shapes->gu[0]);
     if (e != cudaSuccess) return e;
-    return one_row_shape<1>(vstride_dn, T, sms, &shapes->dn[0]);
+    return shape_of(gemv_decode_kernel<1>, (GemvCfg<1>::NW + 1) * 32, decode_smem<1>(stage_dn), sms, true,
+                    &shapes->dn[0]);
 }
 
 cudaError_t ffn_ensure_one_row_smem(const GemvShapes& shapes) {
-    cudaError_t e = raise_smem<0>(shapes.gu[0].smem);
+    GemvShape tmp;
+    const int sms = 1;
+    cudaError_t e = shape_of(gemv_decode_kernel<0>, (GemvCfg<0>::NW + 1) * 32, shapes.gu[0].smem, sms, true, &tmp);
     if (e != cudaSuccess) return e;
-    return raise_smem<1>(shapes.dn[0].smem);
+    return shape_of(gemv_decode_kernel<1>, (GemvCfg<1>::NW + 1) * 32, shapes.dn[0].smem, sms, true, &tmp);
 }
 
 cudaError_t launch_ffn(const GemvLaunch& L, cudaStream_t s, void (*hook)(void*, int), void* hook_arg) {
@@ -476,30 +856,31 @@ cudaError_t launch_ffn(const GemvLaunch& L, cudaStream_t s, void (*hook)(void*, 
     a.y_bf16 = L.y_bf16;
     a.D = L.D;
     a.status = L.status;
-    const int r = L.rmax == 1 ? 0 : 1;
+    const bool one = L.rmax == 1;
     // K3: gate/up -> h
     a.partials = L.partials_gu;
     a.counters = L.counters_gu;
     a.vstride = L.shapes->vstride_gu;
-    const GemvShape& g = L.shapes->gu[r];
+    const GemvShape& g = L.shapes->gu[one ? 0 : 1];
     if (hook) hook(hook_arg, 0);
-    if (r == 0)
-        stream_gemv_kernel<0, 1><<<g.grid, (GemvCfg<0>::NW + 1) * 32, g.smem, s>>>(a);
+    cudaError_t e;
+    if (one)
+        e = launch_kernel(gemv_decode_kernel<0>, dim3(g.grid), dim3((GemvCfg<0>::NW + 1) * 32), g.smem, s, L.pdl, 1, a);
     else
-        stream_gemv_kernel<0, kMaxRows><<<g.grid, (GemvCfg<0>::NW + 1) * 32, g.smem, s>>>(a);
-    cudaError_t e = cudaGetLastError();
+        e = launch_kernel(stream_gemv_kernel<0, kMaxRows>, dim3(g.grid), dim3((GemvCfg<0>::NW + 1) * 32), g.smem, s,
+                          L.pdl, 1, a);
     if (e != cudaSuccess) return e;
     if (hook) hook(hook_arg, 1);
     // K4: down + combine -> y
     a.partials = L.partials_dn;
     a.counters = L.counters_dn;
-    a.vstride = L.shapes->vstride_dn;
-    const GemvShape& d = L.shapes->dn[r];
-    if (r == 0)
-        stream_gemv_kernel<1, 1><<<d.grid, (GemvCfg<1>::NW + 1) * 32, d.smem, s>>>(a);
+    a.vstride = one ? L.shapes->stage_dn_decode : L.shapes->vstride_dn;
+    const GemvShape& d = L.shapes->dn[one ? 0 : 1];
+    if (one)
+        e = launch_kernel(gemv_decode_kernel<1>, dim3(d.grid), dim3((GemvCfg<1>::NW + 1) * 32), d.smem, s, L.pdl, 1, a);
     else
-        stream_gemv_kernel<1, kMaxRows><<<d.grid, (GemvCfg<1>::NW + 1) * 32, d.smem, s>>>(a);
-    e = cudaGetLastError();
+        e = launch_kernel(stream_gemv_kernel<1, kMaxRows>, dim3(d.grid), dim3((GemvCfg<1>::NW + 1) * 32), d.smem, s,
+                          L.pdl, 1, a);
     if (hook) hook(hook_arg, 2);
     return e;
 }
@@ -513,6 +894,8 @@ __global__ void __launch_bounds__(256) build_worklist_kernel(WorkListArgs a) {
     __shared__ int cnt[1024];
     __shared__ int off[1025];
     __shared__ int ent_base[1025];
+    pdl_wait();
+    pdl_trigger();
     const int np = a.T * a.K;
     for (int i = threadIdx.x; i < a.n_slot_range; i += blockDim.x) cnt[i] = 0;
     __syncthreads();
@@ -609,13 +992,19 @@ __global__ void __launch_bounds__(256) build_worklist_kernel(WorkListArgs a) {
         wl.T = a.T;
         wl.units_per_tile_dn = upt;
         wl.max_rows = maxr;
+        wl.n_shared = nsh;
+        wl.ush_gu = a.FS > 0 ? (a.FS / 16) * nsg : 1;
+        wl.urt_gu = (a.F / 16) * nsg;
+        wl.ns_sh_dn = a.FS > 0 ? a.FS / down_ks(a.FS) : 1;
+        wl.ns_rt_dn = a.F / down_ks(a.F);
+        wl.F = a.F;
+        wl.FS = a.FS;
         *a.wl = wl;
     }
 }
 
-cudaError_t launch_build_worklist(const WorkListArgs& a, cudaStream_t s) {
-    build_worklist_kernel<<<1, 256, 0, s>>>(a);
-    return cudaGetLastError();
+cudaError_t launch_build_worklist(const WorkListArgs& a, bool pdl, cudaStream_t s) {
+    return launch_kernel(build_worklist_kernel, dim3(1), dim3(256), 0, s, pdl, 1, a);
 }
 
 }  // namespace moe

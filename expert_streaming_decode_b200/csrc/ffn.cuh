@@ -9,9 +9,10 @@ struct GemvShape {
     size_t smem;    // dynamic shared memory per CTA
 };
 struct GemvShapes {
-    GemvShape gu[2];   // [0]: one token row per entry, [1]: up to kMaxRows
+    GemvShape gu[2];   // [0]: one-token decode kernel, [1]: up to kMaxRows rows per entry
     GemvShape dn[2];
     int vstride_gu, vstride_dn;
+    int stage_dn_decode;  // input values the down decode kernel stages (top_k*F + FS)
 };
 
 struct GemvLaunch {
@@ -31,6 +32,7 @@ struct GemvLaunch {
     int rmax;      // 1 when every entry has one row (T == 1), else kMaxRows
     const GemvShapes* shapes;
     int* status;
+    bool pdl = true;  // launch with programmatic dependent launch
 };
 
 struct WorkListArgs {
@@ -53,17 +55,18 @@ struct WorkListArgs {
     int* status;
 };
 
-cudaError_t ffn_prepare(int D, int Fmax, int T, int sms, GemvShapes* shapes);
-// Launch shapes of the one-row variants (shapes->gu[0], dn[0]) for inputs up
-// to vstride_gu / vstride_dn wide and T tokens, raising (never lowering) each
-// kernel's dynamic shared-memory limit; the [1] entries are left zero.
-cudaError_t ffn_shapes_one_row(int vstride_gu, int vstride_dn, int T, int sms, GemvShapes* shapes);
+cudaError_t ffn_prepare(int D, int F, int FS, int K, int T, int sms, GemvShapes* shapes);
+// Launch shapes of the one-token kernels (shapes->gu[0], dn[0]) for inputs up
+// to vstride_gu wide (gate/up) and stage_dn staged values (down: top_k*F+FS),
+// raising (never lowering) each kernel's dynamic shared-memory limit; the [1]
+// entries are left zero.
+cudaError_t ffn_shapes_one_row(int vstride_gu, int stage_dn, int T, int sms, GemvShapes* shapes);
 // Raises the one-row kernels' shared-memory limits back to what `shapes`
 // needs, should another user of the library have lowered them since.
 cudaError_t ffn_ensure_one_row_smem(const GemvShapes& shapes);
 // Launches K3 (gate/up) then K4 (down); `between` (may be null) is called
 // after K3's launch and `after` after K4's (used for timing events).
 cudaError_t launch_ffn(const GemvLaunch& L, cudaStream_t s, void (*hook)(void*, int), void* hook_arg);
-cudaError_t launch_build_worklist(const WorkListArgs& a, cudaStream_t s);
+cudaError_t launch_build_worklist(const WorkListArgs& a, bool pdl, cudaStream_t s);
 
 }  // namespace moe

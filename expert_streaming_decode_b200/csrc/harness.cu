@@ -3,12 +3,15 @@
 // so its routing) depend on layer l's output, as in the model, where the
 // routing of a layer is only known once the layers below it have run.
 #include "common.cuh"
+#include "launch.cuh"
 
 namespace moe {
 
 // r[t] += y[t];  x_next[t] = bf16(r[t] / sqrt(mean(r[t]^2) + 1e-6)).  One CTA per token.
 __global__ void __launch_bounds__(256) residual_rmsnorm_kernel(float* __restrict__ r, const float* __restrict__ y,
                                                                uint16_t* __restrict__ x_next, int D) {
+    pdl_wait();
+    pdl_trigger();
     const int t = blockIdx.x;
     float* rr = r + size_t(t) * D;
     const float* yy = y + size_t(t) * D;
@@ -29,20 +32,21 @@ __global__ void __launch_bounds__(256) residual_rmsnorm_kernel(float* __restrict
     for (int k = threadIdx.x; k < D; k += blockDim.x) x_next[size_t(t) * D + k] = f32_to_bf16_rn(rr[k] * inv);
 }
 
-cudaError_t launch_residual_rmsnorm(float* r, const float* y, uint16_t* x_next, int T, int D, cudaStream_t s) {
-    residual_rmsnorm_kernel<<<T, 256, 0, s>>>(r, y, x_next, D);
-    return cudaGetLastError();
+cudaError_t launch_residual_rmsnorm(float* r, const float* y, uint16_t* x_next, int T, int D, bool pdl,
+                                    cudaStream_t s) {
+    return launch_kernel(residual_rmsnorm_kernel, dim3(T), dim3(256), 0, s, pdl, 1, r, y, x_next, D);
 }
 
 __global__ void bf16_to_f32_kernel(const uint16_t* __restrict__ x, float* __restrict__ out, size_t n) {
+    pdl_wait();
+    pdl_trigger();
     for (size_t i = blockIdx.x * size_t(blockDim.x) + threadIdx.x; i < n; i += size_t(gridDim.x) * blockDim.x)
         out[i] = bf16_to_f32(x[i]);
 }
 
-cudaError_t launch_bf16_to_f32(const uint16_t* x, float* out, size_t n, cudaStream_t s) {
+cudaError_t launch_bf16_to_f32(const uint16_t* x, float* out, size_t n, bool pdl, cudaStream_t s) {
     const int blocks = int(n / 256 + 1 < 1024 ? n / 256 + 1 : 1024);
-    bf16_to_f32_kernel<<<blocks, 256, 0, s>>>(x, out, n);
-    return cudaGetLastError();
+    return launch_kernel(bf16_to_f32_kernel, dim3(blocks), dim3(256), 0, s, pdl, 1, x, out, n);
 }
 
 }  // namespace moe

@@ -81,7 +81,7 @@ int setup_device(int dev, DeviceState* st) {
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MOE_ERR_CUDA;
     GemvShapes sh;
-    if (ffn_shapes_one_row(kNoAllocMaxD, kNoAllocMaxF, 1, sms, &sh) != cudaSuccess) return MOE_ERR_CUDA;
+    if (ffn_shapes_one_row(kNoAllocMaxD, kNoAllocMaxK * kNoAllocMaxF, 1, sms, &sh) != cudaSuccess) return MOE_ERR_CUDA;
     const Layout L = make_layout(sh);
     if (L.total > kNoAllocScratchBytes) return MOE_ERR_STATE;  // a GPU with more SMs than the array covers
     st->base = static_cast<unsigned char*>(p);
@@ -156,7 +156,7 @@ extern "C" int moe_expert_ffn_noalloc(int d_model, int d_ff, int top_k, const ui
     wa.entries = reinterpret_cast<FfnEntry*>(b + L.entries);
     wa.rows = reinterpret_cast<FfnRow*>(b + L.rows);
     wa.status = status;
-    if (launch_build_worklist(wa, stream) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_build_worklist(wa, true, stream) != cudaSuccess) return MOE_ERR_CUDA;
 
     GemvLaunch G;
     G.wl = wa.wl;

@@ -19,6 +19,8 @@
 // mailbox for the host, published by writing `seq` last.
 #include "common.cuh"
 #include "plan.cuh"
+#include "decode_wl.cuh"
+#include "launch.cuh"
 
 namespace moe {
 
@@ -27,7 +29,7 @@ constexpr int kPlanThreads = 256;
 __global__ void __launch_bounds__(kPlanThreads) cache_plan_kernel(
     const int32_t* __restrict__ ids, int npairs, int E, int S, int32_t* __restrict__ state, uint32_t step,
     int32_t* __restrict__ pair_slot, int32_t* __restrict__ pair_wave, PlanMailbox* mailbox, uint32_t seq,
-    int* status) {
+    int* status, const float* __restrict__ gate_w, DecodeWLTarget wl_shared, DecodeWLTarget wl_routed) {
     extern __shared__ int32_t psm[];
     uint32_t* mult = reinterpret_cast<uint32_t*>(psm);   // [E] selections in this call
     uint32_t* count = mult + E;                           // [E]
@@ -37,12 +39,15 @@ __global__ void __launch_bounds__(kPlanThreads) cache_plan_kernel(
     int32_t* uslot = expert_in + S;                       // [E] slot of expert in its wave
     int32_t* uwave = uslot + E;                           // [E]
     uint8_t* inwave = reinterpret_cast<uint8_t*>(uwave + E);  // [E]
+    uint8_t* uhit = inwave + E;                           // [E] 1: the expert was resident
     __shared__ int32_t ulist[1024];
 
     uint32_t* g_count = reinterpret_cast<uint32_t*>(state);
     uint32_t* g_last = g_count + E;
     int32_t* g_slot_of = state + 2 * E;
     int32_t* g_expert_in = state + 3 * E;
+    pdl_wait();
+    pdl_trigger();
 
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         mult[e] = 0;
@@ -52,6 +57,7 @@ __global__ void __launch_bounds__(kPlanThreads) cache_plan_kernel(
         uslot[e] = -1;
         uwave[e] = -1;
         inwave[e] = 0;
+        uhit[e] = 0;
     }
     for (int s = threadIdx.x; s < S; s += blockDim.x) expert_in[s] = g_expert_in[s];
     __syncthreads();
@@ -143,6 +149,7 @@ __global__ void __launch_bounds__(kPlanThreads) cache_plan_kernel(
                 if (lane == 0) {
                     uslot[e] = slot;
                     uwave[e] = w;
+                    uhit[e] = hit ? 1 : 0;
                     if (mailbox) {
                         mailbox->expert[i] = e;
                         mailbox->slot[i] = slot;
@@ -180,6 +187,23 @@ __global__ void __launch_bounds__(kPlanThreads) cache_plan_kernel(
         g_slot_of[e] = slot_of[e];
     }
     for (int s = threadIdx.x; s < S; s += blockDim.x) g_expert_in[s] = expert_in[s];
+    // one token: the work lists of the shared phase and of the routed phase
+    if (threadIdx.x < 32 && (wl_shared.wl || wl_routed.wl) && npairs <= 32) {
+        const int lane = threadIdx.x;
+        int sl = 0;
+        float w = 0.f;
+        if (lane < npairs) {
+            int e = ids[lane];
+            if (e < 0 || e >= E) e = 0;
+            sl = uslot[e] < 0 ? 0 : uslot[e];
+            w = gate_w ? gate_w[lane] : 1.f;
+        }
+        // list A: shared expert + the selections already resident (runs while
+        // the misses are copied); list B: the misses (runs after the copies)
+        const bool hit = lane < npairs && uhit[ids[lane] < 0 || ids[lane] >= E ? 0 : ids[lane]];
+        if (wl_shared.wl) write_decode_worklist(wl_shared, npairs, sl, w, hit);
+        if (wl_routed.wl) write_decode_worklist(wl_routed, npairs, sl, w, !hit);
+    }
     if (mailbox) {
         __syncthreads();
         if (threadIdx.x == 0) {
@@ -190,24 +214,25 @@ __global__ void __launch_bounds__(kPlanThreads) cache_plan_kernel(
     }
 }
 
-size_t plan_smem_bytes(int E, int S) { return size_t(E) * 4 * 6 + size_t(S) * 4 + size_t(E) + 16; }
+size_t plan_smem_bytes(int E, int S) { return size_t(E) * 4 * 6 + size_t(S) * 4 + 2 * size_t(E) + 16; }
 
 cudaError_t launch_plan(const int32_t* ids, int npairs, int E, int S, int32_t* state, uint32_t step,
                         int32_t* pair_slot, int32_t* pair_wave, PlanMailbox* mailbox, uint32_t seq, int* status,
-                        cudaStream_t s) {
-    cache_plan_kernel<<<1, kPlanThreads, plan_smem_bytes(E, S), s>>>(ids, npairs, E, S, state, step, pair_slot,
-                                                                     pair_wave, mailbox, seq, status);
-    return cudaGetLastError();
+                        const float* gate_w, const DecodeWLTarget& wl_shared, const DecodeWLTarget& wl_routed,
+                        bool pdl, cudaStream_t s) {
+    return launch_kernel(cache_plan_kernel, dim3(1), dim3(kPlanThreads), plan_smem_bytes(E, S), s, pdl, 1, ids, npairs,
+                         E, S, state, step, pair_slot, pair_wave, mailbox, seq, status, gate_w, wl_shared, wl_routed);
 }
 
 __global__ void cache_reset_kernel(int32_t* state, int E, int S) {
+    pdl_wait();
+    pdl_trigger();
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < 3 * E + S; i += gridDim.x * blockDim.x)
         state[i] = (i < 2 * E) ? 0 : -1;
 }
 
-cudaError_t launch_cache_reset(int32_t* state, int E, int S, cudaStream_t s) {
-    cache_reset_kernel<<<4, 256, 0, s>>>(state, E, S);
-    return cudaGetLastError();
+cudaError_t launch_cache_reset(int32_t* state, int E, int S, bool pdl, cudaStream_t s) {
+    return launch_kernel(cache_reset_kernel, dim3(4), dim3(256), 0, s, pdl, 1, state, E, S);
 }
 
 }  // namespace moe

@@ -16,6 +16,8 @@
 #include <cooperative_groups.h>
 
 #include "common.cuh"
+#include "decode_wl.cuh"
+#include "launch.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -30,7 +32,7 @@ constexpr int kMaxE = 1024;
 __global__ void __launch_bounds__(kRouterThreads) router_topk_kernel(
     const uint16_t* __restrict__ x, const int8_t* __restrict__ wq, const uint16_t* __restrict__ ws,
     const float* __restrict__ bias, int E, int D, int K, int32_t* __restrict__ ids, float* __restrict__ gate_w,
-    int* status) {
+    int* status, DecodeWLTarget wlt, const uint8_t* __restrict__ pf_ptr, size_t pf_bytes) {
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = int(cluster.block_rank());
     const int t = blockIdx.y;
@@ -43,6 +45,16 @@ __global__ void __launch_bounds__(kRouterThreads) router_topk_kernel(
     float* gsum = xs + ng * (kGroup + 1); // [e_per][ng] group sums
     __shared__ float logits[kMaxE];       // rank 0 gathers all logits here
 
+    // prologue (may overlap the previous kernel): pull this CTA's router rows
+    // towards L2; they are immutable
+    (void)pf_ptr;
+    (void)pf_bytes;
+    for (int i = threadIdx.x; i < e_per * ng; i += blockDim.x) {
+        const int g = i / e_per, el = i % e_per;
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(wq + size_t(e0 + el) * D + size_t(g) * kGroup));
+    }
+    pdl_wait();
+    pdl_trigger();
     for (int k = threadIdx.x; k < D; k += blockDim.x)
         xs[(k / kGroup) * (kGroup + 1) + k % kGroup] = bf16_to_f32(x[size_t(t) * D + k]);
     __syncthreads();
@@ -92,6 +104,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_topk_kernel(
     if (nan) {
         if (lane < K) { ids[size_t(t) * K + lane] = lane; gate_w[size_t(t) * K + lane] = 1.0f / K; }
         if (lane == 0) set_status(status, MOE_ERR_NAN);
+        if (wlt.wl) write_decode_worklist(wlt, K, lane, 1.0f / K, true);
         return;
     }
     uint32_t taken = 0;  // bit j: id lane + 32*j already selected (E <= 1024)
@@ -123,25 +136,17 @@ __global__ void __launch_bounds__(kRouterThreads) router_topk_kernel(
         ids[size_t(t) * K + lane] = sel_id;
         gate_w[size_t(t) * K + lane] = ex / z;
     }
+    // one token, resident experts: the expert FFN work list (slot = expert id)
+    if (wlt.wl) write_decode_worklist(wlt, K, sel_id, ex / z, true);
 }
 
 cudaError_t launch_router(const uint16_t* x, const int8_t* wq, const uint16_t* ws, const float* bias, int E, int D,
-                          int K, int T, int32_t* ids, float* gate_w, int* status, cudaStream_t s) {
+                          int K, int T, int32_t* ids, float* gate_w, int* status, const DecodeWLTarget& wlt,
+                          const uint8_t* pf_ptr, size_t pf_bytes, bool pdl, cudaStream_t s) {
     const int ng = D / kGroup;
     const size_t smem = size_t(ng) * (kGroup + 1) * 4 + size_t(E / kRouterCtas) * ng * 4;  // < 48 KB for D <= 8192
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(kRouterCtas, T, 1);
-    cfg.blockDim = dim3(kRouterThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = kRouterCtas;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, router_topk_kernel, x, wq, ws, bias, E, D, K, ids, gate_w, status);
+    return launch_kernel(router_topk_kernel, dim3(kRouterCtas, T, 1), dim3(kRouterThreads), smem, s, pdl, kRouterCtas,
+                         x, wq, ws, bias, E, D, K, ids, gate_w, status, wlt, pf_ptr, pf_bytes);
 }
 
 }  // namespace moe
