@@ -217,6 +217,38 @@ int run_ffn(moe_ctx* c, const WorkListArgs& wa, const uint16_t* x, int T, const 
     return run_ffn_list(c, c->wl, c->entries, c->rows, x, T, y_in, y, y_bf16, s);
 }
 
+// Prefill chunk (T > 32): builds a GEMM-mode work list (entries of up to 128
+// rows) and runs the tensor-core grouped GEMM; adds into y, which the caller
+// zeroed before the first call of the layer.
+int run_gemm(moe_ctx* c, WorkListArgs wa, const uint16_t* x, int T, float* y, cudaStream_t s) {
+    wa.gemm = 1;
+    prof_mark(c, MOE_PROF_WORKLIST, true, s);
+    cudaError_t e = launch_build_worklist(wa, c->pdl, s);
+    prof_mark(c, MOE_PROF_WORKLIST, false, s);
+    c->launches += 1;
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    const int pairs = T * wa.K;
+    const int routed = (pairs < wa.n_slot_range ? pairs : wa.n_slot_range) + (pairs + 127) / 128;
+    const int shared = wa.shared_blob ? (T + 127) / 128 : 0;
+    GemmLaunch L;
+    L.wl = c->wl;
+    L.entries = c->entries;
+    L.rows = c->rows;
+    L.x = x;
+    L.h = c->h;
+    L.y = y;
+    L.D = c->d.d_model;
+    L.max_tiles_gu = (wa.K > 0 ? routed * (c->d.d_ff / 64) : 0) + shared * (c->d.d_ff_shared / 64);
+    L.max_tiles_dn = ((wa.K > 0 ? routed : 0) + shared) * (c->d.d_model / 128);
+    L.status = c->status;
+    L.pdl = c->pdl;
+    if (L.max_tiles_gu <= 0 || L.max_tiles_dn <= 0) return MOE_OK;
+    FfnHookArg ha{c, s};
+    e = launch_gemm(L, s, c->prof ? ffn_hook : nullptr, &ha);
+    c->launches += 2;
+    return cuda_status(e);
+}
+
 DecodeWLTarget decode_target(moe_ctx* c, WorkList* wl, FfnEntry* en, FfnRow* rows, const uint8_t* slot_base,
                              size_t stride, const uint8_t* shared_blob) {
     DecodeWLTarget t;
@@ -378,6 +410,7 @@ int moe_ctx_create(const moe_dims* dims, int device, moe_ctx** out) {
     const int T = d.max_tokens, pairs = T * d.top_k;
     const int fmax = d.d_ff > d.d_ff_shared ? d.d_ff : d.d_ff_shared;
     ok = ok && ffn_prepare(d.d_model, d.d_ff, d.d_ff_shared, d.top_k, T, c->sms, &c->shapes) == cudaSuccess;
+    ok = ok && gemm_prepare() == cudaSuccess;
     const int ment = max_entries(d);
     const size_t h_floats = size_t(pairs) * d.d_ff + size_t(T) * d.d_ff_shared;
     c->h_shared_off = pairs * d.d_ff;
@@ -594,11 +627,20 @@ int moe_layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache* ca
         r = moe_router_topk(c, x, W->router_q, W->router_s, bias, T, id, gw, s);
         if (r != MOE_OK) return r;
     }
+    const bool gemm = T > 32;  // a prefill chunk: tensor-core grouped GEMM
     if (!cache) {
         // resident: expert e's blob is W->experts + e * stride, one pass
         WorkListArgs wa = worklist_args(c, T, K, id, gw, W->experts, W->expert_stride, c->d.n_experts, c->d.d_ff,
                                         W->shared_blob);
-        return run_ffn(c, wa, x, T, nullptr, y, y_bf16, s);
+        if (!gemm) return run_ffn(c, wa, x, T, nullptr, y, y_bf16, s);
+        if (cudaMemsetAsync(y, 0, sizeof(float) * size_t(T) * c->d.d_model, s) != cudaSuccess) return MOE_ERR_CUDA;
+        r = run_gemm(c, wa, x, T, y, s);
+        if (r != MOE_OK) return r;
+        if (y_bf16) {
+            c->launches += 1;
+            return cuda_status(launch_f32_to_bf16(y, y_bf16, size_t(T) * c->d.d_model, c->pdl, s));
+        }
+        return MOE_OK;
     }
     // streaming: plan, then the shared expert (queued before the host waits,
     // so it runs during the copies), then the routed experts wave by wave
@@ -628,6 +670,16 @@ int moe_layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache* ca
         r = run_ffn_list(c, c->wl, c->entries, c->rows, x, 1, W->shared_blob ? nullptr : y, y, y_bf16, s);
         if (r != MOE_OK) return r;
         have_y = true;
+    } else if (gemm) {
+        // prefill chunk: every contribution is added into y
+        if (cudaMemsetAsync(y, 0, sizeof(float) * size_t(T) * c->d.d_model, s) != cudaSuccess) return MOE_ERR_CUDA;
+        if (W->shared_blob) {
+            WorkListArgs wa = worklist_args(c, T, 0, c->pair_slot, gw, cache->slots, cache->slot_stride, c->d.n_slots,
+                                            c->d.d_ff, W->shared_blob);
+            r = run_gemm(c, wa, x, T, y, s);
+            if (r != MOE_OK) return r;
+        }
+        have_y = true;
     } else if (W->shared_blob) {
         {
             WorkListArgs wa = worklist_args(c, T, 0, c->pair_slot, gw, cache->slots, cache->slot_stride, c->d.n_slots,
@@ -655,6 +707,12 @@ int moe_layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache* ca
         }
         if (one) {
             r = run_ffn_list(c, c->wl2, c->entries2, c->rows2, x, 1, have_y ? y : nullptr, y, y_bf16, s);
+        } else if (gemm) {
+            WorkListArgs wa = worklist_args(c, T, K, c->pair_slot, gw, cache->slots, cache->slot_stride,
+                                            c->d.n_slots, c->d.d_ff, nullptr);
+            wa.pair_wave = c->pair_wave;
+            wa.wave = w;
+            r = run_gemm(c, wa, x, T, y, s);
         } else {
             WorkListArgs wa = worklist_args(c, T, K, c->pair_slot, gw, cache->slots, cache->slot_stride,
                                             c->d.n_slots, c->d.d_ff, nullptr);
@@ -664,6 +722,10 @@ int moe_layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache* ca
         }
         if (r != MOE_OK) return r;
         have_y = true;
+    }
+    if (gemm && y_bf16) {
+        c->launches += 1;
+        if (launch_f32_to_bf16(y, y_bf16, size_t(T) * c->d.d_model, c->pdl, s) != cudaSuccess) return MOE_ERR_CUDA;
     }
     copy_trace(c->mbox_host, trace, c->blob_routed, bytes);
     return MOE_OK;

@@ -908,14 +908,15 @@ __global__ void __launch_bounds__(256) build_worklist_kernel(WorkListArgs a) {
     }
     if (bad) set_status(a.status, MOE_ERR_RANGE);
     __syncthreads();
-    const int nsh = a.shared_blob ? (a.T + kMaxRows - 1) / kMaxRows : 0;
+    const int mr = a.gemm ? 128 : kMaxRows;  // rows per entry
+    const int nsh = a.shared_blob ? (a.T + mr - 1) / mr : 0;
     if (threadIdx.x == 0) {
         int o = a.shared_blob ? a.T : 0, eb = nsh;
         for (int sl = 0; sl < a.n_slot_range; ++sl) {
             off[sl] = o;
             ent_base[sl] = eb;
             o += cnt[sl];
-            eb += (cnt[sl] + kMaxRows - 1) / kMaxRows;
+            eb += (cnt[sl] + mr - 1) / mr;
         }
         off[a.n_slot_range] = o;
         ent_base[a.n_slot_range] = eb;
@@ -959,27 +960,27 @@ __global__ void __launch_bounds__(256) build_worklist_kernel(WorkListArgs a) {
             FfnEntry en;
             en.blob = a.shared_blob;
             en.F = a.FS;
-            en.row0 = j * kMaxRows;
-            en.n_rows = min(kMaxRows, a.T - j * kMaxRows);
+            en.row0 = j * mr;
+            en.n_rows = min(mr, a.T - j * mr);
             en.ubase_gu = ugu;
             en.ubase_dn = udn;
-            ugu += (a.FS / 16) * nsg;
-            udn += tiles_dn * (a.FS / down_ks(a.FS));
+            ugu += a.gemm ? a.FS / 64 : (a.FS / 16) * nsg;
+            udn += a.gemm ? a.D / 128 : tiles_dn * (a.FS / down_ks(a.FS));
             upt += a.FS / down_ks(a.FS);
             maxr = max(maxr, en.n_rows);
             a.entries[e] = en;
         }
         for (int sl = 0; sl < a.n_slot_range; ++sl) {
-            for (int j = 0; j * kMaxRows < cnt[sl]; ++j, ++e) {
+            for (int j = 0; j * mr < cnt[sl]; ++j, ++e) {
                 FfnEntry en;
                 en.blob = a.slot_base + size_t(sl) * a.slot_stride;
                 en.F = a.F;
-                en.row0 = off[sl] + j * kMaxRows;
-                en.n_rows = min(kMaxRows, cnt[sl] - j * kMaxRows);
+                en.row0 = off[sl] + j * mr;
+                en.n_rows = min(mr, cnt[sl] - j * mr);
                 en.ubase_gu = ugu;
                 en.ubase_dn = udn;
-                ugu += (a.F / 16) * nsg;
-                udn += tiles_dn * (a.F / down_ks(a.F));
+                ugu += a.gemm ? a.F / 64 : (a.F / 16) * nsg;
+                udn += a.gemm ? a.D / 128 : tiles_dn * (a.F / down_ks(a.F));
                 upt += a.F / down_ks(a.F);
                 maxr = max(maxr, en.n_rows);
                 a.entries[e] = en;

@@ -53,7 +53,26 @@ struct WorkListArgs {
     FfnEntry* entries;
     FfnRow* rows;
     int* status;
+    int gemm = 0;  // GEMM mode: entries carry up to 128 rows; unit bases count 128-row GEMM tiles
 };
+
+// Tensor-core grouped GEMM (gemm.cu) over a work list built in GEMM mode.
+struct GemmLaunch {
+    const WorkList* wl;
+    const FfnEntry* entries;
+    const FfnRow* rows;
+    const uint16_t* x;
+    float* h;
+    float* y;          // accumulated with atomics: zero it before the first launch
+    int D;
+    int max_tiles_gu;  // grid bounds (CTAs past the work list's tile count exit)
+    int max_tiles_dn;
+    int* status;
+    bool pdl = true;
+};
+cudaError_t gemm_prepare();
+cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, void (*hook)(void*, int), void* hook_arg);
+cudaError_t launch_f32_to_bf16(const float* y, uint16_t* out, size_t n, bool pdl, cudaStream_t s);
 
 cudaError_t ffn_prepare(int D, int F, int FS, int K, int T, int sms, GemvShapes* shapes);
 // Launch shapes of the one-token kernels (shapes->gu[0], dn[0]) for inputs up

@@ -182,3 +182,24 @@ def test_minimum_slots_equal_top_k(O):
     """S = K: every wave fills the whole cache; still bit-exact."""
     d = TINY
     _streaming(O, d, layers=1, tokens=30, S=d.K)
+
+
+@pytest.mark.parametrize("d,T", [(TINY, 40), (TINY, 128), (FULL, 37), (FULL, 128)],
+                         ids=["tiny-40", "tiny-128", "full-37", "full-128"])
+def test_prefill_resident_tensor_core(O, d, T):
+    """T > 32 runs the tcgen05 grouped GEMM (tokens grouped per expert, fp16
+    dequantised weight tiles, fp32 accumulation in tensor memory)."""
+    L = Layer(d, layer=4, seed=13, zipf_s=1.1)
+    ctx = moe.Ctx.from_dims(d, max_tokens=T)
+    xb = synth.hidden_batch(13, range(T), 4, d.D)
+    y = torch.empty((T, d.D), dtype=torch.float32, device="cuda")
+    yb = torch.empty((T, d.D), dtype=torch.int16, device="cuda")
+    ids = torch.empty((T, d.K), dtype=torch.int32, device="cuda")
+    gw = torch.empty((T, d.K), dtype=torch.float32, device="cuda")
+    moe.layer_forward(ctx, L.weights(), None, bf16_tensor(xb), T, 0, L.bias_t, y, yb, ids, gw)
+    ctx.sync()
+    ids_h, gw_h, y_h = ids.cpu().numpy(), gw.cpu().numpy(), y.cpu().numpy()
+    sample = range(T) if d is TINY else [0, 1, T // 3, T // 2, T - 1]
+    for t in sample:
+        _check_token(O, L, xb[t], ids_h[t], gw_h[t], y_h[t])
+    assert np.array_equal(yb.cpu().numpy().view(np.uint16), synth.to_bf16_bits(y_h))
