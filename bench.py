@@ -37,6 +37,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "MoE decode tokens/s (30 layers, top-8/128, 4-bit g64); HBM GB/s vs peak"
+METRIC_PREFILL = "MoE prefill tokens/s (30 layers, 128-token chunks, top-8/128, 4-bit g64, cold 16-slot caches)"
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -46,7 +47,9 @@ def parse_args():
     p.add_argument("--steps", type=int, default=240)
     p.add_argument("--warmup", type=int, default=16)
     p.add_argument("--impl", default="b200", choices=["b200", "reference"])
-    p.add_argument("--workload", default="decode_stream", choices=["decode_stream", "decode_resident", "prefill"])
+    p.add_argument("--workload", default="decode_stream",
+                   choices=["decode_stream", "decode_resident", "prefill", "sweep"])
+    p.add_argument("--sweep-tokens", type=int, default=4096)
     p.add_argument("--batch", type=int, default=1)
     p.add_argument("--slots", type=int, default=16)
     p.add_argument("--zipf", type=float, default=None,
@@ -168,7 +171,7 @@ class Model:
     routed expert blobs, either streamed (pinned host store + HBM slot
     caches) or resident in HBM."""
 
-    def __init__(self, args, dims, max_tokens, streaming):
+    def __init__(self, args, dims, max_tokens, streaming, store=None):
         import torch
 
         from expert_streaming_decode_b200 import moe, synth
@@ -188,9 +191,10 @@ class Model:
             self.bias.append(None if b is None else torch.from_numpy(b).to(dev))
             self.shared.append(torch.from_numpy(synth.expert_blob(args.seed, l, 0, dims.D, dims.FS, shared=True)).to(dev))
         t0 = time.time()
-        store = torch.empty((self.L, dims.E, self.stride), dtype=torch.uint8, pin_memory=streaming)
-        view = store.numpy()
-        synth.fill_store(view[:, :, :self.nb], args.seed, synth.Dims(**{**dims.as_dict(), "L": self.L}))
+        if store is None:
+            store = torch.empty((self.L, dims.E, self.stride), dtype=torch.uint8, pin_memory=streaming)
+            view = store.numpy()
+            synth.fill_store(view[:, :, :self.nb], args.seed, synth.Dims(**{**dims.as_dict(), "L": self.L}))
         self.gen_s = time.time() - t0
         if streaming:
             self.store = store
@@ -258,6 +262,7 @@ class Runner:
         self.y = torch.empty((T, d.D), dtype=torch.float32, device="cuda")
         self.graph = None
         self.launches_per_step = None
+        self.cold_each_step = False
         if graph:
             s = torch.cuda.Stream()
             s.wait_stream(torch.cuda.current_stream())
@@ -280,6 +285,8 @@ class Runner:
         launches = 0
         for i in range(steps):
             tok = start_tok + i
+            if self.cold_each_step:
+                m.reset()  # a prefill chunk starts from cold caches
             if host_io is not None:
                 xh, yh = host_io
                 src = xh[tok % xh.shape[0]]
@@ -429,6 +436,85 @@ def run_reference(args, dims, dist):
     return 0
 
 
+# ----------------------------------------------------------- cache sweep
+def run_sweep(args, dims, dist):
+    """Cache sweep: for every (slots, Zipf s) the router + LFU plan run over
+    --sweep-tokens decode tokens x 30 layers (seeded generator states for every
+    (token, layer)), giving hit rate and H2D bytes/token; tokens/s comes from a
+    short streamed decode (64 tokens after 16 warm-up) at the same point."""
+    import torch
+
+    from expert_streaming_decode_b200 import moe, synth
+    d = dims
+    nb = synth.blob_bytes(d.D, d.F)
+    results = []
+    routers = [synth.router_weights(args.seed, l, d.E, d.D) for l in range(args.layers)]
+    wq = [torch.from_numpy(r[0]).cuda() for r in routers]
+    ws = [torch.from_numpy(r[1].view(np.int16)).cuda() for r in routers]
+    Tn = args.sweep_tokens
+    t0 = time.time()
+    xs_all = torch.empty((Tn, args.layers, d.D), dtype=torch.int16, device="cuda")
+    for tok in range(Tn):
+        blk = np.stack([synth.hidden(args.seed, tok, l, d.D) for l in range(args.layers)])
+        xs_all[tok].copy_(torch.from_numpy(blk.view(np.int16)))
+    gen_s = time.time() - t0
+    for S in (8, 16, 32, 64):
+        for zs in (0.8, 1.1, 1.4):
+            ctx = moe.Ctx.from_dims(d, max_tokens=1, S=S)
+            bias = [torch.from_numpy(synth.zipf_bias(args.seed, l, d.E, s=zs)).cuda() for l in range(args.layers)]
+            states = [torch.empty(ctx.state_words(), dtype=torch.int32, device="cuda") for _ in range(args.layers)]
+            slots = torch.empty((S, 256), dtype=torch.uint8, device="cuda")  # plan only: never read
+            caches = []
+            for st in states:
+                c = moe.slot_cache(slots, (nb + 255) // 256 * 256, st)
+                moe.cache_reset(ctx, c)
+                caches.append(c)
+            ids = torch.empty((1, d.K), dtype=torch.int32, device="cuda")
+            gw = torch.empty((1, d.K), dtype=torch.float32, device="cuda")
+            ps = torch.empty((1, d.K), dtype=torch.int32, device="cuda")
+            tr = moe.Trace(d.E)
+            hits = misses = 0
+            t0 = time.time()
+            for tok in range(Tn):
+                for l in range(args.layers):
+                    moe.router_topk(ctx, xs_all[tok, l:l + 1], wq[l], ws[l], bias[l], 1, ids, gw)
+                    moe.cache_plan(ctx, caches[l], ids, 1, tok, ps, tr)
+                    r = tr.result()
+                    misses += r["misses"]
+                    hits += r["n_distinct"] - r["misses"]
+            ctx.sync()
+            results.append({"slots": S, "zipf_s": zs, "hit_rate": hits / max(1, hits + misses),
+                            "h2d_bytes_per_token": misses * nb / Tn, "plan_seconds": time.time() - t0})
+            ctx.close()
+    # tokens/s at each point from a short streamed decode (one store for all)
+    store = None
+    for res in results:
+        a2 = argparse.Namespace(**{**vars(args), "slots": res["slots"], "zipf": res["zipf_s"]})
+        model = Model(a2, synth.Dims(L=args.layers, S=res["slots"]), max_tokens=1, streaming=True, store=store)
+        store = model.store
+        xs = np.stack([synth.hidden_batch(args.seed + 17, [i], 0, d.D) for i in range(80)])
+        x_dev = torch.from_numpy(xs.view(np.int16)).cuda()
+        runner = Runner(model, 1, graph=False)
+        model.reset()
+        runner.run(x_dev, 16, 0)
+        ms, _ = timed(dist, model, lambda: runner.run(x_dev, 64, 16))
+        res["tokens_per_s"] = 64 / (ms * 1e-3)
+        model.ctx.close()
+        del model
+        torch.cuda.empty_cache()
+    if dist.rank == 0:
+        base = next(r for r in results if r["slots"] == 16 and abs(r["zipf_s"] - 1.1) < 1e-9)
+        line = {"metric": "MoE decode cache sweep: hit rate, H2D bytes/token, tokens/s (30 layers, 4-bit g64)",
+                "value": base["tokens_per_s"], "unit": "tokens/s", "n_gpus": dist.world, "steps": 64, "warmup": 16,
+                "ms_per_step": 1e3 / base["tokens_per_s"], "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "config": {"workload": "sweep", "layers": args.layers, "sweep_tokens": Tn,
+                           "value_point": "slots 16, zipf 1.1", "hidden_state_generation_s": gen_s},
+                "sweep": results}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 # ------------------------------------------------------------------ main
 def main():
     args = parse_args()
@@ -444,7 +530,13 @@ def main():
     import torch
     torch.cuda.set_device(dist.local)
     dist.init("nccl")
+    if args.workload == "sweep":
+        rc = run_sweep(args, dims, dist)
+        dist.close()
+        return rc
     T = args.batch if args.workload == "decode_resident" else (128 if args.workload == "prefill" else 1)
+    if args.workload == "prefill" and args.steps == 240 and args.warmup == 16:
+        args.steps, args.warmup = 4, 1  # a chunk is ~9 GB of cold fills: keep the default run short
     streaming = args.workload in ("decode_stream", "prefill")
     model = Model(args, dims, max_tokens=T, streaming=streaming)
     W, K = args.warmup, args.steps
@@ -454,6 +546,7 @@ def main():
 
     # ---- timed pass: inputs resident in HBM, no instrumentation
     runner = Runner(model, T, graph=not streaming)
+    runner.cold_each_step = args.workload == "prefill"
     model.reset()
     runner.run(x_dev, W, 0)
     clocks = ClockSampler(dist.local)
@@ -468,7 +561,8 @@ def main():
     kp = min(K, 32)
     model.reset()
     runner_p = Runner(model, T, graph=False)
-    runner_p.run(x_dev, W, 0)
+    runner_p.cold_each_step = args.workload == "prefill"
+    runner_p.run(x_dev, min(W, 2), 0)
     model.ctx.profile(True)
     acc_p = {"misses": 0, "distinct": 0, "h2d": 0}
     ms_p, _ = timed(dist, model, lambda: runner_p.run(x_dev, kp, W, trace_acc=acc_p if streaming else None))
@@ -477,7 +571,8 @@ def main():
 
     tokens_all = dist.sum(K * T)
     value = tokens_all / (ms * 1e-3)
-    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": dist.world, "steps": K, "warmup": W,
+    line = {"metric": METRIC_PREFILL if args.workload == "prefill" else METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": dist.world, "steps": K, "warmup": W,
             "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic"}
     cfg = {"workload": args.workload, "layers": args.layers, "batch": T, "slots": args.slots if streaming else None,
@@ -506,11 +601,21 @@ def main():
             kern[kind] = {"ms_total": tms, "launches": cnt}
     dom = max(("gate_up", "down"), key=lambda k: kern[k]["ms_total"])
     ach = kern[dom]["gbs"]
-    line["roofline"] = {"bound": "hbm", "kernel": f"gemv_decode_kernel ({dom})" if T == 1 else f"stream_gemv_kernel ({dom})",
+    kname = ("gemv_decode_kernel" if T == 1 else "grouped_gemm_kernel (tcgen05)" if T > 32 else "stream_gemv_kernel")
+    line["roofline"] = {"bound": "hbm", "kernel": f"{kname} ({dom})",
                         "achieved": ach, "peak": hbm_peak,
                         "unit": "GB/s", "frac": ach / hbm_peak, "traffic": None,
                         "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
                         else "fallback 6650 GB/s"}
+    if T > 32:
+        # the grouped GEMM's FLOPs: 2 * pairs * (3 * F * D) routed + 2 * T * (3 * FS * D) shared per layer
+        flop_layer = 2.0 * T * dims.K * 3 * dims.F * dims.D + 2.0 * T * 3 * dims.FS * dims.D
+        gemm_ms = kern["gate_up"]["ms_total"] + kern["down"]["ms_total"]
+        tf = flop_layer * n_layer_tok / T / (gemm_ms * 1e-3) / 1e12
+        pk = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["bf16_tflops"] if peak_kind == "measured" else 1590.0
+        line["tensor"] = {"achieved_tflops": tf, "peak_tflops": pk, "frac": tf / pk,
+                          "note": "fp16 tcgen05 MMAs (peak: measured bf16 dense, same rate as fp16); "
+                                  "per-expert rows average ~11, so the GEMM is weight-bandwidth bound"}
     line["kernels"] = kern
     line["kernels_note"] = (f"per-kernel times from a separate pass of {kp} steps with an event pair around every "
                             "kernel (serialised: no overlap between kernels)")
