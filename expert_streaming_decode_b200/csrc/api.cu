@@ -27,13 +27,20 @@
 namespace moe {
 cudaError_t launch_router(const uint16_t* x, const int8_t* wq, const uint16_t* ws, const float* bias, int E, int D,
                           int K, int T, int32_t* ids, float* gate_w, int* status, const DecodeWLTarget& wlt,
-                          const uint8_t* pf_ptr, size_t pf_bytes, bool pdl, cudaStream_t s);
+                          bool pdl, cudaStream_t s);
+size_t router_smem_bytes(int E, int D);
 cudaError_t launch_residual_rmsnorm(float* r, const float* y, uint16_t* x_next, int T, int D, bool pdl,
                                     cudaStream_t s);
 cudaError_t launch_bf16_to_f32(const uint16_t* x, float* out, size_t n, bool pdl, cudaStream_t s);
 }  // namespace moe
 
 using namespace moe;
+
+// Calls of at least this many tokens run the experts as the tcgen05 grouped
+// GEMM (tokens grouped per expert); smaller batches run the streamed GEMV.
+#ifndef MOE_GEMM_MIN_TOKENS
+#define MOE_GEMM_MIN_TOKENS 33
+#endif
 
 struct moe_ctx {
     moe_dims d;
@@ -88,7 +95,7 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA
 bool dims_ok(const moe_dims* d) {
     if (!d) return false;
     auto ff_ok = [](int F) { return F > 0 && F % 64 == 0 && (F <= 704 || F % 704 == 0); };
-    if (d->d_model <= 0 || d->d_model % 256 || d->d_model > 16384) return false;
+    if (d->d_model <= 0 || d->d_model % 256 || d->d_model > 8192) return false;  // batched GEMV stages 8 input rows in shared memory
     if (d->group != 64) return false;
     if (d->n_experts <= 0 || d->n_experts > 1024 || d->n_experts % 8) return false;
     if (d->top_k <= 0 || d->top_k > 16 || d->top_k > d->n_experts) return false;
@@ -96,6 +103,7 @@ bool dims_ok(const moe_dims* d) {
     if (d->d_ff_shared != 0 && (!ff_ok(d->d_ff_shared) || d->d_ff_shared > 3 * 704)) return false;
     if (d->n_slots < d->top_k || d->n_slots > d->n_experts) return false;
     if (d->max_tokens < 1 || d->max_tokens > 1024) return false;
+    if (router_smem_bytes(d->n_experts, d->d_model) > (200u << 10)) return false;
     return true;
 }
 
@@ -512,7 +520,7 @@ int moe_router_topk(moe_ctx* c, const uint16_t* x, const int8_t* wq, const uint1
         return MOE_ERR_ARG;
     prof_mark(c, MOE_PROF_ROUTER, true, s);
     const cudaError_t e = launch_router(x, wq, ws, bias, c->d.n_experts, c->d.d_model, c->d.top_k, T, ids, gate_w,
-                                        c->status, DecodeWLTarget{}, nullptr, 0, c->pdl, s);
+                                        c->status, DecodeWLTarget{}, c->pdl, s);
     prof_mark(c, MOE_PROF_ROUTER, false, s);
     c->launches += 1;
     return cuda_status(e);
@@ -607,27 +615,15 @@ int moe_layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache* ca
                                                W->shared_blob);
         prof_mark(c, MOE_PROF_ROUTER, true, s);
         const cudaError_t e = launch_router(x, W->router_q, W->router_s, bias, c->d.n_experts, c->d.d_model, K, 1,
-                                            id, gw, c->status, t, W->shared_blob, c->blob_shared, c->pdl, s);
+                                            id, gw, c->status, t, c->pdl, s);
         prof_mark(c, MOE_PROF_ROUTER, false, s);
         c->launches += 1;
         if (e != cudaSuccess) return MOE_ERR_CUDA;
         return run_ffn_list(c, c->wl, c->entries, c->rows, x, 1, nullptr, y, y_bf16, s);
     }
-    if (T == 1 && W->shared_blob) {
-        // one streamed token: the router also starts the shared expert's L2 prefetch
-        if (!aligned(x, 16) || !aligned(id, 4) || !aligned(gw, 4)) return MOE_ERR_ARG;
-        prof_mark(c, MOE_PROF_ROUTER, true, s);
-        const cudaError_t e = launch_router(x, W->router_q, W->router_s, bias, c->d.n_experts, c->d.d_model, K, 1,
-                                            id, gw, c->status, DecodeWLTarget{}, W->shared_blob, c->blob_shared,
-                                            c->pdl, s);
-        prof_mark(c, MOE_PROF_ROUTER, false, s);
-        c->launches += 1;
-        if (e != cudaSuccess) return MOE_ERR_CUDA;
-    } else {
-        r = moe_router_topk(c, x, W->router_q, W->router_s, bias, T, id, gw, s);
-        if (r != MOE_OK) return r;
-    }
-    const bool gemm = T > 32;  // a prefill chunk: tensor-core grouped GEMM
+    r = moe_router_topk(c, x, W->router_q, W->router_s, bias, T, id, gw, s);
+    if (r != MOE_OK) return r;
+    const bool gemm = T >= MOE_GEMM_MIN_TOKENS;  // tensor-core grouped GEMM
     if (!cache) {
         // resident: expert e's blob is W->experts + e * stride, one pass
         WorkListArgs wa = worklist_args(c, T, K, id, gw, W->experts, W->expert_stride, c->d.n_experts, c->d.d_ff,

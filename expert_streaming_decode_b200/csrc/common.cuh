@@ -100,6 +100,14 @@ __device__ __forceinline__ void bulk_prefetch_l2(const void* p, size_t bytes, in
     }
 }
 
+// L2 policy for small weights read again on every token (kept in L2 ahead of
+// the streamed expert weights).
+__device__ __forceinline__ uint64_t l2_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
 // L2 policy for weights streamed exactly once per launch.
 __device__ __forceinline__ uint64_t l2_evict_first() {
     uint64_t p;

@@ -8,29 +8,35 @@
 // GEMM: H = gelu_tanh(X W_g^T) * (X W_u^T) [M_e x F], Y = H W_d^T [M_e x D],
 // y[t] += w * Y[t] -- the one dense contraction on the path.
 //
-// B200 mapping (one CTA per (entry, 128 output rows), 4 warps):
+// B200 mapping (one CTA per (entry, 128 output rows); 4 math warps + 1 producer):
 //   * D[128 x N] = A[128 x K] * B[N x K]^T with tcgen05.mma kind::f16, M = 128
 //     weight rows, N = the entry's token rows rounded up to 16 (experts carry
 //     ~11 rows on average, so the weights sit in the M slot), fp32 accumulator
 //     in tensor memory.
-//   * K runs in groups of 64 (one quantisation group).  For each group all
-//     threads dequantise the 128 x 64 weight tile (w = s*q + b rounded to fp16)
-//     and convert the N x 64 activation tile (bf16 x or fp32 h) to fp16, both
-//     in the no-swizzle K-major core-matrix layout (8 rows x 16 bytes per core
-//     matrix; K-direction core stride 128 B, 8-row stride 1024 B); one thread
-//     issues 4 MMAs of K = 16 and commits them to an mbarrier.  Two stages:
+//   * The producer warp streams the raw 4-bit weights of the CTA's four blob
+//     tiles into a shared-memory ring with 1-D bulk copies (mbarrier
+//     transaction counts, L2 evict-first); the down GEMM starts streaming
+//     before it waits on the gate/up GEMM, since its weights do not depend on it.
+//   * K runs in groups of 64 (one quantisation group).  Per group each math
+//     thread dequantises its weight row from the ring (w = s*q + b rounded to
+//     fp16) and writes it, with its share of the N x 64 activation tile
+//     (loaded into registers one group ahead), in the no-swizzle K-major
+//     core-matrix layout (8 rows x 16 bytes per core matrix; K-direction core
+//     stride 128 B, 8-row stride 1024 B); one thread issues 4 MMAs of K = 16
+//     and commits them to an mbarrier.  The fp16 tiles are double-buffered, so
 //     the next group is prepared while the tensor core works on this one.
 //   * gate/up epilogue: warp w holds one 32-row blob tile (16 gate rows then the
 //     16 matching up rows) in its TMEM lanes: h = gelu(g) * u with one shuffle.
 //   * down epilogue: y[token][row] += w * D, fp32 atomics (entries of different
 //     experts add into the same output rows).
+#include <type_traits>
+
 #include "common.cuh"
 #include "ffn.cuh"
 #include "launch.cuh"
 
 namespace moe {
 
-constexpr int kGemmThreads = 128;
 constexpr int kGemmStageBytes = 128 * 64 * 2;  // one 128 x 64 fp16 tile
 
 struct GemmArgs {
@@ -63,31 +69,100 @@ __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
     return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-__device__ __forceinline__ bool gemm_wait(uint64_t* bar, uint32_t parity, int* status) {
-    return mbar_wait(bar, parity, status);
+// bounded wait that gives up at once once any warp of the CTA timed out
+__device__ __forceinline__ bool ring_wait_gemm(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag) {
+    if (*abort_flag) return false;
+    if (mbar_wait(bar, parity, status)) return true;
+    *abort_flag = 1;
+    return false;
+}
+
+// Raw weight stages.  A stage is GPS consecutive quantisation groups of the
+// CTA's four blob tiles; per blob tile its nibble block (GPS x 1 KB: two
+// 16-byte word-quads per row and group) and its scale/bias block (GPS x
+// 128 B) are each contiguous inside one chunk, so a stage is 8 bulk copies.
+// Ring layout: [NST stages][4 blob tiles][GPS KB nibbles | GPS x 128 B s,b].
+template <int MODE>
+struct GemmRing;
+template <>
+struct GemmRing<0> {  // gate/up: 4 groups per 256-input chunk, take 2 at a time
+    static constexpr int kGroupsPerStage = 2;
+    static constexpr int kStages = 4;
+};
+template <>
+struct GemmRing<1> {  // down: chunk widths need not be even in groups
+    static constexpr int kGroupsPerStage = 1;
+    static constexpr int kStages = 8;
+};
+template <int MODE>
+__host__ __device__ constexpr int ring_bt_bytes() { return GemmRing<MODE>::kGroupsPerStage * 1152; }
+template <int MODE>
+__host__ __device__ constexpr int ring_stage_bytes() { return 4 * ring_bt_bytes<MODE>(); }
+template <int MODE>
+constexpr size_t gemm_smem() {
+    return size_t(GemmRing<MODE>::kStages) * ring_stage_bytes<MODE>() + 4 * size_t(kGemmStageBytes) + 1024;
+}
+
+constexpr int kMathWarps = 8;               // thread = (weight row, half of the group's 64 inputs)
+constexpr int kMathThreads = kMathWarps * 32;
+constexpr int kGemmWarps = kMathWarps + 1;  // + 1 producer warp
+constexpr int kBTasks = 128 * 8 / kMathThreads;  // (row, 8-input block) tasks of the activation tile per thread
+
+// Inside every 8-input block the fp16 tiles hold the inputs in the order
+// 0,4,1,5,2,6,3,7 (A and B alike, so the contraction is unchanged): that is
+// the order in which two nibbles at a time come out of a 32-bit word below.
+__device__ __forceinline__ uint4 pack_block_perm(const float v[8]) {
+    return make_uint4(pack_half2(v[0], v[4]), pack_half2(v[1], v[5]), pack_half2(v[2], v[6]),
+                      pack_half2(v[3], v[7]));
+}
+
+// 8 weights w = s*q + b of one 32-bit word (nibble i = input i) as fp16, in the
+// block order above.  A nibble placed in the low mantissa bits of the binary16
+// 1024.0 (0x6400) reads as 1024 + q exactly; subtracting 1024 is exact; the
+// fused multiply-add rounds s*q + b once.
+__device__ __forceinline__ uint4 dequant_word(uint32_t w, uint32_t s2, uint32_t b2) {
+    uint32_t r[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t m = ((w >> (4 * i)) & 0x000F000Fu) | 0x64006400u;  // nibbles i and i+4
+        uint32_t q;
+        asm("sub.f16x2 %0, %1, %2;" : "=r"(q) : "r"(m), "r"(0x64006400u));
+        asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r[i]) : "r"(q), "r"(s2), "r"(b2));
+    }
+    return make_uint4(r[0], r[1], r[2], r[3]);
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(kGemmThreads) grouped_gemm_kernel(GemmArgs A) {
+__global__ void __launch_bounds__(kGemmWarps * 32, 2) grouped_gemm_kernel(GemmArgs A) {
+    constexpr int GPS = GemmRing<MODE>::kGroupsPerStage;
+    constexpr int NST = GemmRing<MODE>::kStages;
+    constexpr int BT_BYTES = ring_bt_bytes<MODE>();
+    constexpr int ST_BYTES = ring_stage_bytes<MODE>();
     extern __shared__ __align__(1024) uint8_t gsm[];
     uint8_t* sA = gsm;                                   // [2][128 x 64 fp16]
     uint8_t* sB = gsm + 2 * kGemmStageBytes;             // [2][128 x 64 fp16]
+    uint8_t* ring = gsm + 4 * kGemmStageBytes;           // [NST][ST_BYTES]
     __shared__ __align__(8) uint64_t mbar[2];
+    __shared__ __align__(8) uint64_t full[NST];
+    __shared__ __align__(8) uint64_t empty[NST];
     __shared__ uint32_t tbase;
     __shared__ FfnEntry s_en;
     __shared__ int s_tile;
     __shared__ FfnRow s_rows[128];
-    __shared__ int s_bad;
+    __shared__ int s_bad, s_abort;
 
-    pdl_wait();
-    pdl_trigger();
+    // gate/up: the work list is the previous launch's output; down: it is two
+    // launches back, so the weights start streaming before the wait
+    if (MODE == 0) {
+        pdl_wait();
+        pdl_trigger();
+    }
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const WorkList W = *A.wl;
     const int total = MODE == 0 ? W.units_gu : W.units_dn;
     if (int(blockIdx.x) >= total) return;
     const int D = A.D;
     if (tid == 0) {
-        // entry of this tile: entries are sorted by their first tile
         int lo = 0, hi = W.n_entries - 1;
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
@@ -97,8 +172,13 @@ __global__ void __launch_bounds__(kGemmThreads) grouped_gemm_kernel(GemmArgs A) 
         s_en = A.entries[lo];
         s_tile = int(blockIdx.x) - (MODE == 0 ? s_en.ubase_gu : s_en.ubase_dn);
         s_bad = 0;
+        s_abort = 0;
         mbar_init(&mbar[0], 1);
         mbar_init(&mbar[1], 1);
+        for (int i = 0; i < NST; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], kMathWarps);
+        }
         mbar_fence_init();
     }
     __syncthreads();
@@ -106,6 +186,46 @@ __global__ void __launch_bounds__(kGemmThreads) grouped_gemm_kernel(GemmArgs A) 
     const int tile = s_tile;
     const int M = min(en.n_rows, 128);
     const int N = (M + 15) & ~15;
+    const int F = en.F;
+    const int Kin = MODE == 0 ? D : F;
+    const int ngroups = Kin / kGroup;
+    const int ks = MODE == 0 ? kGuSlice : down_ks(F);
+    const int nsl = MODE == 0 ? D / kGuSlice : F / ks;
+    const int gpc = ks / kGroup;  // groups per chunk (a multiple of GPS)
+    const uint8_t* sec = en.blob + (MODE == 0 ? size_t(0) : gu_section_bytes(D, F));
+    const int nstages = ngroups / GPS;
+
+    if (warp == kMathWarps) {
+        // -------------------------------------------------------- producer
+        if (lane == 0) {
+            const uint64_t pol = l2_evict_first();
+            int issued = 0;
+            bool ok = true;
+            for (int si = 0; si < nstages && ok; ++si, ++issued) {
+                const int st = si % NST;
+                if (si >= NST) ok = ring_wait_gemm(&empty[st], ((si / NST) - 1) & 1, A.status, &s_abort);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&full[st], ST_BYTES);
+                uint8_t* dst = ring + size_t(st) * ST_BYTES;
+                const int g0 = si * GPS, c = g0 / gpc, gg = g0 % gpc;  // chunk and first group in it
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    const uint8_t* chunk = sec + (size_t(4 * tile + w) * nsl + c) * (18u * ks);
+                    bulk_g2s(dst + w * BT_BYTES, chunk + gg * 1024, GPS * 1024, &full[st], pol);
+                    bulk_g2s(dst + w * BT_BYTES + GPS * 1024, chunk + 16 * ks + gg * 128, GPS * 128, &full[st], pol);
+                }
+            }
+            const int first = issued > NST ? issued - NST : 0;
+            for (int i = first; i < issued; ++i) mbar_wait(&full[i % NST], (i / NST) & 1, A.status);
+        }
+        return;
+    }
+
+    // ------------------------------------------------------------ math warps
+    if (MODE == 1) {
+        pdl_wait();  // h is the gate/up GEMM's output
+        pdl_trigger();
+    }
     if (tid < M) s_rows[tid] = A.rows[en.row0 + tid];
     int ncols = 32;
     while (ncols < N) ncols <<= 1;
@@ -116,79 +236,131 @@ __global__ void __launch_bounds__(kGemmThreads) grouped_gemm_kernel(GemmArgs A) 
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-    __syncthreads();
+    named_sync(1, kMathThreads);
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = tbase;
-    // D f32, A/B f16, both K-major, N, M = 128
     const uint32_t idesc = (1u << 4) | (uint32_t(N >> 3) << 17) | (uint32_t(128 >> 4) << 24);
 
-    const int F = en.F;
-    const int Kin = MODE == 0 ? D : F;
-    const int ngroups = Kin / kGroup;
-    const int ks = MODE == 0 ? kGuSlice : down_ks(F);
-    const int nsl = MODE == 0 ? D / kGuSlice : F / ks;
-    const uint8_t* sec = en.blob + (MODE == 0 ? size_t(0) : gu_section_bytes(D, F));
-    bool ok = true;
-
-    for (int g = 0; g < ngroups; ++g) {
-        const int st = g & 1;
-        if (g >= 2 && ok) ok = gemm_wait(&mbar[st], ((g - 2) >> 1) & 1, A.status);  // stage free again
-        uint8_t* a = sA + st * kGemmStageBytes;
-        uint8_t* b = sB + st * kGemmStageBytes;
-        // A: thread tid dequantises weight row tid (blob tile 4*tile + warp, row lane)
-        {
-            const int bt = 4 * tile + warp;
-            const int s = (g * kGroup) / ks, gg = ((g * kGroup) % ks) / kGroup;
-            const uint8_t* chunk = sec + (size_t(bt) * nsl + s) * (18u * ks);
-            const uint4 qa = *reinterpret_cast<const uint4*>(chunk + ((2 * gg) * 32 + lane) * 16);
-            const uint4 qb = *reinterpret_cast<const uint4*>(chunk + ((2 * gg + 1) * 32 + lane) * 16);
-            const uint32_t sbw = *reinterpret_cast<const uint32_t*>(chunk + 16 * ks + (gg * 32 + lane) * 4);
-            const float sc = f16_to_f32(uint16_t(sbw & 0xFFFF)), bi = f16_to_f32(uint16_t(sbw >> 16));
-            const uint32_t words[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+    // Activation tile tasks: task idx = tid + kMathThreads*i covers row j,
+    // inputs 8*kb .. +7 of the group, with j = 8*(idx/64) + idx%8 and
+    // kb = (idx/8)%8: a warp's 16-byte stores then hit 8 different rows of a
+    // core matrix (no bank conflicts) and its loads still fill whole sectors.
+    // Rows M..N-1 are zero padding.  Raw loads are kept in registers and
+    // converted one group later, so their latency overlaps a whole group.
+    const int ntasks = 8 * N;
+    using Raw = typename std::conditional<MODE == 0, uint4, float4[2]>::type;
+    Raw braw[kBTasks];
+    const void* bsrc[kBTasks];  // row base of each task (nullptr: padding row)
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {  // word j = inputs 8j .. 8j+7 of the group
-                float v[8];
+    for (int i = 0; i < kBTasks; ++i) {
+        const int idx = tid + kMathThreads * i;
+        const int j = 8 * (idx >> 6) + (idx & 7);
+        bsrc[i] = nullptr;
+        if (idx < ntasks && j < M)
+            bsrc[i] = MODE == 0 ? static_cast<const void*>(A.x + size_t(s_rows[j].x_row) * D)
+                                : static_cast<const void*>(A.h + s_rows[j].h_off);
+    }
+    auto load_b = [&](int g) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] = fmaf(sc, float((words[j] >> (4 * i)) & 15u), bi);
-                *reinterpret_cast<uint4*>(a + core_off(tid, 8 * j)) =
-                    make_uint4(pack_half2(v[0], v[1]), pack_half2(v[2], v[3]), pack_half2(v[4], v[5]),
-                               pack_half2(v[6], v[7]));
-            }
-        }
-        // B: N rows x 64 inputs (rows >= M are zero)
-        for (int idx = tid; idx < N * 8; idx += kGemmThreads) {
-            const int j = idx >> 3, kb = idx & 7;
-            float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            if (j < M) {
-                const int k0 = g * kGroup + 8 * kb;
-                if (MODE == 0) {
-                    const uint4 q = *reinterpret_cast<const uint4*>(A.x + size_t(s_rows[j].x_row) * D + k0);
-                    const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        v[2 * i] = __uint_as_float(w4[i] << 16);
-                        v[2 * i + 1] = __uint_as_float(w4[i] & 0xFFFF0000u);
-                    }
+        for (int i = 0; i < kBTasks; ++i) {
+            const int idx = tid + kMathThreads * i;
+            if (idx >= ntasks) break;
+            const int k0 = g * kGroup + 8 * ((idx >> 3) & 7);
+            if (MODE == 0) {
+                uint4& q = reinterpret_cast<uint4&>(braw[i]);
+                q = bsrc[i] ? *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(bsrc[i]) + k0)
+                            : make_uint4(0, 0, 0, 0);
+            } else {
+                float4* f = reinterpret_cast<float4*>(&braw[i]);
+                if (bsrc[i]) {
+                    const float* hp = static_cast<const float*>(bsrc[i]) + k0;
+                    f[0] = *reinterpret_cast<const float4*>(hp);
+                    f[1] = *reinterpret_cast<const float4*>(hp + 4);
                 } else {
-                    const float* hp = A.h + s_rows[j].h_off + k0;
-                    const float4 p0 = *reinterpret_cast<const float4*>(hp);
-                    const float4 p1 = *reinterpret_cast<const float4*>(hp + 4);
-                    v[0] = p0.x; v[1] = p0.y; v[2] = p0.z; v[3] = p0.w;
-                    v[4] = p1.x; v[5] = p1.y; v[6] = p1.z; v[7] = p1.w;
+                    f[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    f[1] = f[0];
                 }
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    if (!(fabsf(v[i]) <= 65504.f)) { s_bad = 1; v[i] = 0.f; }  // beyond fp16 (or NaN)
             }
-            *reinterpret_cast<uint4*>(b + core_off(j, 8 * kb)) =
-                make_uint4(pack_half2(v[0], v[1]), pack_half2(v[2], v[3]), pack_half2(v[4], v[5]),
-                           pack_half2(v[6], v[7]));
         }
+    };
+    load_b(0);
+    bool ok = true;
+    // this thread's weights: row r of the 128 (blob tile 4*tile + r/32, row r%32), inputs 32*hk .. +31 of each group
+    const int r = tid & 127, hk = tid >> 7;
+    const int bt_row = r >> 5, row = r & 31;
+    // One thread waits on every barrier (the ring stage of the next group, the
+    // MMAs that last read the next group's fp16 buffers) just before the CTA
+    // barrier that ends a group, and posts "stop" if a wait timed out; the
+    // flag alternates between two words so that no thread can still be
+    // reading the word being written.
+    __shared__ int s_stop[2], s_fin;
+    if (tid == 0) {
+        s_stop[0] = ring_wait_gemm(&full[0], 0, A.status, &s_abort) ? 0 : 1;
+        s_fin = 0;
+    }
+    named_sync(1, kMathThreads);
+    int g = 0;
+    for (; g < ngroups; ++g) {
+        if (s_stop[g & 1]) break;
+        const int si = g / GPS, gl = g % GPS, st = si % NST;
+        const int buf = g & 1;
+        uint8_t* a = sA + buf * kGemmStageBytes;
+        uint8_t* b = sB + buf * kGemmStageBytes;
+        // B: this group's activations (loaded one group ahead), then the next group's loads
+#pragma unroll
+        for (int i = 0; i < kBTasks; ++i) {
+            const int idx = tid + kMathThreads * i;
+            if (idx >= ntasks) break;
+            float v[8];
+            if (MODE == 0) {
+                const uint4 q = reinterpret_cast<const uint4&>(braw[i]);
+                const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    v[2 * t] = __uint_as_float(w4[t] << 16);
+                    v[2 * t + 1] = __uint_as_float(w4[t] & 0xFFFF0000u);
+                }
+            } else {
+                const float4* f = reinterpret_cast<const float4*>(&braw[i]);
+                v[0] = f[0].x; v[1] = f[0].y; v[2] = f[0].z; v[3] = f[0].w;
+                v[4] = f[1].x; v[5] = f[1].y; v[6] = f[1].z; v[7] = f[1].w;
+            }
+#pragma unroll
+            for (int t = 0; t < 8; ++t)
+                if (!(fabsf(v[t]) <= 65504.f)) { s_bad = 1; v[t] = 0.f; }  // beyond fp16 (or NaN)
+            const int j = 8 * (idx >> 6) + (idx & 7);
+            *reinterpret_cast<uint4*>(b + core_off(j, 8 * ((idx >> 3) & 7))) = pack_block_perm(v);
+        }
+        if (g + 1 < ngroups) load_b(g + 1);
+        // A: dequantise this thread's 32 weights of the group from the raw stage
+        {
+            const uint8_t* raw = ring + size_t(st) * ST_BYTES + bt_row * BT_BYTES;
+            const uint4 q = *reinterpret_cast<const uint4*>(raw + ((2 * gl + hk) * 32 + row) * 16);
+            const uint32_t sbw = *reinterpret_cast<const uint32_t*>(raw + GPS * 1024 + (gl * 32 + row) * 4);
+            const uint32_t s2 = __byte_perm(sbw, 0, 0x1010), b2 = __byte_perm(sbw, 0, 0x3232);  // (s,s), (b,b)
+            const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j)  // word j: inputs 32*hk + 8j .. +7 of the group
+                *reinterpret_cast<uint4*>(a + core_off(r, 32 * hk + 8 * j)) = dequant_word(words[j], s2, b2);
+        }
+        __syncwarp();
+        if (gl == GPS - 1 && lane == 0) mbar_arrive(&empty[st]);  // this warp is done with the raw stage
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic writes -> tensor-core reads
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-        __syncthreads();
+        bool next_ok = true;  // thread 0 only
+        if (tid == 0) {
+            // resources of group g + 1: its ring stage, and the MMAs of group g - 1 (its fp16 buffers)
+            const int g1 = g + 1;
+            next_ok = !s_abort;
+            if (next_ok && g1 < ngroups && g1 % GPS == 0)
+                next_ok = ring_wait_gemm(&full[(g1 / GPS) % NST], ((g1 / GPS) / NST) & 1, A.status, &s_abort);
+            if (next_ok && g1 < ngroups && g >= 1)
+                next_ok = ring_wait_gemm(&mbar[(g - 1) & 1], ((g - 1) >> 1) & 1, A.status, &s_abort);
+            s_stop[g1 & 1] = next_ok ? 0 : 1;
+        }
+        named_sync(1, kMathThreads);
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        if (tid == 0 && ok) {
+        if (tid == 0 && next_ok) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
                 const uint64_t ad = umma_desc(smem_u32(a) + kk * 256);
@@ -201,20 +373,28 @@ __global__ void __launch_bounds__(kGemmThreads) grouped_gemm_kernel(GemmArgs A) 
                     : "memory");
             }
             asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                             smem_u32(&mbar[st]))
+                             smem_u32(&mbar[buf]))
                          : "memory");
         }
     }
-    // all MMAs done (a commit tracks every MMA issued before it)
-    const int last = ngroups - 1;
-    if (ok) ok = gemm_wait(&mbar[last & 1], (last >> 1) & 1, A.status);
+    // every thread left the loop at the same g; after a full pass the last
+    // group's MMAs (and with them all earlier ones) complete before the epilogue
+    const bool stopped = g < ngroups;
+    if (tid == 0 && !stopped) {
+        const int last = ngroups - 1;
+        if (!ring_wait_gemm(&mbar[last & 1], (last >> 1) & 1, A.status, &s_abort)) s_fin = 1;
+    }
+    named_sync(1, kMathThreads);
+    ok = !stopped && !s_fin;
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     if (s_bad && tid == 0) set_status(A.status, MOE_ERR_RANGE);
 
     if (ok) {
-        for (int c0 = 0; c0 < N; c0 += 16) {
+        // warp w reads TMEM lanes 32*(w%4) ..; warps 0-3 take column blocks 0, 32, ..., warps 4-7 blocks 16, 48, ...
+        const int q4 = warp & 3;
+        for (int c0 = 16 * (warp >> 2); c0 < N; c0 += 32) {
             uint32_t v[16];
-            const uint32_t ta = tmem + (uint32_t(warp * 32) << 16) + uint32_t(c0);
+            const uint32_t ta = tmem + (uint32_t(q4 * 32) << 16) + uint32_t(c0);
             asm volatile(
                 "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
@@ -228,30 +408,28 @@ __global__ void __launch_bounds__(kGemmThreads) grouped_gemm_kernel(GemmArgs A) 
                 const int j = c0 + jj;
                 const float d = __uint_as_float(v[jj]);
                 if (MODE == 0) {
-                    // warp = blob tile 4*tile + warp: lanes 0..15 gate, 16..31 up of outputs 16*bt + lane
+                    // lanes of blob tile 4*tile + q4: 0..15 gate, 16..31 up of outputs 16*bt + lane
                     const float up = __shfl_down_sync(0xffffffffu, d, 16);
                     if (lane < 16 && j < M)
-                        A.h[s_rows[j].h_off + 16 * (4 * tile + warp) + lane] = gelu_tanh(d) * up;
+                        A.h[s_rows[j].h_off + 16 * (4 * tile + q4) + lane] = gelu_tanh(d) * up;
                 } else if (j < M) {
-                    atomicAdd(&A.y[size_t(s_rows[j].y_row) * D + 128 * tile + 32 * warp + lane], s_rows[j].w * d);
+                    atomicAdd(&A.y[size_t(s_rows[j].y_row) * D + 128 * tile + 32 * q4 + lane], s_rows[j].w * d);
                 }
             }
         }
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-    __syncthreads();
+    named_sync(1, kMathThreads);
     if (warp == 0)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(ncols) : "memory");
 }
 
-size_t gemm_smem_bytes() { return size_t(4) * kGemmStageBytes; }
-
 cudaError_t gemm_prepare() {
     cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         int(gemm_smem_bytes()));
+                                         int(gemm_smem<0>()));
     if (e != cudaSuccess) return e;
     return cudaFuncSetAttribute(grouped_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                int(gemm_smem_bytes()));
+                                int(gemm_smem<1>()));
 }
 
 cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, void (*hook)(void*, int), void* hook_arg) {
@@ -265,11 +443,11 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, void (*hook)(void*,
     a.D = L.D;
     a.status = L.status;
     if (hook) hook(hook_arg, 0);
-    cudaError_t e = launch_kernel(grouped_gemm_kernel<0>, dim3(L.max_tiles_gu), dim3(kGemmThreads),
-                                  gemm_smem_bytes(), s, L.pdl, 1, a);
+    cudaError_t e = launch_kernel(grouped_gemm_kernel<0>, dim3(L.max_tiles_gu), dim3(kGemmWarps * 32),
+                                  gemm_smem<0>(), s, L.pdl, 1, a);
     if (e != cudaSuccess) return e;
     if (hook) hook(hook_arg, 1);
-    e = launch_kernel(grouped_gemm_kernel<1>, dim3(L.max_tiles_dn), dim3(kGemmThreads), gemm_smem_bytes(), s, L.pdl,
+    e = launch_kernel(grouped_gemm_kernel<1>, dim3(L.max_tiles_dn), dim3(kGemmWarps * 32), gemm_smem<1>(), s, L.pdl,
                       1, a);
     if (hook) hook(hook_arg, 2);
     return e;

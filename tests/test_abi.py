@@ -34,6 +34,10 @@ def test_ctx_create_rejects_bad_dims_without_touching_a_gpu():
     assert moe.lib.moe_ctx_create(C.byref(bad), 0, C.byref(h)) == moe.MOE_ERR_ARG
     bad = moe.moe_dims(2816, 128, 8, 704, 2112, 64, 4, 1)    # fewer slots than top_k
     assert moe.lib.moe_ctx_create(C.byref(bad), 0, C.byref(h)) == moe.MOE_ERR_ARG
+    bad = moe.moe_dims(16384, 128, 8, 704, 2112, 64, 16, 1)  # wider than the batched kernels stage
+    assert moe.lib.moe_ctx_create(C.byref(bad), 0, C.byref(h)) == moe.MOE_ERR_ARG
+    bad = moe.moe_dims(2816, 132, 8, 704, 2112, 64, 16, 1)   # experts not a multiple of the router cluster
+    assert moe.lib.moe_ctx_create(C.byref(bad), 0, C.byref(h)) == moe.MOE_ERR_ARG
     assert moe.lib.moe_ctx_create(C.byref(bad), 0, None) == moe.MOE_ERR_ARG
 
 

@@ -44,6 +44,29 @@ def test_router_ids_bit_exact(O, d, T, with_bias):
         assert np.max(np.abs(gw[t] - O.gate_weights(lg, want))) <= GATE_TOL
 
 
+@pytest.mark.parametrize("D,E", [(8192, 256), (8192, 1024)], ids=["5-passes", "19-passes"])
+def test_router_rows_in_passes(O, D, E):
+    """Router rows that do not fit shared memory at once are staged in passes
+    through two buffers (ragged last pass); ids stay bit-exact."""
+    d = synth.Dims(D=D, E=E, K=8, F=64, FS=128, G=64, L=1, S=8)
+    T = 3
+    ctx = moe.Ctx.from_dims(d, max_tokens=T)
+    wq, ws = synth.router_weights(11, 0, E, D)
+    bias = synth.zipf_bias(11, 0, E)
+    xb = synth.hidden_batch(11, range(T), 0, D)
+    ids = torch.empty((T, d.K), dtype=torch.int32, device="cuda")
+    gw = torch.empty((T, d.K), dtype=torch.float32, device="cuda")
+    moe.router_topk(ctx, bf16_tensor(xb), torch.from_numpy(wq).cuda(), torch.from_numpy(ws.view(np.int16)).cuda(),
+                    torch.from_numpy(bias).cuda(), T, ids, gw)
+    ctx.sync()
+    ids, gw = ids.cpu().numpy(), gw.cpu().numpy()
+    for t in range(T):
+        lg = O.router_logits(xb[t], wq, ws, bias, E, D, 64)
+        want = O.topk(lg, d.K)
+        assert np.array_equal(ids[t], want), (t, ids[t], want)
+        assert np.max(np.abs(gw[t] - O.gate_weights(lg, want))) <= GATE_TOL
+
+
 def test_router_ties_and_nan(O):
     d = TINY
     ctx = moe.Ctx.from_dims(d, max_tokens=4)
