@@ -601,13 +601,14 @@ def main():
             kern[kind] = {"ms_total": tms, "launches": cnt}
     dom = max(("gate_up", "down"), key=lambda k: kern[k]["ms_total"])
     ach = kern[dom]["gbs"]
-    kname = ("gemv_decode_kernel" if T == 1 else "grouped_gemm_kernel (tcgen05)" if T > 32 else "stream_gemv_kernel")
+    gemm = T >= model.moe.lib.moe_gemm_min_tokens()
+    kname = "grouped_gemm_kernel (tcgen05)" if gemm else "gemv_decode_kernel" if T == 1 else "stream_gemv_kernel"
     line["roofline"] = {"bound": "hbm", "kernel": f"{kname} ({dom})",
                         "achieved": ach, "peak": hbm_peak,
                         "unit": "GB/s", "frac": ach / hbm_peak, "traffic": None,
                         "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
                         else "fallback 6650 GB/s"}
-    if T > 32:
+    if gemm:
         # the grouped GEMM's FLOPs: 2 * pairs * (3 * F * D) routed + 2 * T * (3 * FS * D) shared per layer
         flop_layer = 2.0 * T * dims.K * 3 * dims.F * dims.D + 2.0 * T * 3 * dims.FS * dims.D
         gemm_ms = kern["gate_up"]["ms_total"] + kern["down"]["ms_total"]

@@ -15,6 +15,7 @@ namespace moe {
 
 // ------------------------------------------------------------------ limits
 constexpr int kMaxRows = 8;          // token rows one work entry carries (GEMV path)
+constexpr int kGemmMaxRows = 64;     // token rows one work entry carries (grouped GEMM: its N)
 constexpr int kGroup = 64;           // quantisation group
 constexpr int kGuSlice = 256;        // gate/up chunk inputs (KS)
 constexpr int kDownSliceMax = 704;   // down chunk inputs (KS) when F > 704

@@ -908,7 +908,7 @@ __global__ void __launch_bounds__(256) build_worklist_kernel(WorkListArgs a) {
     }
     if (bad) set_status(a.status, MOE_ERR_RANGE);
     __syncthreads();
-    const int mr = a.gemm ? 128 : kMaxRows;  // rows per entry
+    const int mr = a.gemm ? kGemmMaxRows : kMaxRows;  // rows per entry
     const int nsh = a.shared_blob ? (a.T + mr - 1) / mr : 0;
     if (threadIdx.x == 0) {
         int o = a.shared_blob ? a.T : 0, eb = nsh;
@@ -932,24 +932,37 @@ __global__ void __launch_bounds__(256) build_worklist_kernel(WorkListArgs a) {
         r.w = 1.0f;
         a.rows[t] = r;
     }
-    // routed rows: rank of pair p among the earlier pairs of its slot
-    for (int p = threadIdx.x; p < np; p += blockDim.x) {
-        if (a.pair_wave && a.pair_wave[p] != a.wave) continue;
-        int sl = a.pair_slot[p];
-        if (sl < 0 || sl >= a.n_slot_range) sl = 0;
-        int rank = 0;
-        for (int q = 0; q < p; ++q) {
-            if (a.pair_wave && a.pair_wave[q] != a.wave) continue;
-            int s2 = a.pair_slot[q];
-            if (s2 < 0 || s2 >= a.n_slot_range) s2 = 0;
-            rank += (s2 == sl);
+    // routed rows: rank of pair p among the earlier pairs of its slot.  Warp 0
+    // walks the pairs 32 at a time in order; lanes holding the same slot rank
+    // themselves by lane, after the slot's running count (cnt is reused).
+    __syncthreads();
+    for (int i = threadIdx.x; i < a.n_slot_range; i += blockDim.x) cnt[i] = 0;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        for (int base = 0; base < np; base += 32) {
+            const int p = base + lane;
+            int sl = -1;
+            if (p < np && !(a.pair_wave && a.pair_wave[p] != a.wave)) {
+                sl = a.pair_slot[p];
+                if (sl < 0 || sl >= a.n_slot_range) sl = 0;
+            }
+            const unsigned same = __match_any_sync(0xffffffffu, sl);
+            const int before = __popc(same & ((1u << lane) - 1u));
+            int rank = 0;
+            if (sl >= 0) rank = cnt[sl] + before;
+            __syncwarp();
+            if (sl >= 0 && before == 0) cnt[sl] += __popc(same);  // one lane per slot
+            __syncwarp();
+            if (sl >= 0) {
+                FfnRow r;
+                r.x_row = p / a.K;
+                r.h_off = p * a.F;
+                r.y_row = p / a.K;
+                r.w = a.gate_w[p];
+                a.rows[off[sl] + rank] = r;
+            }
         }
-        FfnRow r;
-        r.x_row = p / a.K;
-        r.h_off = p * a.F;
-        r.y_row = p / a.K;
-        r.w = a.gate_w[p];
-        a.rows[off[sl] + rank] = r;
     }
     __syncthreads();
     if (threadIdx.x == 0) {

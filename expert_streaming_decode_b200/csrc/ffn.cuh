@@ -53,7 +53,7 @@ struct WorkListArgs {
     FfnEntry* entries;
     FfnRow* rows;
     int* status;
-    int gemm = 0;  // GEMM mode: entries carry up to 128 rows; unit bases count 128-row GEMM tiles
+    int gemm = 0;  // GEMM mode: entries carry up to kGemmMaxRows rows; unit bases count 128-output GEMM tiles
 };
 
 // Tensor-core grouped GEMM (gemm.cu) over a work list built in GEMM mode.

@@ -1,32 +1,34 @@
 // gemm.cu -- K6: tcgen05 tensor-core grouped GEMM over dequantised expert
-// tiles, for the prefill chunk.
+// tiles, for batches of tokens (a batched decode step, a prefill chunk).
 //
 // Method: the prompt is prefilled in chunks of up to 128 tokens so that an
 // expert fetched once is applied to every row routed to it ("TurboFieldfare:
 // motor open source ...", section "Proceso de generacion de tokens").  With
-// the chunk's (token, k) pairs grouped by expert, each expert is a small dense
+// the call's (token, k) pairs grouped by expert, each expert is a small dense
 // GEMM: H = gelu_tanh(X W_g^T) * (X W_u^T) [M_e x F], Y = H W_d^T [M_e x D],
 // y[t] += w * Y[t] -- the one dense contraction on the path.
 //
-// B200 mapping (one CTA per (entry, 128 output rows); 4 math warps + 1 producer):
+// B200 mapping (one CTA per (entry, 128 output rows); an entry is an expert
+// and up to 64 of its token rows):
 //   * D[128 x N] = A[128 x K] * B[N x K]^T with tcgen05.mma kind::f16, M = 128
 //     weight rows, N = the entry's token rows rounded up to 16 (experts carry
-//     ~11 rows on average, so the weights sit in the M slot), fp32 accumulator
-//     in tensor memory.
-//   * The producer warp streams the raw 4-bit weights of the CTA's four blob
+//     a few rows each, so the weights sit in the M slot), fp32 accumulator in
+//     tensor memory.
+//   * A producer warp streams the raw 4-bit weights of the CTA's four blob
 //     tiles into a shared-memory ring with 1-D bulk copies (mbarrier
 //     transaction counts, L2 evict-first); the down GEMM starts streaming
 //     before it waits on the gate/up GEMM, since its weights do not depend on it.
-//   * K runs in groups of 64 (one quantisation group).  Per group each math
-//     thread dequantises its weight row from the ring (w = s*q + b rounded to
-//     fp16) and writes it, with its share of the N x 64 activation tile
-//     (loaded into registers one group ahead), in the no-swizzle K-major
-//     core-matrix layout (8 rows x 16 bytes per core matrix; K-direction core
-//     stride 128 B, 8-row stride 1024 B); one thread issues 4 MMAs of K = 16
-//     and commits them to an mbarrier.  The fp16 tiles are double-buffered, so
-//     the next group is prepared while the tensor core works on this one.
-//   * gate/up epilogue: warp w holds one 32-row blob tile (16 gate rows then the
-//     16 matching up rows) in its TMEM lanes: h = gelu(g) * u with one shuffle.
+//   * K runs in groups of 64 (one quantisation group).  Per group eight math
+//     warps dequantise the 128 x 64 weight tile from the ring (w = s*q + b
+//     rounded to fp16, two weights per half2 instruction) and write it, with
+//     the N x 64 activation tile (loaded into registers one group ahead), in
+//     the no-swizzle K-major core-matrix layout (8 rows x 16 bytes per core
+//     matrix; K-direction core stride 128 B, 8-row stride 1024 B).  An MMA
+//     warp issues 4 MMAs of K = 16 per group and commits them to an mbarrier;
+//     three fp16 buffer sets let the math warps run two groups ahead of the
+//     tensor core.
+//   * gate/up epilogue: TMEM lanes 32w..32w+31 hold one 32-row blob tile (16
+//     gate rows then the 16 matching up rows): h = gelu(g) * u with one shuffle.
 //   * down epilogue: y[token][row] += w * D, fp32 atomics (entries of different
 //     experts add into the same output rows).
 #include <type_traits>
@@ -37,7 +39,6 @@
 
 namespace moe {
 
-constexpr int kGemmStageBytes = 128 * 64 * 2;  // one 128 x 64 fp16 tile
 
 struct GemmArgs {
     const WorkList* wl;
@@ -87,26 +88,32 @@ struct GemmRing;
 template <>
 struct GemmRing<0> {  // gate/up: 4 groups per 256-input chunk, take 2 at a time
     static constexpr int kGroupsPerStage = 2;
-    static constexpr int kStages = 4;
+    static constexpr int kStages = 3;
 };
 template <>
 struct GemmRing<1> {  // down: chunk widths need not be even in groups
     static constexpr int kGroupsPerStage = 1;
-    static constexpr int kStages = 8;
+    static constexpr int kStages = 6;
 };
 template <int MODE>
 __host__ __device__ constexpr int ring_bt_bytes() { return GemmRing<MODE>::kGroupsPerStage * 1152; }
 template <int MODE>
 __host__ __device__ constexpr int ring_stage_bytes() { return 4 * ring_bt_bytes<MODE>(); }
+
+constexpr int kOpBufs = 3;                          // fp16 operand buffer sets (A and B tiles of one group)
+constexpr int kABytes = 128 * 64 * 2;               // A: 128 weight rows x 64 inputs
+constexpr int kBBytes = kGemmMaxRows * 64 * 2;      // B: up to kGemmMaxRows token rows x 64 inputs
 template <int MODE>
 constexpr size_t gemm_smem() {
-    return size_t(GemmRing<MODE>::kStages) * ring_stage_bytes<MODE>() + 4 * size_t(kGemmStageBytes) + 1024;
+    return size_t(kOpBufs) * (kABytes + kBBytes) + size_t(GemmRing<MODE>::kStages) * ring_stage_bytes<MODE>() + 128;
 }
 
 constexpr int kMathWarps = 8;               // thread = (weight row, half of the group's 64 inputs)
 constexpr int kMathThreads = kMathWarps * 32;
-constexpr int kGemmWarps = kMathWarps + 1;  // + 1 producer warp
-constexpr int kBTasks = 128 * 8 / kMathThreads;  // (row, 8-input block) tasks of the activation tile per thread
+constexpr int kProducerWarp = kMathWarps;   // bulk copies of raw weights
+constexpr int kMmaWarp = kMathWarps + 1;    // issues the tensor-core MMAs
+constexpr int kGemmWarps = kMathWarps + 2;
+constexpr int kBTasks = kGemmMaxRows * 8 / kMathThreads;  // (row, 8-input block) tasks of the B tile per thread
 
 // Inside every 8-input block the fp16 tiles hold the inputs in the order
 // 0,4,1,5,2,6,3,7 (A and B alike, so the contraction is unchanged): that is
@@ -132,23 +139,30 @@ __device__ __forceinline__ uint4 dequant_word(uint32_t w, uint32_t s2, uint32_t 
     return make_uint4(r[0], r[1], r[2], r[3]);
 }
 
+// Warp roles.  Producer warp: bulk copies of raw weight stages into the ring
+// (full/empty barriers).  Math warps: per group, wait for the ring stage and a
+// free operand buffer set, write the fp16 B tile (activations, loaded one
+// group ahead) and the dequantised A tile, arrive on `ready`.  MMA warp: per
+// group, wait for `ready`, issue 4 MMAs (K = 16 each) into the tensor-memory
+// accumulator and commit them to `freed` (the buffer set may be rewritten);
+// a last commit on `done` releases the epilogue.  No CTA-wide barrier runs
+// per group.
 template <int MODE>
 __global__ void __launch_bounds__(kGemmWarps * 32, 2) grouped_gemm_kernel(GemmArgs A) {
     constexpr int GPS = GemmRing<MODE>::kGroupsPerStage;
     constexpr int NST = GemmRing<MODE>::kStages;
     constexpr int BT_BYTES = ring_bt_bytes<MODE>();
     constexpr int ST_BYTES = ring_stage_bytes<MODE>();
-    extern __shared__ __align__(1024) uint8_t gsm[];
-    uint8_t* sA = gsm;                                   // [2][128 x 64 fp16]
-    uint8_t* sB = gsm + 2 * kGemmStageBytes;             // [2][128 x 64 fp16]
-    uint8_t* ring = gsm + 4 * kGemmStageBytes;           // [NST][ST_BYTES]
-    __shared__ __align__(8) uint64_t mbar[2];
-    __shared__ __align__(8) uint64_t full[NST];
-    __shared__ __align__(8) uint64_t empty[NST];
+    extern __shared__ __align__(128) uint8_t gsm[];
+    uint8_t* sA = gsm;                                   // [kOpBufs][128 x 64 fp16]
+    uint8_t* sB = gsm + kOpBufs * kABytes;               // [kOpBufs][kGemmMaxRows x 64 fp16]
+    uint8_t* ring = sB + kOpBufs * kBBytes;              // [NST][ST_BYTES]
+    __shared__ __align__(8) uint64_t full[NST], empty[NST];
+    __shared__ __align__(8) uint64_t ready[kOpBufs], freed[kOpBufs], done;
     __shared__ uint32_t tbase;
     __shared__ FfnEntry s_en;
     __shared__ int s_tile;
-    __shared__ FfnRow s_rows[128];
+    __shared__ FfnRow s_rows[kGemmMaxRows];
     __shared__ int s_bad, s_abort;
 
     // gate/up: the work list is the previous launch's output; down: it is two
@@ -173,18 +187,21 @@ __global__ void __launch_bounds__(kGemmWarps * 32, 2) grouped_gemm_kernel(GemmAr
         s_tile = int(blockIdx.x) - (MODE == 0 ? s_en.ubase_gu : s_en.ubase_dn);
         s_bad = 0;
         s_abort = 0;
-        mbar_init(&mbar[0], 1);
-        mbar_init(&mbar[1], 1);
         for (int i = 0; i < NST; ++i) {
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], kMathWarps);
         }
+        for (int i = 0; i < kOpBufs; ++i) {
+            mbar_init(&ready[i], kMathWarps);
+            mbar_init(&freed[i], 1);
+        }
+        mbar_init(&done, 1);
         mbar_fence_init();
     }
     __syncthreads();
     const FfnEntry en = s_en;
     const int tile = s_tile;
-    const int M = min(en.n_rows, 128);
+    const int M = min(en.n_rows, kGemmMaxRows);
     const int N = (M + 15) & ~15;
     const int F = en.F;
     const int Kin = MODE == 0 ? D : F;
@@ -194,8 +211,9 @@ __global__ void __launch_bounds__(kGemmWarps * 32, 2) grouped_gemm_kernel(GemmAr
     const int gpc = ks / kGroup;  // groups per chunk (a multiple of GPS)
     const uint8_t* sec = en.blob + (MODE == 0 ? size_t(0) : gu_section_bytes(D, F));
     const int nstages = ngroups / GPS;
+    const int ncols = N <= 32 ? 32 : 64;  // tensor-memory columns: fp32 accumulator [128 lanes][N]
 
-    if (warp == kMathWarps) {
+    if (warp == kProducerWarp) {
         // -------------------------------------------------------- producer
         if (lane == 0) {
             const uint64_t pol = l2_evict_first();
@@ -215,8 +233,53 @@ __global__ void __launch_bounds__(kGemmWarps * 32, 2) grouped_gemm_kernel(GemmAr
                     bulk_g2s(dst + w * BT_BYTES + GPS * 1024, chunk + 16 * ks + gg * 128, GPS * 128, &full[st], pol);
                 }
             }
+            // no copy may land after the CTA exits
             const int first = issued > NST ? issued - NST : 0;
             for (int i = first; i < issued; ++i) mbar_wait(&full[i % NST], (i / NST) & 1, A.status);
+        }
+        return;
+    }
+
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tbase)),
+                     "r"(ncols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (tid < M) s_rows[tid] = A.rows[en.row0 + tid];
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    named_sync(2, kMathThreads + 32);  // math warps + MMA warp
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = tbase;
+
+    if (warp == kMmaWarp) {
+        // ----------------------------------------------------------- MMA issue
+        if (lane == 0) {
+            const uint32_t idesc = (1u << 4) | (uint32_t(N >> 3) << 17) | (uint32_t(128 >> 4) << 24);
+            for (int g = 0; g < ngroups; ++g) {
+                const int b = g % kOpBufs;
+                if (!ring_wait_gemm(&ready[b], (g / kOpBufs) & 1, A.status, &s_abort)) break;
+                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                const uint32_t a_addr = smem_u32(sA + b * kABytes), b_addr = smem_u32(sB + b * kBBytes);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t ad = umma_desc(a_addr + kk * 256);
+                    const uint64_t bd = umma_desc(b_addr + kk * 256);
+                    const uint32_t acc = (g > 0 || kk > 0) ? 1u : 0u;
+                    asm volatile(
+                        "{\n .reg .pred p;\n setp.ne.u32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, "
+                        "%3, p;\n}\n" ::"r"(tmem),
+                        "l"(ad), "l"(bd), "r"(idesc), "r"(acc)
+                        : "memory");
+                }
+                asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                                 smem_u32(&freed[b]))
+                             : "memory");
+            }
+            // completes when every MMA issued above has (also after an early stop)
+            asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                             smem_u32(&done))
+                         : "memory");
         }
         return;
     }
@@ -226,21 +289,6 @@ __global__ void __launch_bounds__(kGemmWarps * 32, 2) grouped_gemm_kernel(GemmAr
         pdl_wait();  // h is the gate/up GEMM's output
         pdl_trigger();
     }
-    if (tid < M) s_rows[tid] = A.rows[en.row0 + tid];
-    int ncols = 32;
-    while (ncols < N) ncols <<= 1;
-    if (warp == 0) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tbase)),
-                     "r"(ncols)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-    }
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-    named_sync(1, kMathThreads);
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    const uint32_t tmem = tbase;
-    const uint32_t idesc = (1u << 4) | (uint32_t(N >> 3) << 17) | (uint32_t(128 >> 4) << 24);
-
     // Activation tile tasks: task idx = tid + kMathThreads*i covers row j,
     // inputs 8*kb .. +7 of the group, with j = 8*(idx/64) + idx%8 and
     // kb = (idx/8)%8: a warp's 16-byte stores then hit 8 different rows of a
@@ -284,28 +332,19 @@ __global__ void __launch_bounds__(kGemmWarps * 32, 2) grouped_gemm_kernel(GemmAr
         }
     };
     load_b(0);
-    bool ok = true;
     // this thread's weights: row r of the 128 (blob tile 4*tile + r/32, row r%32), inputs 32*hk .. +31 of each group
     const int r = tid & 127, hk = tid >> 7;
     const int bt_row = r >> 5, row = r & 31;
-    // One thread waits on every barrier (the ring stage of the next group, the
-    // MMAs that last read the next group's fp16 buffers) just before the CTA
-    // barrier that ends a group, and posts "stop" if a wait timed out; the
-    // flag alternates between two words so that no thread can still be
-    // reading the word being written.
-    __shared__ int s_stop[2], s_fin;
-    if (tid == 0) {
-        s_stop[0] = ring_wait_gemm(&full[0], 0, A.status, &s_abort) ? 0 : 1;
-        s_fin = 0;
-    }
-    named_sync(1, kMathThreads);
-    int g = 0;
-    for (; g < ngroups; ++g) {
-        if (s_stop[g & 1]) break;
+    bool ok = true;
+    for (int g = 0; g < ngroups && ok; ++g) {
         const int si = g / GPS, gl = g % GPS, st = si % NST;
-        const int buf = g & 1;
-        uint8_t* a = sA + buf * kGemmStageBytes;
-        uint8_t* b = sB + buf * kGemmStageBytes;
+        const int b = g % kOpBufs;
+        // the buffer set's previous MMAs are done; the ring stage has landed
+        if (g >= kOpBufs) ok = ring_wait_gemm(&freed[b], ((g / kOpBufs) - 1) & 1, A.status, &s_abort);
+        if (ok && gl == 0) ok = ring_wait_gemm(&full[st], (si / NST) & 1, A.status, &s_abort);
+        if (!ok) break;
+        uint8_t* a = sA + b * kABytes;
+        uint8_t* bt = sB + b * kBBytes;
         // B: this group's activations (loaded one group ahead), then the next group's loads
 #pragma unroll
         for (int i = 0; i < kBTasks; ++i) {
@@ -329,7 +368,7 @@ __global__ void __launch_bounds__(kGemmWarps * 32, 2) grouped_gemm_kernel(GemmAr
             for (int t = 0; t < 8; ++t)
                 if (!(fabsf(v[t]) <= 65504.f)) { s_bad = 1; v[t] = 0.f; }  // beyond fp16 (or NaN)
             const int j = 8 * (idx >> 6) + (idx & 7);
-            *reinterpret_cast<uint4*>(b + core_off(j, 8 * ((idx >> 3) & 7))) = pack_block_perm(v);
+            *reinterpret_cast<uint4*>(bt + core_off(j, 8 * ((idx >> 3) & 7))) = pack_block_perm(v);
         }
         if (g + 1 < ngroups) load_b(g + 1);
         // A: dequantise this thread's 32 weights of the group from the raw stage
@@ -343,54 +382,21 @@ __global__ void __launch_bounds__(kGemmWarps * 32, 2) grouped_gemm_kernel(GemmAr
             for (int j = 0; j < 4; ++j)  // word j: inputs 32*hk + 8j .. +7 of the group
                 *reinterpret_cast<uint4*>(a + core_off(r, 32 * hk + 8 * j)) = dequant_word(words[j], s2, b2);
         }
-        __syncwarp();
-        if (gl == GPS - 1 && lane == 0) mbar_arrive(&empty[st]);  // this warp is done with the raw stage
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic writes -> tensor-core reads
-        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-        bool next_ok = true;  // thread 0 only
-        if (tid == 0) {
-            // resources of group g + 1: its ring stage, and the MMAs of group g - 1 (its fp16 buffers)
-            const int g1 = g + 1;
-            next_ok = !s_abort;
-            if (next_ok && g1 < ngroups && g1 % GPS == 0)
-                next_ok = ring_wait_gemm(&full[(g1 / GPS) % NST], ((g1 / GPS) / NST) & 1, A.status, &s_abort);
-            if (next_ok && g1 < ngroups && g >= 1)
-                next_ok = ring_wait_gemm(&mbar[(g - 1) & 1], ((g - 1) >> 1) & 1, A.status, &s_abort);
-            s_stop[g1 & 1] = next_ok ? 0 : 1;
-        }
-        named_sync(1, kMathThreads);
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        if (tid == 0 && next_ok) {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t ad = umma_desc(smem_u32(a) + kk * 256);
-                const uint64_t bd = umma_desc(smem_u32(b) + kk * 256);
-                const uint32_t acc = (g > 0 || kk > 0) ? 1u : 0u;
-                asm volatile(
-                    "{\n .reg .pred p;\n setp.ne.u32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, "
-                    "p;\n}\n" ::"r"(tmem),
-                    "l"(ad), "l"(bd), "r"(idesc), "r"(acc)
-                    : "memory");
-            }
-            asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                             smem_u32(&mbar[buf]))
-                         : "memory");
+        __syncwarp();
+        if (lane == 0) {
+            mbar_arrive(&ready[b]);
+            if (gl == GPS - 1) mbar_arrive(&empty[st]);  // this warp is done with the raw stage
         }
     }
-    // every thread left the loop at the same g; after a full pass the last
-    // group's MMAs (and with them all earlier ones) complete before the epilogue
-    const bool stopped = g < ngroups;
-    if (tid == 0 && !stopped) {
-        const int last = ngroups - 1;
-        if (!ring_wait_gemm(&mbar[last & 1], (last >> 1) & 1, A.status, &s_abort)) s_fin = 1;
-    }
-    named_sync(1, kMathThreads);
-    ok = !stopped && !s_fin;
+    // every MMA the MMA warp issued has completed
+    if (ok) ok = ring_wait_gemm(&done, 0, A.status, &s_abort);
+    ok = __all_sync(0xffffffffu, ok);  // the tensor-memory loads below are warp-collective
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     if (s_bad && tid == 0) set_status(A.status, MOE_ERR_RANGE);
 
     if (ok) {
-        // warp w reads TMEM lanes 32*(w%4) ..; warps 0-3 take column blocks 0, 32, ..., warps 4-7 blocks 16, 48, ...
+        // warp w reads TMEM lanes 32*(w%4) ..; warps 0-3 take column blocks 0, 32, warps 4-7 blocks 16, 48
         const int q4 = warp & 3;
         for (int c0 = 16 * (warp >> 2); c0 < N; c0 += 32) {
             uint32_t v[16];

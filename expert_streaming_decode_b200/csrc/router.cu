@@ -86,6 +86,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_topk_kernel(
     float* gsum = xs + ng * (kGroup + 1);                                   // [rows][ng]
     float* scl = gsum + sh.rows * ng;                                       // [rows][ng]
     __shared__ float logits[kMaxE];  // rank 0 gathers all logits here
+    __shared__ float s_bias[kMaxE / kRouterCtas];
     __shared__ __align__(8) uint64_t full[2];
     __shared__ int s_ok;
 
@@ -125,8 +126,31 @@ __global__ void __launch_bounds__(kRouterThreads) router_topk_kernel(
 
     pdl_wait();
     pdl_trigger();
-    for (int k = threadIdx.x; k < D; k += blockDim.x)
-        xs[(k / kGroup) * (kGroup + 1) + k % kGroup] = bf16_to_f32(x[size_t(t) * D + k]);
+    // hidden state: one 16-byte load (8 inputs of one group) per thread and
+    // round, all issued before any is used; the CTA's logit biases likewise
+    {
+        const uint4* x8 = reinterpret_cast<const uint4*>(x + size_t(t) * D);
+        constexpr int kRounds = 2;  // D / 8 <= kRounds * kRouterThreads for D <= 8192
+        uint4 v[kRounds];
+#pragma unroll
+        for (int i = 0; i < kRounds; ++i) {
+            const int c = threadIdx.x + i * kRouterThreads;
+            if (c < D / 8) v[i] = x8[c];
+        }
+        if (bias && threadIdx.x < sh.e_per) s_bias[threadIdx.x] = bias[e0 + threadIdx.x];
+#pragma unroll
+        for (int i = 0; i < kRounds; ++i) {
+            const int c = threadIdx.x + i * kRouterThreads;
+            if (c >= D / 8) continue;
+            float* dst = xs + (c / 8) * (kGroup + 1) + (c % 8) * 8;  // inputs 8c .. 8c+7, one group
+            const uint32_t w4[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                dst[2 * j] = __uint_as_float(w4[j] << 16);
+                dst[2 * j + 1] = __uint_as_float(w4[j] & 0xFFFF0000u);
+            }
+        }
+    }
     float* logits0 = cluster.map_shared_rank(logits, 0);
 
     int consumed = 0;  // passes whose copies have landed
@@ -171,7 +195,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_topk_kernel(
             const int e = e0 + p * sh.rows + r;
             float acc = 0.0f;
             for (int g = 0; g < ng; ++g) acc = __fmaf_rn(scl[r * ng + g], gsum[r * ng + g], acc);
-            if (bias) acc = __fadd_rn(acc, bias[e]);
+            if (bias) acc = __fadd_rn(acc, s_bias[p * sh.rows + r]);
             logits0[e] = acc;
         }
         __syncthreads();  // gsum and scales are rewritten by the next pass

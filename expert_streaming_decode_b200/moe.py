@@ -68,6 +68,8 @@ lib.moe_ctx_sync.restype = _i
 lib.moe_ctx_sync.argtypes = [_vp, _vp, _i]
 lib.moe_ctx_launches.restype = C.c_uint64
 lib.moe_ctx_launches.argtypes = [_vp]
+lib.moe_gemm_min_tokens.restype = _i
+lib.moe_gemm_min_tokens.argtypes = []
 lib.moe_router_topk.restype = _i
 lib.moe_router_topk.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp]
 lib.moe_cache_reset.restype = _i

@@ -128,6 +128,11 @@ const char *moe_status_str(int status);
  * points, all streams).  Host counter; used to report launch counts. */
 uint64_t moe_ctx_launches(const moe_ctx *ctx);
 
+/* Smallest token count T for which moe_layer_forward runs the experts as the
+ * tcgen05 grouped GEMM (tokens grouped per expert, fp16 dequantised weight
+ * tiles); one-token calls run the streamed GEMV kernels.  Host only. */
+int moe_gemm_min_tokens(void);
+
 /* --------------------------------------------------------------- router
  * Router + top-K + gate weights for T tokens ("El milagro ...", "Por que la
  * mayor parte ...": the layer's small router keeps the K most relevant of the
@@ -317,7 +322,8 @@ int moe_ctx_profile_read(moe_ctx *ctx, double *total_ms, uint64_t *count);
  * between layers so that layer l+1's routing depends on layer l's output.
  *   r[t] += y[t] (fp32, in place);  x_next[t] = bf16(r[t] / rms(r[t])),
  *   rms = sqrt(mean(r^2) + 1e-6).   r dev fp32 [T][D], y dev fp32 [T][D],
- *   x_next dev bf16 [T][D].  One launch. */
+ *   x_next dev bf16 [T][D]; r and y 16-byte aligned, x_next 8-byte aligned
+ *   (MOE_ERR_ARG otherwise).  One launch. */
 int moe_residual_rmsnorm(moe_ctx *ctx, float *r, const float *y, uint16_t *x_next, int T,
                          cudaStream_t stream);
 

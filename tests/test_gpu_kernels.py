@@ -206,3 +206,28 @@ def test_expert_ffn_argument_errors():
         moe.expert_ffn(ctx, x, 1, d.K, ps, w, blobs, 1000, d.E, d.F, None, y)          # stride % 256
     with pytest.raises(moe.MoeError):
         moe.expert_ffn(ctx, x, 1, d.K, ps, w, blobs, 256 * 256, d.E, 100, None, y)     # unknown width
+
+
+# ------------------------------------------------------------------ harness
+@pytest.mark.parametrize("D", [512, 2816, 8192], ids=["512", "2816", "8192-looped"])
+def test_residual_rmsnorm_harness(D):
+    """The layer-chaining step of the benchmark: r += y exactly in fp32, and
+    x_next = bf16(r / sqrt(mean(r^2) + 1e-6)) within one bf16 step of an
+    fp64 evaluation (rows longer than the register path take the loop)."""
+    d = synth.Dims(D=D, E=16, K=4, F=64, FS=128, G=64, L=1, S=6)
+    T = 3
+    ctx = moe.Ctx.from_dims(d, max_tokens=T)
+    rng = np.random.default_rng(D)
+    r0 = rng.standard_normal((T, D)).astype(np.float32)
+    y0 = (0.3 * rng.standard_normal((T, D))).astype(np.float32)
+    r = torch.from_numpy(r0).cuda()
+    y = torch.from_numpy(y0).cuda()
+    xn = torch.empty((T, D), dtype=torch.int16, device="cuda")
+    moe.residual_rmsnorm(ctx, r, y, xn, T)
+    ctx.sync()
+    want_r = r0 + y0
+    assert np.array_equal(r.cpu().numpy(), want_r)
+    ref = want_r.astype(np.float64)
+    ref = ref / np.sqrt(np.mean(ref * ref, axis=1, keepdims=True) + 1e-6)
+    got = synth.bf16_bits_to_f32(xn.cpu().numpy().view(np.uint16)).astype(np.float64)
+    assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-30)
