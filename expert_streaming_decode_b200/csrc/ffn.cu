@@ -523,22 +523,11 @@ __global__ void __launch_bounds__((GemvCfg<MODE>::NW + 1) * 32) gemv_decode_kern
     constexpr int kStages = GemvCfg<MODE>::NSTAGES;
     constexpr int NCONS = NW * 32;
     // gate/up: the work list is the previous launch's output, so wait before
-    // reading it.  down: the work list is two launches back (written before
-    // the gate/up kernel), so weights stream while gate/up finishes; only the
-    // consumers wait, before staging h.
-    if (MODE == 0) {
-        pdl_wait();
-        pdl_trigger();
-    }
-    const WorkList W = *A.wl;
-    const int D = A.D;
-    const int U = MODE == 0 ? W.units_gu : W.units_dn;
-    const int G = gridDim.x, c = blockIdx.x;
-    const int u_begin = range_start(c, U, G), u_end = range_start(c + 1, U, G);
-    const DecodeMap M{W.n_shared, W.ush_gu, W.urt_gu, W.ns_sh_dn, W.ns_rt_dn, W.units_per_tile_dn, W.F, W.FS, D};
-    const int n_ent = min(W.n_entries, kCtaEntries);
-    const int NSg = D / kGuSlice;
-
+    // reading it; the token's hidden state is two or more launches back, so
+    // the consumers stage it first.  down: the work list is two launches back
+    // (written before the gate/up kernel), so weights stream while gate/up
+    // finishes; only the consumers wait, before staging h.
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     extern __shared__ __align__(128) uint8_t smem[];
     uint8_t* ring = smem;
     uint64_t* full = reinterpret_cast<uint64_t*>(ring + kStages * STAGE);
@@ -551,8 +540,61 @@ __global__ void __launch_bounds__((GemvCfg<MODE>::NW + 1) * 32) gemv_decode_kern
     float* Xs = sx + gs;                                                 // [gs]
     uint4* xq = reinterpret_cast<uint4*>(Xs + gs);                       // [vstride / 8]
     __shared__ int s_abort;
+    // 16-bit fixed-point image of the inputs, one load round trip per kBatch
+    // tasks (8 values each) per thread: MODE 0 the token's x (row 0: these
+    // lists carry one token), MODE 1 every entry's h segment
+    auto stage = [&](int tasks, const DecodeMap& M) {
+        constexpr int kBatch = 3;
+        for (int base = 0; base < tasks; base += kBatch * NCONS) {
+            float v[kBatch][8];
+#pragma unroll
+            for (int r = 0; r < kBatch; ++r) {  // all loads first: one round trip
+                const int t = base + r * NCONS + int(threadIdx.x);
+                if (t < tasks) {
+                    if (MODE == 0) {
+                        const uint4 q = reinterpret_cast<const uint4*>(A.x)[t];
+                        const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            v[r][2 * j] = __uint_as_float(w4[j] << 16);
+                            v[r][2 * j + 1] = __uint_as_float(w4[j] & 0xFFFF0000u);
+                        }
+                    } else {
+                        const int shc = M.nsh * (M.FS / 8);
+                        const int ee = t < shc ? t / (M.FS / 8) : M.nsh + (t - shc) / (M.F / 8);
+                        const float* h = A.h + s_row[ee].h_off + 8 * (t - M.stage_chunk0(ee));
+                        const float4 a4 = reinterpret_cast<const float4*>(h)[0];
+                        const float4 b4 = reinterpret_cast<const float4*>(h)[1];
+                        v[r][0] = a4.x; v[r][1] = a4.y; v[r][2] = a4.z; v[r][3] = a4.w;
+                        v[r][4] = b4.x; v[r][5] = b4.y; v[r][6] = b4.z; v[r][7] = b4.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) v[r][j] = 0.f;
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < kBatch; ++r) {
+                const int t = base + r * NCONS + int(threadIdx.x);
+                stage_task(v[r], t < tasks, t, xq, sx, Xs);
+            }
+        }
+        named_sync(1, NCONS);
+    };
+    if (MODE == 0) {
+        if (warp < NW) stage(A.D / 8, DecodeMap{});
+        pdl_wait();
+        pdl_trigger();
+    }
+    const WorkList W = *A.wl;
+    const int D = A.D;
+    const int U = MODE == 0 ? W.units_gu : W.units_dn;
+    const int G = gridDim.x, c = blockIdx.x;
+    const int u_begin = range_start(c, U, G), u_end = range_start(c + 1, U, G);
+    const DecodeMap M{W.n_shared, W.ush_gu, W.urt_gu, W.ns_sh_dn, W.ns_rt_dn, W.units_per_tile_dn, W.F, W.FS, D};
+    const int n_ent = min(W.n_entries, kCtaEntries);
+    const int NSg = D / kGuSlice;
 
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         s_abort = 0;
         for (int i = 0; i < kStages; ++i) {
@@ -608,49 +650,11 @@ __global__ void __launch_bounds__((GemvCfg<MODE>::NW + 1) * 32) gemv_decode_kern
         return;
     }
 
-    // ----------------------------------------- consumers: stage the inputs once
+    // ------------------------------------------------ consumers: stage h (down)
     if (MODE == 1) {
         pdl_wait();  // h is the gate/up kernel's output
         pdl_trigger();
-    }
-    {
-        const int tasks = MODE == 0 ? D / 8 : M.stage_chunk0(W.n_entries);
-        constexpr int kBatch = 3;  // tasks per thread per round trip
-        for (int base = 0; base < tasks; base += kBatch * NCONS) {
-            float v[kBatch][8];
-#pragma unroll
-            for (int r = 0; r < kBatch; ++r) {  // all loads first: one round trip
-                const int t = base + r * NCONS + int(threadIdx.x);
-                if (t < tasks) {
-                    if (MODE == 0) {
-                        const uint4 q = reinterpret_cast<const uint4*>(A.x + size_t(s_row[0].x_row) * D)[t];
-                        const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            v[r][2 * j] = __uint_as_float(w4[j] << 16);
-                            v[r][2 * j + 1] = __uint_as_float(w4[j] & 0xFFFF0000u);
-                        }
-                    } else {
-                        const int shc = M.nsh * (M.FS / 8);
-                        const int ee = t < shc ? t / (M.FS / 8) : M.nsh + (t - shc) / (M.F / 8);
-                        const float* h = A.h + s_row[ee].h_off + 8 * (t - M.stage_chunk0(ee));
-                        const float4 a4 = reinterpret_cast<const float4*>(h)[0];
-                        const float4 b4 = reinterpret_cast<const float4*>(h)[1];
-                        v[r][0] = a4.x; v[r][1] = a4.y; v[r][2] = a4.z; v[r][3] = a4.w;
-                        v[r][4] = b4.x; v[r][5] = b4.y; v[r][6] = b4.z; v[r][7] = b4.w;
-                    }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) v[r][j] = 0.f;
-                }
-            }
-#pragma unroll
-            for (int r = 0; r < kBatch; ++r) {
-                const int t = base + r * NCONS + int(threadIdx.x);
-                stage_task(v[r], t < tasks, t, xq, sx, Xs);
-            }
-        }
-        named_sync(1, NCONS);
+        stage(M.stage_chunk0(W.n_entries), M);
     }
 
     // -------------------------------------------------- consumers: the units
@@ -888,41 +892,88 @@ cudaError_t launch_ffn(const GemvLaunch& L, cudaStream_t s, void (*hook)(void*, 
 // ------------------------------------------------------ work-list builder
 // Groups the call's (token, k) pairs by expert slot (ascending slot, pairs in
 // ascending index inside a slot), splits each group into entries of at most
-// kMaxRows rows, puts the shared expert (all tokens) first, and computes each
-// entry's first gate/up and down unit.
-__global__ void __launch_bounds__(256) build_worklist_kernel(WorkListArgs a) {
+// kMaxRows rows (kGemmMaxRows in GEMM mode), puts the shared expert (all
+// tokens) first, and computes each entry's first gate/up and down unit.  One
+// CTA: counts with shared-memory atomics, prefix sums by block scans, ranks
+// by an in-order warp scan over pairs staged in shared memory, entries
+// written in parallel.
+constexpr int kWlThreads = 256;
+constexpr int kWlChunk = 2048;  // pairs staged per round of the ranking scan
+
+// Exclusive scan of v over the CTA (kWlThreads threads); returns the prefix
+// of this thread and the total in *total.
+__device__ int wl_block_scan(int v, int* warp_tot, int* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int inc = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, inc, off);
+        if (lane >= off) inc += o;
+    }
+    if (lane == 31) warp_tot[warp] = inc;
+    __syncthreads();
+    int before = 0, all = 0;
+    for (int w = 0; w < kWlThreads / 32; ++w) {
+        if (w < warp) before += warp_tot[w];
+        all += warp_tot[w];
+    }
+    __syncthreads();
+    *total = all;
+    return before + inc - v;
+}
+
+__global__ void __launch_bounds__(kWlThreads) build_worklist_kernel(WorkListArgs a) {
     __shared__ int cnt[1024];
-    __shared__ int off[1025];
-    __shared__ int ent_base[1025];
+    __shared__ int off[1024];
+    __shared__ int ebase[1024];
+    __shared__ int run[1024];
+    __shared__ int16_t sl_s[kWlChunk];
+    __shared__ int warp_tot[kWlThreads / 32];
+    __shared__ int s_maxr;
     pdl_wait();
     pdl_trigger();
     const int np = a.T * a.K;
-    for (int i = threadIdx.x; i < a.n_slot_range; i += blockDim.x) cnt[i] = 0;
+    const int S = a.n_slot_range;
+    auto slot_of = [&](int p) -> int {  // -1: not in this wave
+        if (a.pair_wave && a.pair_wave[p] != a.wave) return -1;
+        const int sl = a.pair_slot[p];
+        return (sl < 0 || sl >= S) ? 0 : sl;
+    };
+    for (int i = threadIdx.x; i < S; i += blockDim.x) { cnt[i] = 0; run[i] = 0; }
+    if (threadIdx.x == 0) s_maxr = 0;
     __syncthreads();
     bool bad = false;
     for (int p = threadIdx.x; p < np; p += blockDim.x) {
         if (a.pair_wave && a.pair_wave[p] != a.wave) continue;
-        int sl = a.pair_slot[p];
-        if (sl < 0 || sl >= a.n_slot_range) { bad = true; sl = 0; }
-        atomicAdd(&cnt[sl], 1);
+        const int sl = a.pair_slot[p];
+        if (sl < 0 || sl >= S) bad = true;
+        atomicAdd(&cnt[(sl < 0 || sl >= S) ? 0 : sl], 1);
     }
     if (bad) set_status(a.status, MOE_ERR_RANGE);
     __syncthreads();
+
     const int mr = a.gemm ? kGemmMaxRows : kMaxRows;  // rows per entry
     const int nsh = a.shared_blob ? (a.T + mr - 1) / mr : 0;
-    if (threadIdx.x == 0) {
-        int o = a.shared_blob ? a.T : 0, eb = nsh;
-        for (int sl = 0; sl < a.n_slot_range; ++sl) {
-            off[sl] = o;
-            ent_base[sl] = eb;
-            o += cnt[sl];
-            eb += (cnt[sl] + mr - 1) / mr;
-        }
-        off[a.n_slot_range] = o;
-        ent_base[a.n_slot_range] = eb;
+    // prefix sums over slots: first row (after the shared rows) and first entry
+    // (after the shared entries) of every slot; each thread scans a run of slots
+    const int per = (S + kWlThreads - 1) / kWlThreads;
+    const int s0 = min(S, int(threadIdx.x) * per), s1 = min(S, s0 + per);
+    int rows_mine = 0, ents_mine = 0, maxr_mine = 0;
+    for (int sl = s0; sl < s1; ++sl) {
+        rows_mine += cnt[sl];
+        ents_mine += (cnt[sl] + mr - 1) / mr;
+        maxr_mine = max(maxr_mine, min(cnt[sl], mr));
     }
-    __syncthreads();
-    const int n_ent = ent_base[a.n_slot_range];
+    int rows_tot, ents_tot;
+    int ro = wl_block_scan(rows_mine, warp_tot, &rows_tot) + (a.shared_blob ? a.T : 0);
+    int eo = wl_block_scan(ents_mine, warp_tot, &ents_tot) + nsh;
+    for (int sl = s0; sl < s1; ++sl) {
+        off[sl] = ro;
+        ebase[sl] = eo;
+        ro += cnt[sl];
+        eo += (cnt[sl] + mr - 1) / mr;
+    }
+    if (maxr_mine > 0) atomicMax(&s_maxr, maxr_mine);
     // rows of the shared expert
     for (int t = threadIdx.x; a.shared_blob && t < a.T; t += blockDim.x) {
         FfnRow r;
@@ -932,80 +983,79 @@ __global__ void __launch_bounds__(256) build_worklist_kernel(WorkListArgs a) {
         r.w = 1.0f;
         a.rows[t] = r;
     }
-    // routed rows: rank of pair p among the earlier pairs of its slot.  Warp 0
-    // walks the pairs 32 at a time in order; lanes holding the same slot rank
-    // themselves by lane, after the slot's running count (cnt is reused).
     __syncthreads();
-    for (int i = threadIdx.x; i < a.n_slot_range; i += blockDim.x) cnt[i] = 0;
-    __syncthreads();
-    if (threadIdx.x < 32) {
-        const int lane = threadIdx.x;
-        for (int base = 0; base < np; base += 32) {
-            const int p = base + lane;
-            int sl = -1;
-            if (p < np && !(a.pair_wave && a.pair_wave[p] != a.wave)) {
-                sl = a.pair_slot[p];
-                if (sl < 0 || sl >= a.n_slot_range) sl = 0;
-            }
-            const unsigned same = __match_any_sync(0xffffffffu, sl);
-            const int before = __popc(same & ((1u << lane) - 1u));
-            int rank = 0;
-            if (sl >= 0) rank = cnt[sl] + before;
-            __syncwarp();
-            if (sl >= 0 && before == 0) cnt[sl] += __popc(same);  // one lane per slot
-            __syncwarp();
-            if (sl >= 0) {
-                FfnRow r;
-                r.x_row = p / a.K;
-                r.h_off = p * a.F;
-                r.y_row = p / a.K;
-                r.w = a.gate_w[p];
-                a.rows[off[sl] + rank] = r;
+
+    // routed rows: rank of pair p among the earlier pairs of its slot.  Pairs
+    // are staged a chunk at a time; warp 0 walks them 32 at a time in order,
+    // lanes holding the same slot rank themselves by lane after the slot's
+    // running count.
+    for (int base = 0; base < np; base += kWlChunk) {
+        const int n = min(kWlChunk, np - base);
+        for (int i = threadIdx.x; i < n; i += blockDim.x) sl_s[i] = int16_t(slot_of(base + i));
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            const int lane = threadIdx.x;
+            for (int c = 0; c < n; c += 32) {
+                const int i = c + lane;
+                const int sl = i < n ? int(sl_s[i]) : -1;
+                const unsigned same = __match_any_sync(0xffffffffu, sl);
+                const int before = __popc(same & ((1u << lane) - 1u));
+                const int rank = sl >= 0 ? run[sl] + before : 0;
+                __syncwarp();
+                if (sl >= 0 && before == 0) run[sl] += __popc(same);  // one lane per slot
+                __syncwarp();
+                if (sl >= 0) {
+                    const int p = base + i;
+                    FfnRow r;
+                    r.x_row = p / a.K;
+                    r.h_off = p * a.F;
+                    r.y_row = p / a.K;
+                    r.w = a.gate_w[p];
+                    a.rows[off[sl] + rank] = r;
+                }
             }
         }
+        __syncthreads();
     }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        const int nsg = a.D / kGuSlice, tiles_dn = a.D / kChunkRows;
-        int ugu = 0, udn = 0, maxr = 0, upt = 0;
-        int e = 0;
-        for (int j = 0; j < nsh; ++j, ++e) {
+
+    // entries: the shared expert's first, then every slot's in slot order
+    const int nsg = a.D / kGuSlice, tiles_dn = a.D / kChunkRows;
+    const int ugu_sh = a.gemm ? a.FS / 64 : (a.FS / 16) * nsg;           // units of one shared entry
+    const int udn_sh = a.gemm ? a.D / 128 : tiles_dn * (a.FS > 0 ? a.FS / down_ks(a.FS) : 0);
+    const int ugu_rt = a.gemm ? a.F / 64 : (a.F / 16) * nsg;             // units of one routed entry
+    const int udn_rt = a.gemm ? a.D / 128 : tiles_dn * (a.F / down_ks(a.F));
+    for (int j = threadIdx.x; j < nsh; j += blockDim.x) {
+        FfnEntry en;
+        en.blob = a.shared_blob;
+        en.F = a.FS;
+        en.row0 = j * mr;
+        en.n_rows = min(mr, a.T - j * mr);
+        en.ubase_gu = j * ugu_sh;
+        en.ubase_dn = j * udn_sh;
+        a.entries[j] = en;
+    }
+    for (int sl = threadIdx.x; sl < S; sl += blockDim.x) {
+        for (int j = 0; j * mr < cnt[sl]; ++j) {
+            const int e = ebase[sl] + j;
             FfnEntry en;
-            en.blob = a.shared_blob;
-            en.F = a.FS;
-            en.row0 = j * mr;
-            en.n_rows = min(mr, a.T - j * mr);
-            en.ubase_gu = ugu;
-            en.ubase_dn = udn;
-            ugu += a.gemm ? a.FS / 64 : (a.FS / 16) * nsg;
-            udn += a.gemm ? a.D / 128 : tiles_dn * (a.FS / down_ks(a.FS));
-            upt += a.FS / down_ks(a.FS);
-            maxr = max(maxr, en.n_rows);
+            en.blob = a.slot_base + size_t(sl) * a.slot_stride;
+            en.F = a.F;
+            en.row0 = off[sl] + j * mr;
+            en.n_rows = min(mr, cnt[sl] - j * mr);
+            en.ubase_gu = nsh * ugu_sh + (e - nsh) * ugu_rt;
+            en.ubase_dn = nsh * udn_sh + (e - nsh) * udn_rt;
             a.entries[e] = en;
         }
-        for (int sl = 0; sl < a.n_slot_range; ++sl) {
-            for (int j = 0; j * mr < cnt[sl]; ++j, ++e) {
-                FfnEntry en;
-                en.blob = a.slot_base + size_t(sl) * a.slot_stride;
-                en.F = a.F;
-                en.row0 = off[sl] + j * mr;
-                en.n_rows = min(mr, cnt[sl] - j * mr);
-                en.ubase_gu = ugu;
-                en.ubase_dn = udn;
-                ugu += a.gemm ? a.F / 64 : (a.F / 16) * nsg;
-                udn += a.gemm ? a.D / 128 : tiles_dn * (a.F / down_ks(a.F));
-                upt += a.F / down_ks(a.F);
-                maxr = max(maxr, en.n_rows);
-                a.entries[e] = en;
-            }
-        }
+    }
+    if (threadIdx.x == 0) {
+        const int n_rt = ents_tot;
         WorkList wl;
-        wl.n_entries = n_ent;
-        wl.units_gu = ugu;
-        wl.units_dn = udn;
+        wl.n_entries = nsh + n_rt;
+        wl.units_gu = nsh * ugu_sh + n_rt * ugu_rt;
+        wl.units_dn = nsh * udn_sh + n_rt * udn_rt;
         wl.T = a.T;
-        wl.units_per_tile_dn = upt;
-        wl.max_rows = maxr;
+        wl.units_per_tile_dn = nsh * (a.FS > 0 ? a.FS / down_ks(a.FS) : 0) + n_rt * (a.F / down_ks(a.F));
+        wl.max_rows = max(s_maxr, nsh > 0 ? min(mr, a.T) : 0);
         wl.n_shared = nsh;
         wl.ush_gu = a.FS > 0 ? (a.FS / 16) * nsg : 1;
         wl.urt_gu = (a.F / 16) * nsg;
@@ -1018,7 +1068,7 @@ __global__ void __launch_bounds__(256) build_worklist_kernel(WorkListArgs a) {
 }
 
 cudaError_t launch_build_worklist(const WorkListArgs& a, bool pdl, cudaStream_t s) {
-    return launch_kernel(build_worklist_kernel, dim3(1), dim3(256), 0, s, pdl, 1, a);
+    return launch_kernel(build_worklist_kernel, dim3(1), dim3(kWlThreads), 0, s, pdl, 1, a);
 }
 
 }  // namespace moe

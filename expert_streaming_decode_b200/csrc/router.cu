@@ -15,9 +15,10 @@
 // go in passes through two buffers.  Every thread then runs the fp32 FMA
 // chain of one (expert, group of 64) pair; one thread per expert chains the
 // group sums with their scales.  Logits land in rank 0's shared memory through
-// distributed shared memory; rank 0's first warp selects the top-K with
-// shuffles and writes ids and weights.  The FMA order is fixed (below), so ids
-// are bit-reproducible.
+// distributed shared memory; in rank 0 every expert counts the experts that
+// rank above it (logit descending, id ascending), the K with fewer than K
+// above are the selection, and the first warp writes ids and weights.  The
+// FMA order is fixed (below), so ids are bit-reproducible.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -31,6 +32,7 @@ namespace moe {
 constexpr int kRouterCtas = 8;
 constexpr int kRouterThreads = 512;
 constexpr int kMaxE = 1024;
+constexpr int kMaxK = 16;
 constexpr int kRouterRowPad = 16;               // bytes added to every staged row
 constexpr size_t kRouterRingBudget = 120 << 10; // shared memory for staged rows
 constexpr size_t kRouterSmemMax = 200 << 10;    // dynamic shared memory limit of the kernel
@@ -87,6 +89,8 @@ __global__ void __launch_bounds__(kRouterThreads) router_topk_kernel(
     float* scl = gsum + sh.rows * ng;                                       // [rows][ng]
     __shared__ float logits[kMaxE];  // rank 0 gathers all logits here
     __shared__ float s_bias[kMaxE / kRouterCtas];
+    __shared__ int s_sel_id[kMaxK], s_nan;
+    __shared__ float s_sel_l[kMaxK];
     __shared__ __align__(8) uint64_t full[2];
     __shared__ int s_ok;
 
@@ -114,6 +118,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_topk_kernel(
         mbar_init(&full[1], 1);
         mbar_fence_init();
         s_ok = 1;
+        s_nan = 0;
     }
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -207,39 +212,37 @@ __global__ void __launch_bounds__(kRouterThreads) router_topk_kernel(
     if (!s_ok)
         for (int e = e0 + threadIdx.x; e < e0 + sh.e_per; e += blockDim.x) logits0[e] = __int_as_float(0x7fc00000);
     cluster.sync();
-    if (rank != 0 || threadIdx.x >= 32) return;
+    if (rank != 0) return;
 
-    // top-K by (logit desc, id asc) with warp shuffles; lane L owns ids L, L+32, ...
+    // top-K by (logit desc, id asc): every expert counts the experts ranked
+    // above it (shared-memory broadcast reads); ranks 0..K-1 are the selection
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        const float v = logits[e];
+        if (isnan(v)) {
+            s_nan = 1;
+            continue;
+        }
+        int above = 0;
+        for (int f = 0; f < E; ++f) {
+            const float u = logits[f];
+            above += (u > v) || (u == v && f < e);
+        }
+        if (above < K) {
+            s_sel_id[above] = e;
+            s_sel_l[above] = v;
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x >= 32) return;
     const int lane = threadIdx.x;
-    bool nan = false;
-    for (int e = lane; e < E; e += 32) nan |= isnan(logits[e]);
-    nan = __any_sync(0xffffffffu, nan);
-    if (nan) {
+    if (s_nan) {
         if (lane < K) { ids[size_t(t) * K + lane] = lane; gate_w[size_t(t) * K + lane] = 1.0f / K; }
         if (lane == 0) set_status(status, MOE_ERR_NAN);
         if (wlt.wl) write_decode_worklist(wlt, K, lane, 1.0f / K, true);
         return;
     }
-    uint32_t taken = 0;  // bit j: id lane + 32*j already selected (E <= 1024)
-    float sel_l = 0.f;
-    int sel_id = 0;
-    for (int i = 0; i < K; ++i) {
-        float bv = -INFINITY;
-        int bi = 0x7fffffff;
-        for (int j = 0, e = lane; e < E; ++j, e += 32) {
-            if ((taken >> j) & 1u) continue;
-            const float v = logits[e];
-            if (v > bv || (v == bv && e < bi)) { bv = v; bi = e; }
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-            if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-        }
-        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-        if (lane == i) { sel_l = bv; sel_id = bi; }
-    }
+    const float sel_l = lane < K ? s_sel_l[lane] : 0.f;
+    const int sel_id = lane < K ? s_sel_id[lane] : 0;
     // softmax over the K chosen (lane i holds the i-th largest; lane 0 the max)
     const float m = __shfl_sync(0xffffffffu, sel_l, 0);
     const float ex = lane < K ? expf(sel_l - m) : 0.0f;
