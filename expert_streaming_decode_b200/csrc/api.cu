@@ -65,6 +65,7 @@ struct moe_ctx {
     FfnRow* rows2 = nullptr;
     float* h = nullptr;
     int h_shared_off = 0;
+    int list_cap = 0;  // entries and rows each work-list buffer holds
     float* partials_gu = nullptr;
     int* counters_gu = nullptr;
     float* partials_dn = nullptr;
@@ -189,8 +190,11 @@ int max_entries(const moe_dims& d) {
 }
 
 // K3 (gate/up) and K4 (down + combine) over a work list already on the device.
+// shared_blob: the list's first entry is this shared expert and the gate/up
+// kernel may start it before the list exists (one-token lists only), or null.
 int run_ffn_list(moe_ctx* c, WorkList* wl, FfnEntry* entries, FfnRow* rows, const uint16_t* x, int T,
-                 const float* y_in, float* y, uint16_t* y_bf16, cudaStream_t s) {
+                 const float* y_in, float* y, uint16_t* y_bf16, cudaStream_t s,
+                 const uint8_t* shared_blob = nullptr) {
     cudaError_t e;
     GemvLaunch L;
     L.wl = wl;
@@ -210,6 +214,12 @@ int run_ffn_list(moe_ctx* c, WorkList* wl, FfnEntry* entries, FfnRow* rows, cons
     L.shapes = &c->shapes;
     L.status = c->status;
     L.pdl = c->pdl;
+    L.list_cap = c->list_cap;
+    if (T == 1 && shared_blob) {
+        L.shared_blob = shared_blob;
+        L.FS = c->d.d_ff_shared;
+        L.h_shared_off = c->h_shared_off;
+    }
     FfnHookArg ha{c, s};
     e = launch_ffn(L, s, c->prof ? ffn_hook : nullptr, &ha);
     c->launches += 2;
@@ -429,6 +439,7 @@ int moe_ctx_create(const moe_dims* dims, int device, moe_ctx** out) {
     const int ns_dn_max = fmax / down_ks(fmax);
     const size_t units_dn = size_t(ment) * (d.d_model / kChunkRows) * ns_dn_max;
     ok = ok && dalloc(&c->status, 1) == cudaSuccess;
+    c->list_cap = ment < T + pairs ? ment : T + pairs;
     ok = ok && dalloc(&c->wl, 1) == cudaSuccess;
     ok = ok && dalloc(&c->entries, ment) == cudaSuccess;
     ok = ok && dalloc(&c->rows, size_t(T) + pairs) == cudaSuccess;
@@ -623,7 +634,7 @@ int moe_layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache* ca
         prof_mark(c, MOE_PROF_ROUTER, false, s);
         c->launches += 1;
         if (e != cudaSuccess) return MOE_ERR_CUDA;
-        return run_ffn_list(c, c->wl, c->entries, c->rows, x, 1, nullptr, y, y_bf16, s);
+        return run_ffn_list(c, c->wl, c->entries, c->rows, x, 1, nullptr, y, y_bf16, s, W->shared_blob);
     }
     r = moe_router_topk(c, x, W->router_q, W->router_s, bias, T, id, gw, s);
     if (r != MOE_OK) return r;
@@ -667,7 +678,8 @@ int moe_layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache* ca
         // empty, so y starts from zero and both lists accumulate into it
         if (!W->shared_blob && cudaMemsetAsync(y, 0, sizeof(float) * c->d.d_model, s) != cudaSuccess)
             return MOE_ERR_CUDA;
-        r = run_ffn_list(c, c->wl, c->entries, c->rows, x, 1, W->shared_blob ? nullptr : y, y, y_bf16, s);
+        r = run_ffn_list(c, c->wl, c->entries, c->rows, x, 1, W->shared_blob ? nullptr : y, y, y_bf16, s,
+                         W->shared_blob);
         if (r != MOE_OK) return r;
         have_y = true;
     } else if (gemm) {

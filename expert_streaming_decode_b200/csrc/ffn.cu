@@ -64,6 +64,13 @@ struct GemvArgs {
     int D;
     int vstride;            // widest staged input row (D for gate/up, max F for down)
     int* status;
+    int list_cap;           // entries (and rows) the work-list buffers hold
+    // one-token gate/up: CTAs [0, gs) run the shared expert's tiles, which need
+    // nothing the preceding launch writes, without waiting for it
+    const uint8_t* shared_blob;
+    int FS;
+    int h_shared_off;
+    int gs;
 };
 
 __device__ __forceinline__ int range_start(int c, int U, int G) { return int((long long)c * U / G); }
@@ -581,19 +588,70 @@ __global__ void __launch_bounds__((GemvCfg<MODE>::NW + 1) * 32) gemv_decode_kern
         }
         named_sync(1, NCONS);
     };
-    if (MODE == 0) {
-        if (warp < NW) stage(A.D / 8, DecodeMap{});
-        pdl_wait();
-        pdl_trigger();
-    }
-    const WorkList W = *A.wl;
     const int D = A.D;
-    const int U = MODE == 0 ? W.units_gu : W.units_dn;
+    const int NSg = D / kGuSlice;
     const int G = gridDim.x, c = blockIdx.x;
-    const int u_begin = range_start(c, U, G), u_end = range_start(c + 1, U, G);
+    // gate/up CTAs [0, gs): the shared expert's tiles (the list's first entry),
+    // known before the wait; the other CTAs wait for the work list
+    const bool early = MODE == 0 && c < A.gs;
+    if (MODE == 0) {
+        if (warp < NW) stage(D / 8, DecodeMap{});
+        if (!early) {
+            pdl_wait();
+            pdl_trigger();
+        }
+    }
+    WorkList W;
+    FfnEntry my_en;
+    FfnRow my_row;
+    const int n_spec = min(kCtaEntries, A.list_cap);
+    if (early) {
+        W = WorkList{};
+        W.n_entries = 1;
+        W.n_shared = 1;
+        W.ush_gu = (A.FS / 16) * NSg;
+        W.urt_gu = 1;
+        W.units_gu = W.ush_gu;
+        W.max_rows = 1;
+        W.F = 64;
+        W.FS = A.FS;
+        my_en.blob = A.shared_blob;
+        my_en.F = A.FS;
+        my_en.n_rows = 1;
+        my_en.row0 = 0;
+        my_en.ubase_gu = 0;
+        my_en.ubase_dn = 0;
+        my_row.x_row = 0;
+        my_row.h_off = A.h_shared_off;
+        my_row.y_row = 0;
+        my_row.w = 1.0f;
+    } else {
+        // header, entries and rows in one round trip: in a one-token list entry
+        // e's row is row e
+        W = *A.wl;
+        if (int(threadIdx.x) < n_spec) {
+            my_en = A.entries[threadIdx.x];
+            my_row = A.rows[threadIdx.x];
+        }
+    }
+    const int U = MODE == 0 ? W.units_gu : W.units_dn;
+    // unit range: gate/up takes whole output tiles (no cross-CTA reduction),
+    // shared-expert tiles on CTAs [0, gs), the rest on [gs, G); down splits
+    // its units evenly
+    int u_begin, u_end;
+    if (MODE == 0) {
+        const int t_lo = A.gs > 0 ? (A.FS / 16) : 0;  // first tile of this CTA class
+        const int t_hi = early ? t_lo : U / NSg;
+        const int c0 = early ? 0 : A.gs, gc = early ? A.gs : G - A.gs;
+        const int tb = early ? 0 : t_lo, nt = early ? A.FS / 16 : t_hi - t_lo;
+        u_begin = (tb + range_start(c - c0, nt, gc)) * NSg;
+        u_end = (tb + range_start(c - c0 + 1, nt, gc)) * NSg;
+    } else {
+        u_begin = range_start(c, U, G);
+        u_end = range_start(c + 1, U, G);
+    }
     const DecodeMap M{W.n_shared, W.ush_gu, W.urt_gu, W.ns_sh_dn, W.ns_rt_dn, W.units_per_tile_dn, W.F, W.FS, D};
     const int n_ent = min(W.n_entries, kCtaEntries);
-    const int NSg = D / kGuSlice;
 
     if (threadIdx.x == 0) {
         s_abort = 0;
@@ -603,16 +661,18 @@ __global__ void __launch_bounds__((GemvCfg<MODE>::NW + 1) * 32) gemv_decode_kern
         }
         mbar_fence_init();
     }
-    if (threadIdx.x < n_ent) {
-        const FfnEntry en = A.entries[threadIdx.x];
-        s_ent[threadIdx.x] = en;
-        s_row[threadIdx.x] = A.rows[en.row0];
+    if (int(threadIdx.x) < n_ent) {
+        s_ent[threadIdx.x] = my_en;
+        s_row[threadIdx.x] = my_row;
     }
     __syncthreads();
     if (u_begin >= u_end) return;
-    {
+    if (!early) {
         const int need = MODE == 0 ? D : M.stage_chunk0(W.n_entries) * 8;  // staged input values
-        if (W.n_entries > kCtaEntries || W.max_rows > 1 || need > A.vstride) {  // not a one-token list
+        bool bad = W.n_entries > n_spec || W.max_rows > 1 || need > A.vstride;  // not a one-token list
+        if (MODE == 0 && A.gs > 0) bad |= W.n_shared != 1 || W.ush_gu != (A.FS / 16) * NSg;
+        if (MODE == 0) bad |= (U % NSg) != 0;
+        if (bad) {
             if (threadIdx.x == 0) set_status(A.status, MOE_ERR_STATE);
             return;
         }
@@ -860,12 +920,22 @@ cudaError_t launch_ffn(const GemvLaunch& L, cudaStream_t s, void (*hook)(void*, 
     a.y_bf16 = L.y_bf16;
     a.D = L.D;
     a.status = L.status;
+    a.list_cap = L.list_cap;
+    a.shared_blob = L.shared_blob;
+    a.FS = L.FS;
+    a.h_shared_off = L.h_shared_off;
+    a.gs = 0;
     const bool one = L.rmax == 1;
     // K3: gate/up -> h
     a.partials = L.partials_gu;
     a.counters = L.counters_gu;
     a.vstride = L.shapes->vstride_gu;
     const GemvShape& g = L.shapes->gu[one ? 0 : 1];
+    if (one && L.shared_blob && L.FS >= 16) {
+        // one CTA per shared-expert tile, at most a third of the grid
+        const int sh_tiles = L.FS / 16;
+        a.gs = sh_tiles < g.grid / 3 ? sh_tiles : g.grid / 3;
+    }
     if (hook) hook(hook_arg, 0);
     cudaError_t e;
     if (one)
@@ -876,6 +946,7 @@ cudaError_t launch_ffn(const GemvLaunch& L, cudaStream_t s, void (*hook)(void*, 
     if (e != cudaSuccess) return e;
     if (hook) hook(hook_arg, 1);
     // K4: down + combine -> y
+    a.gs = 0;
     a.partials = L.partials_dn;
     a.counters = L.counters_dn;
     a.vstride = one ? L.shapes->stage_dn_decode : L.shapes->vstride_dn;

@@ -33,6 +33,13 @@ struct GemvLaunch {
     const GemvShapes* shapes;
     int* status;
     bool pdl = true;  // launch with programmatic dependent launch
+    int list_cap = 0;  // entries and rows the work-list buffers hold
+    // one-token lists whose first entry is the shared expert: its blob, width
+    // and h offset, so the gate/up kernel can start it before the work list
+    // exists (null: no such entry, or do not start early)
+    const uint8_t* shared_blob = nullptr;
+    int FS = 0;
+    int h_shared_off = 0;
 };
 
 struct WorkListArgs {
