@@ -215,6 +215,7 @@ int run_ffn_list(moe_ctx* c, WorkList* wl, FfnEntry* entries, FfnRow* rows, cons
     L.status = c->status;
     L.pdl = c->pdl;
     L.list_cap = c->list_cap;
+    if (T == 1) L.max_tiles_gu = (shared_blob ? c->d.d_ff_shared / 16 : 0) + c->d.top_k * (c->d.d_ff / 16);
     if (T == 1 && shared_blob) {
         L.shared_blob = shared_blob;
         L.FS = c->d.d_ff_shared;

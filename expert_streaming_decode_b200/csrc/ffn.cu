@@ -48,6 +48,23 @@ struct GemvCfg<1> {  // down: KS <= 704, up to 11 groups per chunk, one per warp
     static constexpr int NSTAGES = 6;
 };
 
+// One-token decode kernels.  Gate/up CTAs take one whole output tile each
+// (11 units of 4.6 KB for the 26B-A4B shapes); consumer warps 0-3 read one
+// group of every unit, warps 4-7 (when NW = 8) alternate units with them.
+template <int MODE>
+struct DecodeCfg;
+template <>
+struct DecodeCfg<0> {
+    static constexpr int NW = 4;  // a multiple of 4 (groups per 256-input unit)
+    static constexpr int NSTAGES = 8;
+    static constexpr int kTilesPerCta = 1;
+};
+template <>
+struct DecodeCfg<1> {
+    static constexpr int NW = 11;
+    static constexpr int NSTAGES = 6;
+};
+
 constexpr int kCtaEntries = 24;  // work-list entries a CTA keeps in shared memory
 
 struct GemvArgs {
@@ -524,10 +541,10 @@ __device__ __forceinline__ void stage_task(const float (&v)[8], bool ok, int chu
 }
 
 template <int MODE>
-__global__ void __launch_bounds__((GemvCfg<MODE>::NW + 1) * 32) gemv_decode_kernel(GemvArgs A) {
-    constexpr int NW = GemvCfg<MODE>::NW;
+__global__ void __launch_bounds__((DecodeCfg<MODE>::NW + 1) * 32) gemv_decode_kernel(GemvArgs A) {
+    constexpr int NW = DecodeCfg<MODE>::NW;
     constexpr int STAGE = GemvCfg<MODE>::STAGE;
-    constexpr int kStages = GemvCfg<MODE>::NSTAGES;
+    constexpr int kStages = DecodeCfg<MODE>::NSTAGES;
     constexpr int NCONS = NW * 32;
     // gate/up: the work list is the previous launch's output, so wait before
     // reading it; the token's hidden state is two or more launches back, so
@@ -657,7 +674,7 @@ __global__ void __launch_bounds__((GemvCfg<MODE>::NW + 1) * 32) gemv_decode_kern
         s_abort = 0;
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&full[i], 1);
-            mbar_init(&empty[i], NW);
+            mbar_init(&empty[i], MODE == 0 ? 4 : NW);  // the warps that read a unit
         }
         mbar_fence_init();
     }
@@ -739,9 +756,13 @@ __global__ void __launch_bounds__((GemvCfg<MODE>::NW + 1) * 32) gemv_decode_kern
         const int g_in0 = MODE == 0 ? slice * (kGuSlice / kGroup) : M.stage_chunk0(e) / 8 + slice * (ks / kGroup);
         const float w = MODE == 0 ? 1.f : s_row[e].w;
 
-        const bool have = ring_wait(&full[st], (i / kStages) & 1, A.status, &s_abort);
+        // gate/up: warps 4j .. 4j+3 read units i = j (mod NW / 4) of the
+        // range, one group each; down: every warp reads every unit
+        const bool mine = MODE == 1 || (i % (NW / 4)) == (warp >> 2);
+        const int gw = MODE == 0 ? (warp & 3) : warp, gstep = MODE == 0 ? 4 : NW;
+        const bool have = mine && ring_wait(&full[st], (i / kStages) & 1, A.status, &s_abort);
         const uint8_t* chunk = ring + size_t(st) * STAGE;
-        for (int g = warp; have && g < ks / kGroup; g += NW) {
+        for (int g = gw; have && g < ks / kGroup; g += gstep) {
             const uint4 qa = lds128(chunk + ((2 * g) * 32 + lane) * 16);
             const uint4 qb = lds128(chunk + ((2 * g + 1) * 32 + lane) * 16);
             const uint32_t sbw = *reinterpret_cast<const uint32_t*>(chunk + 16 * ks + (g * 32 + lane) * 4);
@@ -765,7 +786,7 @@ __global__ void __launch_bounds__((GemvCfg<MODE>::NW + 1) * 32) gemv_decode_kern
             acc = fmaf(w, part, acc);
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[st]);
+        if (mine && lane == 0) mbar_arrive(&empty[st]);
 
         const bool seg_end = (u + 1 == u_end) || (u + 1 == key_u0 + key_len);
         if (!seg_end) continue;
@@ -835,8 +856,8 @@ static size_t gemv_smem(int vstride, int T) {
 // Decode kernel: entries + their rows, red, per-group scale/sum, staged image.
 template <int MODE>
 static size_t decode_smem(int vstride) {
-    constexpr int NW = GemvCfg<MODE>::NW;
-    size_t b = size_t(GemvCfg<MODE>::NSTAGES) * GemvCfg<MODE>::STAGE + 2 * GemvCfg<MODE>::NSTAGES * sizeof(uint64_t);
+    constexpr int NW = DecodeCfg<MODE>::NW;
+    size_t b = size_t(DecodeCfg<MODE>::NSTAGES) * GemvCfg<MODE>::STAGE + 2 * DecodeCfg<MODE>::NSTAGES * sizeof(uint64_t);
     b += (sizeof(FfnEntry) + sizeof(FfnRow)) * kCtaEntries;
     b += size_t(NW) * 32 * 4;
     b += size_t(((vstride / kGroup) + 3) & ~3) * 4 * 2;
@@ -873,7 +894,7 @@ cudaError_t ffn_prepare(int D, int F, int FS, int K, int T, int sms, GemvShapes*
     shapes->vstride_gu = D;
     shapes->vstride_dn = vdn;
     shapes->stage_dn_decode = K * F + FS;
-    if ((e = shape_of(gemv_decode_kernel<0>, (GemvCfg<0>::NW + 1) * 32, decode_smem<0>(D), sms, false,
+    if ((e = shape_of(gemv_decode_kernel<0>, (DecodeCfg<0>::NW + 1) * 32, decode_smem<0>(D), sms, false,
                       &shapes->gu[0])) != cudaSuccess)
         return e;
     if ((e = shape_of(stream_gemv_kernel<0, kMaxRows>, (GemvCfg<0>::NW + 1) * 32, gemv_smem<0, kMaxRows>(D, T), sms,
@@ -893,7 +914,7 @@ cudaError_t ffn_shapes_one_row(int vstride_gu, int stage_dn, int T, int sms, Gem
     *shapes = GemvShapes{};
     shapes->vstride_gu = vstride_gu;
     shapes->stage_dn_decode = stage_dn;
-    cudaError_t e = shape_of(gemv_decode_kernel<0>, (GemvCfg<0>::NW + 1) * 32, decode_smem<0>(vstride_gu), sms, true,
+    cudaError_t e = shape_of(gemv_decode_kernel<0>, (DecodeCfg<0>::NW + 1) * 32, decode_smem<0>(vstride_gu), sms, true,
                              &shapes->gu[0]);
     if (e != cudaSuccess) return e;
     return shape_of(gemv_decode_kernel<1>, (GemvCfg<1>::NW + 1) * 32, decode_smem<1>(stage_dn), sms, true,
@@ -903,7 +924,7 @@ cudaError_t ffn_shapes_one_row(int vstride_gu, int stage_dn, int T, int sms, Gem
 cudaError_t ffn_ensure_one_row_smem(const GemvShapes& shapes) {
     GemvShape tmp;
     const int sms = 1;
-    cudaError_t e = shape_of(gemv_decode_kernel<0>, (GemvCfg<0>::NW + 1) * 32, shapes.gu[0].smem, sms, true, &tmp);
+    cudaError_t e = shape_of(gemv_decode_kernel<0>, (DecodeCfg<0>::NW + 1) * 32, shapes.gu[0].smem, sms, true, &tmp);
     if (e != cudaSuccess) return e;
     return shape_of(gemv_decode_kernel<1>, (GemvCfg<1>::NW + 1) * 32, shapes.dn[0].smem, sms, true, &tmp);
 }
@@ -931,15 +952,22 @@ cudaError_t launch_ffn(const GemvLaunch& L, cudaStream_t s, void (*hook)(void*, 
     a.counters = L.counters_gu;
     a.vstride = L.shapes->vstride_gu;
     const GemvShape& g = L.shapes->gu[one ? 0 : 1];
-    if (one && L.shared_blob && L.FS >= 16) {
-        // one CTA per shared-expert tile, at most a third of the grid
-        const int sh_tiles = L.FS / 16;
-        a.gs = sh_tiles < g.grid / 3 ? sh_tiles : g.grid / 3;
+    int grid_gu = g.grid;
+    if (one && L.max_tiles_gu > 0) {
+        // whole tiles, kTilesPerCta per CTA: the shared expert's on CTAs
+        // [0, gs) (started before the list exists), the rest after them
+        constexpr int tpc = DecodeCfg<0>::kTilesPerCta;
+        const int sh = L.shared_blob ? L.FS / 16 : 0;
+        const int gs = (sh + tpc - 1) / tpc;
+        int gr = (L.max_tiles_gu - sh + tpc - 1) / tpc;
+        gr = gr < 1 ? 1 : gr;
+        grid_gu = gs + gr < g.grid ? gs + gr : g.grid;
+        a.gs = gs < grid_gu - 1 ? gs : grid_gu - 1;
     }
     if (hook) hook(hook_arg, 0);
     cudaError_t e;
     if (one)
-        e = launch_kernel(gemv_decode_kernel<0>, dim3(g.grid), dim3((GemvCfg<0>::NW + 1) * 32), g.smem, s, L.pdl, 1, a);
+        e = launch_kernel(gemv_decode_kernel<0>, dim3(grid_gu), dim3((DecodeCfg<0>::NW + 1) * 32), g.smem, s, L.pdl, 1, a);
     else
         e = launch_kernel(stream_gemv_kernel<0, kMaxRows>, dim3(g.grid), dim3((GemvCfg<0>::NW + 1) * 32), g.smem, s,
                           L.pdl, 1, a);

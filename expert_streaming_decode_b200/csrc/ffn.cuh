@@ -34,6 +34,7 @@ struct GemvLaunch {
     int* status;
     bool pdl = true;  // launch with programmatic dependent launch
     int list_cap = 0;  // entries and rows the work-list buffers hold
+    int max_tiles_gu = 0;  // one-token lists: most gate/up output tiles the list can hold (0: unknown)
     // one-token lists whose first entry is the shared expert: its blob, width
     // and h offset, so the gate/up kernel can start it before the work list
     // exists (null: no such entry, or do not start early)

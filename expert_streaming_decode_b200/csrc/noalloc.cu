@@ -174,6 +174,7 @@ extern "C" int moe_expert_ffn_noalloc(int d_model, int d_ff, int top_k, const ui
     G.D = d_model;
     G.rmax = 1;
     G.list_cap = kNoAllocMaxK;  // entries capacity (rows hold one more)
+    G.max_tiles_gu = top_k * (d_ff / 16);
     G.shapes = &st->shapes;
     G.status = status;
     return launch_ffn(G, stream, nullptr, nullptr) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
