@@ -67,6 +67,32 @@ def parse_args():
 
 
 # --------------------------------------------------------------- helpers
+def csrc_sha256():
+    """Hash of the CUDA sources: DRAM traffic recorded under profiles/ is
+    reported only for the kernels it was measured on."""
+    import hashlib
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "expert_streaming_decode_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(f.encode())
+            h.update(open(os.path.join(d, f), "rb").read())
+    return h.hexdigest()
+
+
+def recorded_traffic(key):
+    """DRAM bytes (read + write) per layer-token of one kernel on one workload,
+    from one ncu capture (profiles/traffic.json), or None when absent or taken
+    on other kernel sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    rec = json.load(open(p))
+    if rec.get("source_sha256") != csrc_sha256():
+        return None
+    return rec.get("bytes_per_layer_token", {}).get(key)
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -605,7 +631,9 @@ def main():
     kname = "grouped_gemm_kernel (tcgen05)" if gemm else "gemv_decode_kernel" if T == 1 else "stream_gemv_kernel"
     line["roofline"] = {"bound": "hbm", "kernel": f"{kname} ({dom})",
                         "achieved": ach, "peak": hbm_peak,
-                        "unit": "GB/s", "frac": ach / hbm_peak, "traffic": None,
+                        "unit": "GB/s", "frac": ach / hbm_peak,
+                        "traffic": recorded_traffic(f"{args.workload}:{dom}"),
+                        "traffic_unit": "DRAM bytes per layer-token (ncu, profiles/traffic.json)",
                         "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
                         else "fallback 6650 GB/s"}
     if gemm:
