@@ -100,7 +100,7 @@ bool dims_ok(const moe_dims* d) {
     auto ff_ok = [](int F) { return F > 0 && F % 64 == 0 && (F <= 704 || F % 704 == 0); };
     if (d->d_model <= 0 || d->d_model % 256 || d->d_model > 8192) return false;  // batched GEMV stages 8 input rows in shared memory
     if (d->group != 64) return false;
-    if (d->n_experts <= 0 || d->n_experts > 1024 || d->n_experts % 8) return false;
+    if (d->n_experts <= 0 || d->n_experts > 1024 || d->n_experts % 16) return false;  // 16 router CTAs
     if (d->top_k <= 0 || d->top_k > 16 || d->top_k > d->n_experts) return false;
     if (!ff_ok(d->d_ff) || d->d_ff > 3 * 704) return false;
     if (d->d_ff_shared != 0 && (!ff_ok(d->d_ff_shared) || d->d_ff_shared > 3 * 704)) return false;

@@ -26,6 +26,10 @@ namespace moe {
 
 constexpr int kPlanThreads = 256;
 
+// shared-memory words before the staged mailbox rows: 6 int arrays of E, one
+// of S, two byte arrays of E (rounded up to whole words)
+__host__ __device__ inline int plan_mb_offset_words(int E, int S) { return 6 * E + S + (2 * E + 3) / 4; }
+
 __global__ void __launch_bounds__(kPlanThreads) cache_plan_kernel(
     const int32_t* __restrict__ ids, int npairs, int E, int S, int32_t* __restrict__ state, uint32_t step,
     int32_t* __restrict__ pair_slot, int32_t* __restrict__ pair_wave, PlanMailbox* mailbox, uint32_t seq,
@@ -40,7 +44,9 @@ __global__ void __launch_bounds__(kPlanThreads) cache_plan_kernel(
     int32_t* uwave = uslot + E;                           // [E]
     uint8_t* inwave = reinterpret_cast<uint8_t*>(uwave + E);  // [E]
     uint8_t* uhit = inwave + E;                           // [E] 1: the expert was resident
+    int32_t* mb = reinterpret_cast<int32_t*>(psm) + plan_mb_offset_words(E, S);  // [5][E] mailbox rows, staged
     __shared__ int32_t ulist[1024];
+    __shared__ int s_n;
 
     uint32_t* g_count = reinterpret_cast<uint32_t*>(state);
     uint32_t* g_last = g_count + E;
@@ -49,6 +55,8 @@ __global__ void __launch_bounds__(kPlanThreads) cache_plan_kernel(
     pdl_wait();
     pdl_trigger();
 
+    // the first pairs' ids load together with the state: one round trip
+    const int id_first = int(threadIdx.x) < npairs ? ids[threadIdx.x] : 0;
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         mult[e] = 0;
         count[e] = g_count[e];
@@ -63,7 +71,7 @@ __global__ void __launch_bounds__(kPlanThreads) cache_plan_kernel(
     __syncthreads();
     bool bad = false;
     for (int p = threadIdx.x; p < npairs; p += blockDim.x) {
-        int e = ids[p];
+        int e = p == int(threadIdx.x) ? id_first : ids[p];
         if (e < 0 || e >= E) { bad = true; e = 0; }
         atomicAdd(&mult[e], 1u);
     }
@@ -150,13 +158,11 @@ __global__ void __launch_bounds__(kPlanThreads) cache_plan_kernel(
                     uslot[e] = slot;
                     uwave[e] = w;
                     uhit[e] = hit ? 1 : 0;
-                    if (mailbox) {
-                        mailbox->expert[i] = e;
-                        mailbox->slot[i] = slot;
-                        mailbox->hit[i] = hit ? 1 : 0;
-                        mailbox->victim[i] = victim;
-                        mailbox->wave[i] = w;
-                    }
+                    mb[i] = e;  // staged; copied to the host mailbox by all threads at the end
+                    mb[E + i] = slot;
+                    mb[2 * E + i] = hit ? 1 : 0;
+                    mb[3 * E + i] = victim;
+                    mb[4 * E + i] = w;
                 }
                 __syncwarp();
             }
@@ -167,6 +173,7 @@ __global__ void __launch_bounds__(kPlanThreads) cache_plan_kernel(
             __syncwarp();
         }
         if (lane == 0) {
+            s_n = n;
             if (mailbox) {
                 mailbox->n_distinct = n;
                 mailbox->n_waves = waves;
@@ -204,22 +211,40 @@ __global__ void __launch_bounds__(kPlanThreads) cache_plan_kernel(
         if (wl_shared.wl) write_decode_worklist(wl_shared, npairs, sl, w, hit);
         if (wl_routed.wl) write_decode_worklist(wl_routed, npairs, sl, w, !hit);
     }
+    // the host's copy of the plan: rows written by all threads at once, then
+    // one system-scope fence and `seq`, which the host polls for
     if (mailbox) {
+        for (int i = threadIdx.x; i < s_n; i += blockDim.x) {
+            mailbox->expert[i] = mb[i];
+            mailbox->slot[i] = mb[E + i];
+            mailbox->hit[i] = mb[2 * E + i];
+            mailbox->victim[i] = mb[3 * E + i];
+            mailbox->wave[i] = mb[4 * E + i];
+        }
         __syncthreads();
         if (threadIdx.x == 0) {
             __threadfence_system();
             *reinterpret_cast<volatile uint32_t*>(&mailbox->seq) = seq;
-            __threadfence_system();
         }
     }
 }
 
-size_t plan_smem_bytes(int E, int S) { return size_t(E) * 4 * 6 + size_t(S) * 4 + 2 * size_t(E) + 16; }
+size_t plan_smem_bytes(int E, int S) { return (size_t(plan_mb_offset_words(E, S)) + 5 * size_t(E)) * 4; }
 
 cudaError_t launch_plan(const int32_t* ids, int npairs, int E, int S, int32_t* state, uint32_t step,
                         int32_t* pair_slot, int32_t* pair_wave, PlanMailbox* mailbox, uint32_t seq, int* status,
                         const float* gate_w, const DecodeWLTarget& wl_shared, const DecodeWLTarget& wl_routed,
                         bool pdl, cudaStream_t s) {
+    static thread_local int attr_set_for = -1;  // device whose attribute this thread last set
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (attr_set_for != dev) {  // up to 51 KB for 1024 experts
+        e = cudaFuncSetAttribute(cache_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(plan_smem_bytes(1024, 1024)));
+        if (e != cudaSuccess) return e;
+        attr_set_for = dev;
+    }
     return launch_kernel(cache_plan_kernel, dim3(1), dim3(kPlanThreads), plan_smem_bytes(E, S), s, pdl, 1, ids, npairs,
                          E, S, state, step, pair_slot, pair_wave, mailbox, seq, status, gate_w, wl_shared, wl_routed);
 }

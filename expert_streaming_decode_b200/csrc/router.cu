@@ -29,7 +29,7 @@ namespace cg = cooperative_groups;
 
 namespace moe {
 
-constexpr int kRouterCtas = 8;
+constexpr int kRouterCtas = 16;  // a non-portable cluster size (B200 allows 16)
 constexpr int kRouterThreads = 512;
 constexpr int kMaxE = 1024;
 constexpr int kMaxK = 16;
@@ -215,21 +215,26 @@ __global__ void __launch_bounds__(kRouterThreads) router_topk_kernel(
     if (rank != 0) return;
 
     // top-K by (logit desc, id asc): every expert counts the experts ranked
-    // above it (shared-memory broadcast reads); ranks 0..K-1 are the selection
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        const float v = logits[e];
-        if (isnan(v)) {
-            s_nan = 1;
-            continue;
-        }
+    // above it, four threads per expert each over every fourth id
+    // (shared-memory broadcast reads); ranks 0..K-1 are the selection
+    for (int eb = 0; eb < E; eb += kRouterThreads / 4) {
+        const int e = eb + int(threadIdx.x >> 2), part = threadIdx.x & 3;
+        const float v = e < E ? logits[e] : 0.f;
         int above = 0;
-        for (int f = 0; f < E; ++f) {
-            const float u = logits[f];
-            above += (u > v) || (u == v && f < e);
+        if (e < E) {
+            for (int f = part; f < E; f += 4) {  // the four threads read four neighbouring words
+                const float u = logits[f];
+                above += (u > v) || (u == v && f < e);
+            }
         }
-        if (above < K) {
-            s_sel_id[above] = e;
-            s_sel_l[above] = v;
+        above += __shfl_xor_sync(0xffffffffu, above, 1);
+        above += __shfl_xor_sync(0xffffffffu, above, 2);
+        if (e < E && part == 0) {
+            if (isnan(v)) s_nan = 1;
+            else if (above < K) {
+                s_sel_id[above] = e;
+                s_sel_l[above] = v;
+            }
         }
     }
     __syncthreads();
@@ -268,6 +273,8 @@ cudaError_t launch_router(const uint16_t* x, const int8_t* wq, const uint16_t* w
     if (e != cudaSuccess) return e;
     if (attr_set_for != dev) {
         e = cudaFuncSetAttribute(router_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kRouterSmemMax));
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(router_topk_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         if (e != cudaSuccess) return e;
         attr_set_for = dev;
     }

@@ -66,7 +66,7 @@ extern "C" {
  * width 704, shared-expert FFN width 2112, quantisation group 64, 16 slots.
  * Supported: d_model % 256 == 0 and d_model <= 8192; d_ff and d_ff_shared
  * multiples of 64 that are <= 704 or multiples of 704 (at most 2112); group ==
- * 64; top_k <= 16; n_experts % 8 == 0 and n_experts <= 1024; top_k <= n_slots
+ * 64; top_k <= 16; n_experts % 16 == 0 and n_experts <= 1024; top_k <= n_slots
  * <= n_experts; 1 <= max_tokens <= 1024.  moe_ctx_create returns MOE_ERR_ARG
  * for anything else. */
 typedef struct moe_dims {

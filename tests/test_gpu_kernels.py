@@ -44,7 +44,7 @@ def test_router_ids_bit_exact(O, d, T, with_bias):
         assert np.max(np.abs(gw[t] - O.gate_weights(lg, want))) <= GATE_TOL
 
 
-@pytest.mark.parametrize("D,E", [(8192, 256), (8192, 1024)], ids=["5-passes", "19-passes"])
+@pytest.mark.parametrize("D,E", [(8192, 256), (8192, 1024)], ids=["3-passes", "10-passes"])
 def test_router_rows_in_passes(O, D, E):
     """Router rows that do not fit shared memory at once are staged in passes
     through two buffers (ragged last pass); ids stay bit-exact."""
