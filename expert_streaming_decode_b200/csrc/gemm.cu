@@ -25,8 +25,8 @@
 //     the no-swizzle K-major core-matrix layout (8 rows x 16 bytes per core
 //     matrix; K-direction core stride 128 B, 8-row stride 1024 B).  An MMA
 //     warp issues 4 MMAs of K = 16 per group and commits them to an mbarrier;
-//     three fp16 buffer sets let the math warps run two groups ahead of the
-//     tensor core.
+//     two fp16 buffer sets let the math warps run a group ahead of the tensor
+//     core, and the raw-weight ring holds 12 groups per CTA.
 //   * gate/up epilogue: TMEM lanes 32w..32w+31 hold one 32-row blob tile (16
 //     gate rows then the 16 matching up rows): h = gelu(g) * u with one shuffle.
 //   * down epilogue: y[token][row] += w * D, fp32 atomics (entries of different
@@ -88,19 +88,19 @@ struct GemmRing;
 template <>
 struct GemmRing<0> {  // gate/up: 4 groups per 256-input chunk, take 2 at a time
     static constexpr int kGroupsPerStage = 2;
-    static constexpr int kStages = 3;
+    static constexpr int kStages = 6;
 };
 template <>
 struct GemmRing<1> {  // down: chunk widths need not be even in groups
     static constexpr int kGroupsPerStage = 1;
-    static constexpr int kStages = 6;
+    static constexpr int kStages = 12;
 };
 template <int MODE>
 __host__ __device__ constexpr int ring_bt_bytes() { return GemmRing<MODE>::kGroupsPerStage * 1152; }
 template <int MODE>
 __host__ __device__ constexpr int ring_stage_bytes() { return 4 * ring_bt_bytes<MODE>(); }
 
-constexpr int kOpBufs = 3;                          // fp16 operand buffer sets (A and B tiles of one group)
+constexpr int kOpBufs = 2;                          // fp16 operand buffer sets (A and B tiles of one group)
 constexpr int kABytes = 128 * 64 * 2;               // A: 128 weight rows x 64 inputs
 constexpr int kBBytes = kGemmMaxRows * 64 * 2;      // B: up to kGemmMaxRows token rows x 64 inputs
 template <int MODE>
@@ -293,11 +293,10 @@ __global__ void __launch_bounds__(kGemmWarps * 32, 2) grouped_gemm_kernel(GemmAr
     // inputs 8*kb .. +7 of the group, with j = 8*(idx/64) + idx%8 and
     // kb = (idx/8)%8: a warp's 16-byte stores then hit 8 different rows of a
     // core matrix (no bank conflicts) and its loads still fill whole sectors.
-    // Rows M..N-1 are zero padding.  Raw loads are kept in registers and
-    // converted one group later, so their latency overlaps a whole group.
+    // Rows M..N-1 are zero padding.  Raw loads are kept in registers, two
+    // groups ahead (two register sets, alternating), and converted when used.
     const int ntasks = 8 * N;
     using Raw = typename std::conditional<MODE == 0, uint4, float4[2]>::type;
-    Raw braw[kBTasks];
     const void* bsrc[kBTasks];  // row base of each task (nullptr: padding row)
 #pragma unroll
     for (int i = 0; i < kBTasks; ++i) {
@@ -308,7 +307,7 @@ __global__ void __launch_bounds__(kGemmWarps * 32, 2) grouped_gemm_kernel(GemmAr
             bsrc[i] = MODE == 0 ? static_cast<const void*>(A.x + size_t(s_rows[j].x_row) * D)
                                 : static_cast<const void*>(A.h + s_rows[j].h_off);
     }
-    auto load_b = [&](int g) {
+    auto load_b = [&](int g, Raw (&braw)[kBTasks]) {
 #pragma unroll
         for (int i = 0; i < kBTasks; ++i) {
             const int idx = tid + kMathThreads * i;
@@ -331,21 +330,19 @@ __global__ void __launch_bounds__(kGemmWarps * 32, 2) grouped_gemm_kernel(GemmAr
             }
         }
     };
-    load_b(0);
     // this thread's weights: row r of the 128 (blob tile 4*tile + r/32, row r%32), inputs 32*hk .. +31 of each group
     const int r = tid & 127, hk = tid >> 7;
     const int bt_row = r >> 5, row = r & 31;
-    bool ok = true;
-    for (int g = 0; g < ngroups && ok; ++g) {
+    // one group: wait for its ring stage and a free buffer set, write B (from
+    // braw, then reload braw with group g + 2) and the dequantised A, arrive
+    auto step = [&](int g, Raw (&braw)[kBTasks]) -> bool {
         const int si = g / GPS, gl = g % GPS, st = si % NST;
         const int b = g % kOpBufs;
         // the buffer set's previous MMAs are done; the ring stage has landed
-        if (g >= kOpBufs) ok = ring_wait_gemm(&freed[b], ((g / kOpBufs) - 1) & 1, A.status, &s_abort);
-        if (ok && gl == 0) ok = ring_wait_gemm(&full[st], (si / NST) & 1, A.status, &s_abort);
-        if (!ok) break;
+        if (g >= kOpBufs && !ring_wait_gemm(&freed[b], ((g / kOpBufs) - 1) & 1, A.status, &s_abort)) return false;
+        if (gl == 0 && !ring_wait_gemm(&full[st], (si / NST) & 1, A.status, &s_abort)) return false;
         uint8_t* a = sA + b * kABytes;
         uint8_t* bt = sB + b * kBBytes;
-        // B: this group's activations (loaded one group ahead), then the next group's loads
 #pragma unroll
         for (int i = 0; i < kBTasks; ++i) {
             const int idx = tid + kMathThreads * i;
@@ -370,7 +367,7 @@ __global__ void __launch_bounds__(kGemmWarps * 32, 2) grouped_gemm_kernel(GemmAr
             const int j = 8 * (idx >> 6) + (idx & 7);
             *reinterpret_cast<uint4*>(bt + core_off(j, 8 * ((idx >> 3) & 7))) = pack_block_perm(v);
         }
-        if (g + 1 < ngroups) load_b(g + 1);
+        if (g + 2 < ngroups) load_b(g + 2, braw);
         // A: dequantise this thread's 32 weights of the group from the raw stage
         {
             const uint8_t* raw = ring + size_t(st) * ST_BYTES + bt_row * BT_BYTES;
@@ -388,6 +385,15 @@ __global__ void __launch_bounds__(kGemmWarps * 32, 2) grouped_gemm_kernel(GemmAr
             mbar_arrive(&ready[b]);
             if (gl == GPS - 1) mbar_arrive(&empty[st]);  // this warp is done with the raw stage
         }
+        return true;
+    };
+    Raw braw0[kBTasks], braw1[kBTasks];
+    load_b(0, braw0);
+    if (ngroups > 1) load_b(1, braw1);
+    bool ok = true;
+    for (int g = 0; g < ngroups && ok; g += 2) {
+        ok = step(g, braw0);
+        if (ok && g + 1 < ngroups) ok = step(g + 1, braw1);
     }
     // every MMA the MMA warp issued has completed
     if (ok) ok = ring_wait_gemm(&done, 0, A.status, &s_abort);
