@@ -567,14 +567,19 @@ __global__ void __launch_bounds__((DecodeCfg<MODE>::NW + 1) * 32) gemv_decode_ke
     // 16-bit fixed-point image of the inputs, one load round trip per kBatch
     // tasks (8 values each) per thread: MODE 0 the token's x (row 0: these
     // lists carry one token), MODE 1 every entry's h segment
-    auto stage = [&](int tasks, const DecodeMap& M) {
+    // task_of maps 0..tasks-1 to the staged task (8 input values) indices;
+    // runs of 8 consecutive flat indices must map to one group, in order
+    auto stage = [&](int tasks, const DecodeMap& M, auto task_of) {
         constexpr int kBatch = 3;
         for (int base = 0; base < tasks; base += kBatch * NCONS) {
             float v[kBatch][8];
+            int tt[kBatch];
 #pragma unroll
             for (int r = 0; r < kBatch; ++r) {  // all loads first: one round trip
-                const int t = base + r * NCONS + int(threadIdx.x);
-                if (t < tasks) {
+                const int fi = base + r * NCONS + int(threadIdx.x);
+                const int t = fi < tasks ? task_of(fi) : 0;
+                tt[r] = t;
+                if (fi < tasks) {
                     if (MODE == 0) {
                         const uint4 q = reinterpret_cast<const uint4*>(A.x)[t];
                         const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
@@ -599,8 +604,8 @@ __global__ void __launch_bounds__((DecodeCfg<MODE>::NW + 1) * 32) gemv_decode_ke
             }
 #pragma unroll
             for (int r = 0; r < kBatch; ++r) {
-                const int t = base + r * NCONS + int(threadIdx.x);
-                stage_task(v[r], t < tasks, t, xq, sx, Xs);
+                const int fi = base + r * NCONS + int(threadIdx.x);
+                stage_task(v[r], fi < tasks, tt[r], xq, sx, Xs);
             }
         }
         named_sync(1, NCONS);
@@ -612,7 +617,7 @@ __global__ void __launch_bounds__((DecodeCfg<MODE>::NW + 1) * 32) gemv_decode_ke
     // known before the wait; the other CTAs wait for the work list
     const bool early = MODE == 0 && c < A.gs;
     if (MODE == 0) {
-        if (warp < NW) stage(D / 8, DecodeMap{});
+        if (warp < NW) stage(D / 8, DecodeMap{}, [](int fi) { return fi; });
         if (!early) {
             pdl_wait();
             pdl_trigger();
@@ -729,9 +734,33 @@ __global__ void __launch_bounds__((DecodeCfg<MODE>::NW + 1) * 32) gemv_decode_ke
 
     // ------------------------------------------------ consumers: stage h (down)
     if (MODE == 1) {
+        // the input segments this CTA's units read (one slice of one entry's
+        // h each), or every entry's h when the range is long
+        constexpr int kMaxUnitsStaged = 16;
+        __shared__ int s_ub[kMaxUnitsStaged], s_uc[kMaxUnitsStaged + 1];
+        const int nu = u_end - u_begin;
+        if (threadIdx.x == 0 && nu <= kMaxUnitsStaged) {
+            s_uc[0] = 0;
+            for (int q = 0; q < nu; ++q) {
+                int e, tile, slice;
+                M.dn_unit(u_begin + q, e, tile, slice);
+                const int ks = down_ks(M.width(e));
+                s_ub[q] = M.stage_chunk0(e) + slice * (ks / 8);
+                s_uc[q + 1] = s_uc[q] + ks / 8;
+            }
+        }
         pdl_wait();  // h is the gate/up kernel's output
         pdl_trigger();
-        stage(M.stage_chunk0(W.n_entries), M);
+        named_sync(1, NCONS);
+        if (nu <= kMaxUnitsStaged) {
+            stage(s_uc[nu], M, [&](int fi) {
+                int q = 0;
+                while (fi >= s_uc[q + 1]) ++q;
+                return s_ub[q] + (fi - s_uc[q]);
+            });
+        } else {
+            stage(M.stage_chunk0(W.n_entries), M, [](int fi) { return fi; });
+        }
     }
 
     // -------------------------------------------------- consumers: the units
