@@ -192,9 +192,10 @@ int max_entries(const moe_dims& d) {
 // K3 (gate/up) and K4 (down + combine) over a work list already on the device.
 // shared_blob: the list's first entry is this shared expert and the gate/up
 // kernel may start it before the list exists (one-token lists only), or null.
+// n_routed_max: most routed entries the list can hold (-1: top_k).
 int run_ffn_list(moe_ctx* c, WorkList* wl, FfnEntry* entries, FfnRow* rows, const uint16_t* x, int T,
                  const float* y_in, float* y, uint16_t* y_bf16, cudaStream_t s,
-                 const uint8_t* shared_blob = nullptr) {
+                 const uint8_t* shared_blob = nullptr, int n_routed_max = -1) {
     cudaError_t e;
     GemvLaunch L;
     L.wl = wl;
@@ -215,7 +216,9 @@ int run_ffn_list(moe_ctx* c, WorkList* wl, FfnEntry* entries, FfnRow* rows, cons
     L.status = c->status;
     L.pdl = c->pdl;
     L.list_cap = c->list_cap;
-    if (T == 1) L.max_tiles_gu = (shared_blob ? c->d.d_ff_shared / 16 : 0) + c->d.top_k * (c->d.d_ff / 16);
+    if (T == 1)
+        L.max_tiles_gu = (shared_blob ? c->d.d_ff_shared / 16 : 0) +
+                         (n_routed_max >= 0 ? n_routed_max : c->d.top_k) * (c->d.d_ff / 16);
     if (T == 1 && shared_blob) {
         L.shared_blob = shared_blob;
         L.FS = c->d.d_ff_shared;
@@ -719,7 +722,9 @@ int moe_layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache* ca
             if (r != MOE_OK) return r;
         }
         if (one) {
-            r = run_ffn_list(c, c->wl2, c->entries2, c->rows2, x, 1, have_y ? y : nullptr, y, y_bf16, s);
+            // list B holds exactly the misses the mailbox reported
+            r = run_ffn_list(c, c->wl2, c->entries2, c->rows2, x, 1, have_y ? y : nullptr, y, y_bf16, s, nullptr,
+                             c->mbox_host->n_misses);
         } else if (gemm) {
             WorkListArgs wa = worklist_args(c, T, K, c->pair_slot, gw, cache->slots, cache->slot_stride,
                                             c->d.n_slots, c->d.d_ff, nullptr);
