@@ -67,16 +67,19 @@ def parse_args():
 
 
 # --------------------------------------------------------------- helpers
-def csrc_sha256():
-    """Hash of the CUDA sources: DRAM traffic recorded under profiles/ is
-    reported only for the kernels it was measured on."""
+# sources of the one-token expert GEMV kernels whose DRAM traffic profiles/traffic.json records
+TRAFFIC_SOURCES = ("ffn.cu", "ffn.cuh", "common.cuh", "decode_wl.cuh", "launch.cuh")
+
+
+def csrc_sha256(files=TRAFFIC_SOURCES):
+    """Hash of the kernel sources: DRAM traffic recorded under profiles/ is
+    reported only for the kernel source it was measured on."""
     import hashlib
     h = hashlib.sha256()
     d = os.path.join(ROOT, "expert_streaming_decode_b200", "csrc")
-    for f in sorted(os.listdir(d)):
-        if f.endswith((".cu", ".cuh")):
-            h.update(f.encode())
-            h.update(open(os.path.join(d, f), "rb").read())
+    for f in sorted(files):
+        h.update(f.encode())
+        h.update(open(os.path.join(d, f), "rb").read())
     return h.hexdigest()
 
 
@@ -88,7 +91,7 @@ def recorded_traffic(key):
     if not os.path.exists(p):
         return None
     rec = json.load(open(p))
-    if rec.get("source_sha256") != csrc_sha256():
+    if rec.get("source_sha256") != csrc_sha256(tuple(rec.get("sources", TRAFFIC_SOURCES))):
         return None
     return rec.get("bytes_per_layer_token", {}).get(key)
 
