@@ -228,7 +228,8 @@ int moe_cache_plan(moe_ctx *ctx, moe_slot_cache *cache, const int32_t *ids, int 
  *              expert passed as top_k = 1, pair_slot 0, gate_w 1)
  *   y_in       dev fp32 [T][D] or NULL; y dev fp32 [T][D] out (may equal y_in)
  *   y_bf16     dev bf16 bits [T][D] out, or NULL
- * 1 <= T <= 32 (larger T: moe_layer_forward's grouped tensor-core path).
+ * 1 <= T <= 32 (dequantising GEMV kernels; moe_layer_forward runs batches on
+ * the grouped tensor-core path instead).
  * Slot indices outside [0, n_slot_range) are clamped and MOE_ERR_RANGE is
  * recorded.  Uses context scratch; calls on one context must not overlap. */
 int moe_expert_ffn(moe_ctx *ctx, const uint16_t *x, int T, int top_k, const int32_t *pair_slot,
@@ -284,9 +285,10 @@ typedef struct moe_layer_weights {
  * cache == NULL: resident mode, expert e read from W->experts + e*stride.
  * cache != NULL: experts are served from cache->slots; misses are copied from
  * cache->store (host-synchronous on the plan, see moe_cache_plan).
- * T <= 32 runs the dequantising GEMV kernels; T > 32 (a prefill chunk) groups
- * the tokens by expert and runs the tcgen05 tensor-core grouped GEMM, one
- * wave of at most n_slots experts at a time.
+ * T = 1 runs the dequantising GEMV kernels; T >= moe_gemm_min_tokens() (a
+ * batched decode step or a prefill chunk) groups the tokens by expert and runs
+ * the tcgen05 tensor-core grouped GEMM, one wave of at most n_slots experts at
+ * a time.
  *   x dev bf16 [T][D]; bias dev fp32 [E] or NULL; y dev fp32 [T][D] out;
  *   y_bf16 dev bf16 [T][D] out or NULL; ids/gate_w dev [T][K] out or NULL;
  *   trace host, or NULL. */

@@ -187,7 +187,7 @@ def test_minimum_slots_equal_top_k(O):
 @pytest.mark.parametrize("d,T", [(TINY, 40), (TINY, 128), (FULL, 37), (FULL, 128)],
                          ids=["tiny-40", "tiny-128", "full-37", "full-128"])
 def test_prefill_resident_tensor_core(O, d, T):
-    """T > 32 runs the tcgen05 grouped GEMM (tokens grouped per expert, fp16
+    """Batches run the tcgen05 grouped GEMM (tokens grouped per expert, fp16
     dequantised weight tiles, fp32 accumulation in tensor memory)."""
     L = Layer(d, layer=4, seed=13, zipf_s=1.1)
     ctx = moe.Ctx.from_dims(d, max_tokens=T)
