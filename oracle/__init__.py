@@ -73,6 +73,9 @@ class Oracle:
         L.orc_lfu_plan.restype = C.c_int
         L.orc_lfu_plan.argtypes = ([C.c_int, C.c_int] + [C.c_void_p] * 5
                                    + [C.c_int, C.c_int, C.c_uint32] + [C.c_void_p] * 7)
+        L.orc_cache_plan.restype = C.c_int
+        L.orc_cache_plan.argtypes = ([C.c_int, C.c_int, C.c_int, C.c_uint32] + [C.c_void_p] * 5
+                                     + [C.c_int, C.c_int, C.c_uint32] + [C.c_void_p] * 7)
         L.orc_group_by_expert.restype = C.c_int
         L.orc_group_by_expert.argtypes = [C.c_void_p, C.c_int, C.c_int, C.c_int,
                                           C.c_void_p, C.c_void_p]
@@ -169,10 +172,17 @@ class Oracle:
         pair_slot = np.full((T, K), -1, dtype=np.int32)
         ue, us, uh, uv, uw = (np.full(E, -1, dtype=np.int32) for _ in range(5))
         nu = C.c_int(0)
-        waves = self.lib.orc_lfu_plan(E, state.S, _p(state.count), _p(state.last_use),
-                                      _p(state.slot_of), _p(state.expert_in),
-                                      _p(ids), T, K, C.c_uint32(step), _p(pair_slot),
-                                      _p(ue), _p(us), _p(uh), _p(uv), _p(uw), C.byref(nu))
+        if state.policy == POLICY_LFU and state.decay_period == 0:
+            waves = self.lib.orc_lfu_plan(E, state.S, _p(state.count), _p(state.last_use),
+                                          _p(state.slot_of), _p(state.expert_in),
+                                          _p(ids), T, K, C.c_uint32(step), _p(pair_slot),
+                                          _p(ue), _p(us), _p(uh), _p(uv), _p(uw), C.byref(nu))
+        else:
+            waves = self.lib.orc_cache_plan(E, state.S, state.policy, C.c_uint32(state.decay_period),
+                                            _p(state.count), _p(state.last_use),
+                                            _p(state.slot_of), _p(state.expert_in),
+                                            _p(ids), T, K, C.c_uint32(step), _p(pair_slot),
+                                            _p(ue), _p(us), _p(uh), _p(uv), _p(uw), C.byref(nu))
         if waves < 0:
             raise ValueError("oracle: expert id out of range")
         n = nu.value
@@ -190,19 +200,24 @@ class Oracle:
         return off, pairs
 
 
-class LfuState:
-    """Caller-owned LFU state of one layer, cold start: counts 0, last_use 0,
-    nothing resident, every slot empty."""
+POLICY_LFU, POLICY_LRU, POLICY_LFU_DECAY, POLICY_LFU_IN_CACHE = 0, 1, 2, 3
 
-    def __init__(self, E: int, S: int):
+
+class LfuState:
+    """Caller-owned cache state of one layer, cold start: counts 0, last_use 0,
+    nothing resident, every slot empty.  `policy` selects the replacement
+    rule (POLICY_*); `decay_period` is used by POLICY_LFU_DECAY."""
+
+    def __init__(self, E: int, S: int, policy: int = POLICY_LFU, decay_period: int = 0):
         self.E, self.S = E, S
+        self.policy, self.decay_period = policy, decay_period
         self.count = np.zeros(E, dtype=np.uint32)
         self.last_use = np.zeros(E, dtype=np.uint32)
         self.slot_of = np.full(E, -1, dtype=np.int32)
         self.expert_in = np.full(S, -1, dtype=np.int32)
 
     def copy(self) -> "LfuState":
-        c = LfuState(self.E, self.S)
+        c = LfuState(self.E, self.S, self.policy, self.decay_period)
         for a in ("count", "last_use", "slot_of", "expert_in"):
             setattr(c, a, getattr(self, a).copy())
         return c

@@ -327,19 +327,37 @@ int orc_moe_token(int D, int E, int K, int F, int FS, int G,
  * Outputs: pair_slot[T*K] (slot holding the pair's expert during its wave),
  * and per distinct expert u (ascending id): u_expert, u_slot, u_hit (1 hit,
  * 0 miss), u_victim (evicted expert or -1), u_wave.  *n_u = number of distinct
- * experts.  Returns the number of waves, or -1 on an out-of-range id. */
-int orc_lfu_plan(int E, int S, uint32_t *count, uint32_t *last_use,
-                 int32_t *slot_of, int32_t *expert_in,
-                 const int32_t *ids, int T, int K, uint32_t step,
-                 int32_t *pair_slot, int32_t *u_expert, int32_t *u_slot,
-                 int32_t *u_hit, int32_t *u_victim, int32_t *u_wave, int *n_u)
+ * experts.  Returns the number of waves, or -1 on an out-of-range id.
+ *
+ * Replacement-policy variants (the pages report that several policies were
+ * compared before LFU was kept; they do not define them, so these readings
+ * are the plain ones), all with the same waves, pinning, empty-slot and
+ * last_use rules:
+ *   ORC_POLICY_LFU        the rule above;
+ *   ORC_POLICY_LRU        victim = smallest (last_use, expert id);
+ *   ORC_POLICY_LFU_DECAY  LFU whose counts are halved (integer shift) at the
+ *                         start of every call whose step is a positive
+ *                         multiple of decay_period, before the call's
+ *                         selections are added;
+ *   ORC_POLICY_LFU_IN_CACHE  LFU whose count of an expert restarts at 0 when
+ *                         it is evicted (frequency while resident). */
+int orc_cache_plan(int E, int S, int policy, uint32_t decay_period,
+                   uint32_t *count, uint32_t *last_use,
+                   int32_t *slot_of, int32_t *expert_in,
+                   const int32_t *ids, int T, int K, uint32_t step,
+                   int32_t *pair_slot, int32_t *u_expert, int32_t *u_slot,
+                   int32_t *u_hit, int32_t *u_victim, int32_t *u_wave, int *n_u)
 {
     int n = 0, waves;
-    unsigned char *sel = (unsigned char *)calloc((size_t)E, 1);
+    unsigned char *sel;
+    if (policy < ORC_POLICY_LFU || policy > ORC_POLICY_LFU_IN_CACHE) return -1;
+    sel = (unsigned char *)calloc((size_t)E, 1);
     for (int p = 0; p < T * K; ++p) {
         if (ids[p] < 0 || ids[p] >= E) { free(sel); return -1; }
         sel[ids[p]] = 1;
     }
+    if (policy == ORC_POLICY_LFU_DECAY && decay_period > 0u && step > 0u && step % decay_period == 0u)
+        for (int e = 0; e < E; ++e) count[e] >>= 1;
     for (int p = 0; p < T * K; ++p) count[ids[p]] += 1u;
     for (int e = 0; e < E; ++e)
         if (sel[e]) u_expert[n++] = e;
@@ -366,7 +384,11 @@ int orc_lfu_plan(int E, int S, uint32_t *count, uint32_t *last_use,
                     for (int j = lo; j < hi; ++j)
                         if (u_expert[j] == r) { pinned = 1; break; }
                     if (pinned) continue;
-                    if (victim < 0 ||
+                    if (policy == ORC_POLICY_LRU) {
+                        if (victim < 0 || last_use[victim] > last_use[r] ||
+                            (last_use[victim] == last_use[r] && victim > r))
+                            victim = r;
+                    } else if (victim < 0 ||
                         count[r] < count[victim] ||
                         (count[r] == count[victim] &&
                          (last_use[r] < last_use[victim] ||
@@ -375,6 +397,7 @@ int orc_lfu_plan(int E, int S, uint32_t *count, uint32_t *last_use,
                 }
                 slot = slot_of[victim];
                 slot_of[victim] = -1;
+                if (policy == ORC_POLICY_LFU_IN_CACHE) count[victim] = 0u;
                 u_victim[i] = victim;
             }
             slot_of[e] = slot;
@@ -390,6 +413,16 @@ int orc_lfu_plan(int E, int S, uint32_t *count, uint32_t *last_use,
     }
     free(sel);
     return waves;
+}
+
+int orc_lfu_plan(int E, int S, uint32_t *count, uint32_t *last_use,
+                 int32_t *slot_of, int32_t *expert_in,
+                 const int32_t *ids, int T, int K, uint32_t step,
+                 int32_t *pair_slot, int32_t *u_expert, int32_t *u_slot,
+                 int32_t *u_hit, int32_t *u_victim, int32_t *u_wave, int *n_u)
+{
+    return orc_cache_plan(E, S, ORC_POLICY_LFU, 0u, count, last_use, slot_of, expert_in, ids, T, K, step,
+                          pair_slot, u_expert, u_slot, u_hit, u_victim, u_wave, n_u);
 }
 
 /* ------------------------------------------------ prefill token grouping

@@ -28,6 +28,18 @@ int orc_moe_token(int D, int E, int K, int F, int FS, int G,
                   const uint8_t *shared_blob, const uint8_t *const *expert_blobs,
                   int32_t *ids, double *gate_w, float *logits, double *y);
 
+#define ORC_POLICY_LFU 0
+#define ORC_POLICY_LRU 1
+#define ORC_POLICY_LFU_DECAY 2
+#define ORC_POLICY_LFU_IN_CACHE 3
+
+int orc_cache_plan(int E, int S, int policy, uint32_t decay_period,
+                   uint32_t *count, uint32_t *last_use,
+                   int32_t *slot_of, int32_t *expert_in,
+                   const int32_t *ids, int T, int K, uint32_t step,
+                   int32_t *pair_slot, int32_t *u_expert, int32_t *u_slot,
+                   int32_t *u_hit, int32_t *u_victim, int32_t *u_wave, int *n_u);
+
 int orc_lfu_plan(int E, int S, uint32_t *count, uint32_t *last_use,
                  int32_t *slot_of, int32_t *expert_in,
                  const int32_t *ids, int T, int K, uint32_t step,

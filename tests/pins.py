@@ -256,10 +256,10 @@ def pin_layer(O):
 
 
 # --------------------------------------------------------------------- LFU
-def _lfu_trace(O, E, S, K, T, steps, seed, zipf=None):
+def _lfu_trace(O, E, S, K, T, steps, seed, zipf=None, policy=0, period=0):
     import oracle
-    st = oracle.LfuState(E, S)
-    sim = NaiveLfu(E, S)
+    st = oracle.LfuState(E, S, policy, period)
+    sim = NaiveLfu(E, S, policy, period)
     rng = np.random.default_rng(seed)
     for step in range(steps):
         if zipf is not None:
@@ -285,6 +285,57 @@ def pin_lfu_naive(O):
     _lfu_trace(O, 32, 8, 4, 3, 60, 1)
     _lfu_trace(O, 24, 5, 3, 6, 25, 2)          # many waves per call
     _lfu_trace(O, 128, 16, 8, 1, 150, 3, zipf=synth.zipf_bias(0, 0, 128))
+
+
+def pin_cache_policies_naive(O):
+    """The LRU, decaying-LFU and in-cache-LFU variants give traces identical
+    to the naive simulator, which recomputes each key from the full history
+    (decay by replaying every call, in-cache frequency by scanning for the
+    last eviction)."""
+    import oracle
+    for pol, per in ((oracle.POLICY_LRU, 0), (oracle.POLICY_LFU_DECAY, 7), (oracle.POLICY_LFU_DECAY, 1),
+                     (oracle.POLICY_LFU_IN_CACHE, 0)):
+        _lfu_trace(O, 16, 6, 4, 1, 100, 10 + pol, policy=pol, period=per)
+        _lfu_trace(O, 24, 5, 3, 6, 20, 20 + pol, policy=pol, period=per)   # several waves per call
+        _lfu_trace(O, 128, 16, 8, 1, 120, 30 + pol, zipf=synth.zipf_bias(0, 0, 128), policy=pol, period=per)
+
+
+def pin_cache_policies_cases(O):
+    """Hand-worked evictions that tell the variants apart (2 slots, 8 experts)."""
+    import oracle
+
+    def run(policy, calls, period=0):
+        st = oracle.LfuState(8, 2, policy, period)
+        r = None
+        for step, ids in calls:
+            r = O.lfu_plan(st, np.array([ids], np.int32), step)
+        return st, r
+    # expert 0 used three times long ago, expert 1 once recently: LFU evicts 1, LRU evicts 0
+    calls = [(0, [0]), (1, [0]), (2, [0]), (3, [1]), (4, [2])]
+    assert run(oracle.POLICY_LFU, calls)[1]["victim"][0] == 1
+    assert run(oracle.POLICY_LRU, calls)[1]["victim"][0] == 0
+    # halving at steps 2 and 4 (period 2): count0 = ((1 + 1) >> 1) + 1 = 2 after step 2, then
+    # 1 at step 4; count1 = 1 after step 3, 0 at step 4; the victim is still 1
+    st, r = run(oracle.POLICY_LFU_DECAY, calls, period=2)
+    assert r["victim"][0] == 1 and st.count[0] == 1 and st.count[1] == 0
+    # decay lets a once-hot expert go: counts 3 (expert 0) vs 2 (expert 1) under LFU; with
+    # period 4 the only halving call is step 12, giving 1 vs 1, and the older last use loses
+    calls = [(0, [0]), (1, [0]), (2, [0]), (10, [1]), (11, [1]), (12, [2])]
+    assert run(oracle.POLICY_LFU, calls)[1]["victim"][0] == 1
+    st, r = run(oracle.POLICY_LFU_DECAY, calls, period=4)
+    assert r["victim"][0] == 0
+    # in-cache: step 3 evicts 1 (count 1 vs 2) and its count restarts at 0; step 5 evicts 2
+    calls = [(0, [0]), (1, [0]), (2, [1]), (3, [2]), (4, [0]), (5, [3])]
+    assert run(oracle.POLICY_LFU, calls)[1]["victim"][0] == 2
+    st, r = run(oracle.POLICY_LFU_IN_CACHE, calls)
+    assert r["victim"][0] == 2 and st.count[1] == 0
+    # in-cache: step 3 evicts 0 (count 1 vs 2), step 4 reloads 0 with count 1 and evicts 2
+    # (count 1 vs 2); step 5 evicts 0 again (count 1 vs 2), while plain LFU (count0 = 2 at
+    # step 4, a tie with 1 broken by recency) keeps 0 and evicts 1 at step 5
+    calls = [(0, [0]), (1, [1]), (2, [1]), (3, [2]), (4, [0]), (5, [3])]
+    st, r = run(oracle.POLICY_LFU_IN_CACHE, calls)
+    assert r["victim"][0] == 0 and st.count[2] == 0
+    assert run(oracle.POLICY_LFU, calls)[1]["victim"][0] == 1
 
 
 def pin_lfu_invariants(O):
@@ -342,4 +393,5 @@ def pin_group_by_expert(O):
 
 ALL_PINS = [pin_binary16, pin_bf16, pin_layout_points, pin_packer_points, pin_dequant_random,
             pin_router_exact, pin_router_random, pin_topk, pin_gate_weights, pin_gelu, pin_ffn,
-            pin_layer, pin_lfu_naive, pin_lfu_invariants, pin_group_by_expert]
+            pin_layer, pin_lfu_naive, pin_cache_policies_naive, pin_cache_policies_cases, pin_lfu_invariants,
+            pin_group_by_expert]

@@ -42,6 +42,12 @@ MUTANTS = {
     "lfu_highest_empty_slot": ("if (expert_in[s] < 0) { slot = s; break; }", "if (expert_in[s] < 0) { slot = s; }"),
     "lfu_counts_per_expert": ("for (int p = 0; p < T * K; ++p) count[ids[p]] += 1u;",
                               "for (int e2 = 0; e2 < E; ++e2) if (sel[e2]) count[e2] += 1u;"),
+    "lru_recency_reversed": ("if (victim < 0 || last_use[victim] > last_use[r] ||",
+                             "if (victim < 0 || last_use[victim] < last_use[r] ||"),
+    "decay_not_halving": ("for (int e = 0; e < E; ++e) count[e] >>= 1;",
+                          "for (int e = 0; e < E; ++e) count[e] >>= 0;"),
+    "in_cache_count_kept": ("if (policy == ORC_POLICY_LFU_IN_CACHE) count[victim] = 0u;",
+                            "if (policy == ORC_POLICY_LFU_IN_CACHE) count[victim] = count[victim];"),
     "group_unstable": ("        for (int p = 0; p < T * K; ++p)\n            if (ids[p] == e) pairs[pos++] = p;",
                        "        for (int p = T * K - 1; p >= 0; --p)\n            if (ids[p] == e) pairs[pos++] = p;"),
 }
