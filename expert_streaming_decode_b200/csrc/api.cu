@@ -384,6 +384,7 @@ int check_cache(const moe_ctx* c, const moe_slot_cache* cache) {
     if (!aligned(cache->slots, 256) || cache->slot_stride % 256 || cache->slot_stride < c->blob_routed) return MOE_ERR_ARG;
     if (!aligned(cache->state, 16)) return MOE_ERR_ARG;
     if (cache->store && cache->store_stride < c->blob_routed) return MOE_ERR_ARG;
+    if (cache->policy < MOE_POLICY_LFU || cache->policy > MOE_POLICY_LFU_IN_CACHE) return MOE_ERR_ARG;
     return MOE_OK;
 }
 
@@ -557,7 +558,8 @@ static int plan_call(moe_ctx* c, moe_slot_cache* cache, const int32_t* ids, int 
                      bool need_host, int* waves, cudaStream_t s) {
     const uint32_t seq = ++c->seq;
     prof_mark(c, MOE_PROF_PLAN, true, s);
-    cudaError_t e = launch_plan(ids, T * c->d.top_k, c->d.n_experts, c->d.n_slots, cache->state, step, pair_slot,
+    cudaError_t e = launch_plan(ids, T * c->d.top_k, c->d.n_experts, c->d.n_slots, cache->policy, cache->decay_period,
+                                cache->state, step, pair_slot,
                                 c->pair_wave, need_host ? c->mbox_dev : nullptr, seq, c->status, nullptr,
                                 DecodeWLTarget{}, DecodeWLTarget{}, c->pdl, s);
     prof_mark(c, MOE_PROF_PLAN, false, s);
@@ -670,7 +672,8 @@ int moe_layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache* ca
                                                     cache->slot_stride, nullptr)
                                     : DecodeWLTarget{};
     prof_mark(c, MOE_PROF_PLAN, true, s);
-    cudaError_t e = launch_plan(id, T * K, c->d.n_experts, c->d.n_slots, cache->state, step, c->pair_slot,
+    cudaError_t e = launch_plan(id, T * K, c->d.n_experts, c->d.n_slots, cache->policy, cache->decay_period,
+                                cache->state, step, c->pair_slot,
                                 c->pair_wave, c->mbox_dev, seq, c->status, gw, t_sh, t_rt, c->pdl, s);
     prof_mark(c, MOE_PROF_PLAN, false, s);
     c->launches += 1;

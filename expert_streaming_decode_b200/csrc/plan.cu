@@ -9,7 +9,8 @@
 // selections so far (kept across evictions); ties by older last use, then
 // lower id; the experts of the current wave are never evicted; empty slots
 // fill lowest first; distinct experts are planned in ascending id, in waves of
-// at most S; last_use = step + 1 after a wave.
+// at most S; last_use = step + 1 after a wave.  Variants of the replacement
+// rule (MOE_POLICY_*): LRU, LFU with periodic halving, in-cache LFU.
 //
 // One CTA per call.  State is staged in shared memory, counts are gathered
 // with shared atomics, and a single warp walks the distinct experts in order;
@@ -31,7 +32,8 @@ constexpr int kPlanThreads = 256;
 __host__ __device__ inline int plan_mb_offset_words(int E, int S) { return 6 * E + S + (2 * E + 3) / 4; }
 
 __global__ void __launch_bounds__(kPlanThreads) cache_plan_kernel(
-    const int32_t* __restrict__ ids, int npairs, int E, int S, int32_t* __restrict__ state, uint32_t step,
+    const int32_t* __restrict__ ids, int npairs, int E, int S, int policy, uint32_t decay_period,
+    int32_t* __restrict__ state, uint32_t step,
     int32_t* __restrict__ pair_slot, int32_t* __restrict__ pair_wave, PlanMailbox* mailbox, uint32_t seq,
     int* status, const float* __restrict__ gate_w, DecodeWLTarget wl_shared, DecodeWLTarget wl_routed) {
     extern __shared__ int32_t psm[];
@@ -57,9 +59,12 @@ __global__ void __launch_bounds__(kPlanThreads) cache_plan_kernel(
 
     // the first pairs' ids load together with the state: one round trip
     const int id_first = int(threadIdx.x) < npairs ? ids[threadIdx.x] : 0;
+    // LFU_DECAY: the counts are halved at the start of a call whose step is a
+    // positive multiple of the period, before its selections are added
+    const bool halve = policy == MOE_POLICY_LFU_DECAY && decay_period > 0u && step > 0u && step % decay_period == 0u;
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         mult[e] = 0;
-        count[e] = g_count[e];
+        count[e] = halve ? (uint32_t(g_count[e]) >> 1) : uint32_t(g_count[e]);
         last[e] = g_last[e];
         slot_of[e] = g_slot_of[e];
         uslot[e] = -1;
@@ -115,14 +120,16 @@ __global__ void __launch_bounds__(kPlanThreads) cache_plan_kernel(
                         if (b) slot = base + __ffs(b) - 1;
                     }
                     if (slot < 0) {
-                        // victim: smallest (count, last_use, id) among resident, not in this wave
+                        // victim: smallest (count, last_use, id) among resident, not in
+                        // this wave; LRU drops the count from the key
                         uint32_t bc = 0xffffffffu, bl = 0xffffffffu;
                         int br = 0x7fffffff;
                         for (int s = lane; s < S; s += 32) {
                             const int r = expert_in[s];
                             if (r < 0 || r >= E || inwave[r]) continue;
-                            if (count[r] < bc || (count[r] == bc && (last[r] < bl || (last[r] == bl && r < br)))) {
-                                bc = count[r]; bl = last[r]; br = r;
+                            const uint32_t cr = policy == MOE_POLICY_LRU ? 0u : count[r];
+                            if (cr < bc || (cr == bc && (last[r] < bl || (last[r] == bl && r < br)))) {
+                                bc = cr; bl = last[r]; br = r;
                             }
                         }
 #pragma unroll
@@ -146,7 +153,10 @@ __global__ void __launch_bounds__(kPlanThreads) cache_plan_kernel(
                     }
                     __syncwarp();
                     if (lane == 0) {
-                        if (victim >= 0) slot_of[victim] = -1;
+                        if (victim >= 0) {
+                            slot_of[victim] = -1;
+                            if (policy == MOE_POLICY_LFU_IN_CACHE) count[victim] = 0u;  // restarts when evicted
+                        }
                         const int prev = expert_in[slot];
                         if (prev >= 0 && prev < E && prev != victim) slot_of[prev] = -1;
                         slot_of[e] = slot;
@@ -231,7 +241,8 @@ __global__ void __launch_bounds__(kPlanThreads) cache_plan_kernel(
 
 size_t plan_smem_bytes(int E, int S) { return (size_t(plan_mb_offset_words(E, S)) + 5 * size_t(E)) * 4; }
 
-cudaError_t launch_plan(const int32_t* ids, int npairs, int E, int S, int32_t* state, uint32_t step,
+cudaError_t launch_plan(const int32_t* ids, int npairs, int E, int S, int policy, uint32_t decay_period,
+                        int32_t* state, uint32_t step,
                         int32_t* pair_slot, int32_t* pair_wave, PlanMailbox* mailbox, uint32_t seq, int* status,
                         const float* gate_w, const DecodeWLTarget& wl_shared, const DecodeWLTarget& wl_routed,
                         bool pdl, cudaStream_t s) {
@@ -246,7 +257,8 @@ cudaError_t launch_plan(const int32_t* ids, int npairs, int E, int S, int32_t* s
         attr_set_for = dev;
     }
     return launch_kernel(cache_plan_kernel, dim3(1), dim3(kPlanThreads), plan_smem_bytes(E, S), s, pdl, 1, ids, npairs,
-                         E, S, state, step, pair_slot, pair_wave, mailbox, seq, status, gate_w, wl_shared, wl_routed);
+                         E, S, policy, decay_period, state, step, pair_slot, pair_wave, mailbox, seq, status, gate_w,
+                         wl_shared, wl_routed);
 }
 
 __global__ void cache_reset_kernel(int32_t* state, int E, int S) {

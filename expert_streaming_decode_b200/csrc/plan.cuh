@@ -22,7 +22,8 @@ struct PlanMailbox {
 size_t plan_smem_bytes(int E, int S);
 // `wl_shared` / `wl_routed` (wl == nullptr: skip): one-token work lists of the
 // shared-expert phase and of the routed phase, written when npairs <= 32 (T = 1).
-cudaError_t launch_plan(const int32_t* ids, int npairs, int E, int S, int32_t* state, uint32_t step,
+cudaError_t launch_plan(const int32_t* ids, int npairs, int E, int S, int policy, uint32_t decay_period,
+                        int32_t* state, uint32_t step,
                         int32_t* pair_slot, int32_t* pair_wave, PlanMailbox* mailbox, uint32_t seq, int* status,
                         const float* gate_w, const DecodeWLTarget& wl_shared, const DecodeWLTarget& wl_routed,
                         bool pdl, cudaStream_t s);

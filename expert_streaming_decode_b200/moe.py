@@ -36,7 +36,11 @@ class moe_dims(C.Structure):
 
 class moe_slot_cache(C.Structure):
     _fields_ = [("slots", C.c_void_p), ("slot_stride", C.c_size_t), ("state", C.c_void_p),
-                ("store", C.c_void_p), ("store_stride", C.c_size_t)]
+                ("store", C.c_void_p), ("store_stride", C.c_size_t), ("policy", C.c_int32),
+                ("decay_period", C.c_uint32)]
+
+
+MOE_POLICY_LFU, MOE_POLICY_LRU, MOE_POLICY_LFU_DECAY, MOE_POLICY_LFU_IN_CACHE = 0, 1, 2, 3
 
 
 class moe_layer_weights(C.Structure):
@@ -179,11 +183,12 @@ def router_topk(ctx: Ctx, x, wq, ws, bias, T, ids, gate_w, stream=None):
                                _stream(stream)), "moe_router_topk")
 
 
-def slot_cache(slots, slot_stride, state, store=None, store_stride=0) -> moe_slot_cache:
+def slot_cache(slots, slot_stride, state, store=None, store_stride=0, policy=MOE_POLICY_LFU,
+               decay_period=0) -> moe_slot_cache:
     """moe_slot_cache for torch tensors.  The struct keeps references to the
     tensors, so their memory lives at least as long as the struct."""
     c = moe_slot_cache(slots.data_ptr(), slot_stride, state.data_ptr(),
-                       None if store is None else store.data_ptr(), store_stride)
+                       None if store is None else store.data_ptr(), store_stride, policy, decay_period)
     c._keep = (slots, state, store)
     return c
 

@@ -163,14 +163,35 @@ int moe_router_topk(moe_ctx *ctx, const uint16_t *x, const int8_t *wq, const uin
  *                 store + e*store_stride; NULL = no backing store (the plan
  *                 is computed but nothing is copied: slots must be filled
  *                 by the caller)
- *   store_stride  bytes, >= moe_blob_bytes(D, F)  */
+ *   store_stride  bytes, >= moe_blob_bytes(D, F)
+ *   policy        replacement rule (MOE_POLICY_*; 0 = LFU, the pages' rule)
+ *   decay_period  MOE_POLICY_LFU_DECAY: counts are halved at the start of
+ *                 every call whose step is a positive multiple of it (0: never)
+ * A zero-initialised struct field selects LFU without decay. */
 typedef struct moe_slot_cache {
     uint8_t *slots;
     size_t slot_stride;
     int32_t *state;
     const uint8_t *store;
     size_t store_stride;
+    int32_t policy;
+    uint32_t decay_period;
 } moe_slot_cache;
+
+/* Replacement rules of the slot cache ("El milagro ...", "Mas inteligente
+ * que tu RAM": a miss replaces the least frequently used resident expert; the
+ * other rules are the variants compared against it).  All share the waves,
+ * the pinning of the current wave's experts and the empty-slot rule:
+ *   LFU          victim = smallest (count, last_use, id); count = selections
+ *                so far, kept across evictions
+ *   LRU          victim = smallest (last_use, id)
+ *   LFU_DECAY    LFU with counts halved (integer shift) at the start of every
+ *                call whose step is a positive multiple of decay_period
+ *   LFU_IN_CACHE LFU whose count of an expert restarts at 0 when evicted */
+#define MOE_POLICY_LFU          0
+#define MOE_POLICY_LRU          1
+#define MOE_POLICY_LFU_DECAY    2
+#define MOE_POLICY_LFU_IN_CACHE 3
 
 /* int32 words of LFU state per layer: count[E], last_use[E], slot_of[E],
  * expert_in[S]. */

@@ -91,15 +91,15 @@ def test_router_ties_and_nan(O):
 
 
 # -------------------------------------------------------------- cache plan
-def _plan_sequence(O, d, S, T, steps, seed, zipf=True):
+def _plan_sequence(O, d, S, T, steps, seed, zipf=True, policy=0, period=0):
     E, K = d.E, d.K
     ctx = moe.Ctx(d.D, E, K, d.F, d.FS, S, max_tokens=max(T, 1))
     state = torch.empty(ctx.state_words(), dtype=torch.int32, device="cuda")
     slots = torch.empty((S, 256), dtype=torch.uint8, device="cuda")  # plan only: slots never read
-    cache = moe.slot_cache(slots, 256, state)
+    cache = moe.slot_cache(slots, 256, state, policy=policy, decay_period=period)
     cache.slot_stride = synth.blob_bytes(d.D, d.F) + 255 & ~255
     moe.cache_reset(ctx, cache)
-    ost = oracle.LfuState(E, S)
+    ost = oracle.LfuState(E, S, policy, period)
     rng = np.random.default_rng(seed)
     zb = synth.zipf_bias(seed, 0, E) if zipf else np.zeros(E)
     ps = torch.empty((T, K), dtype=torch.int32, device="cuda")
@@ -126,6 +126,29 @@ def _plan_sequence(O, d, S, T, steps, seed, zipf=True):
 @pytest.mark.parametrize("S,T,steps", [(16, 1, 300), (8, 1, 200), (64, 1, 200), (16, 4, 80), (16, 128, 6), (8, 32, 10)])
 def test_cache_plan_trace_bit_exact(O, S, T, steps):
     _plan_sequence(O, FULL, S, T, steps, seed=S * 1000 + T)
+
+
+@pytest.mark.parametrize("policy,period", [(moe.MOE_POLICY_LRU, 0), (moe.MOE_POLICY_LFU_DECAY, 16),
+                                           (moe.MOE_POLICY_LFU_DECAY, 1), (moe.MOE_POLICY_LFU_IN_CACHE, 0)],
+                         ids=["lru", "decay16", "decay1", "in-cache"])
+@pytest.mark.parametrize("S,T,steps", [(16, 1, 300), (16, 128, 6)], ids=["decode", "prefill-waves"])
+def test_cache_policy_traces_bit_exact(O, policy, period, S, T, steps):
+    """Replacement-rule variants: traces, pair slots and the final state equal
+    the oracle's bit for bit."""
+    _plan_sequence(O, FULL, S, T, steps, seed=S * 1000 + T + 7 * policy, policy=policy, period=period)
+
+
+def test_cache_policy_rejected_when_unknown():
+    d = TINY
+    ctx = moe.Ctx.from_dims(d, max_tokens=1)
+    state = torch.empty(ctx.state_words(), dtype=torch.int32, device="cuda")
+    slots = torch.empty((d.S, 256), dtype=torch.uint8, device="cuda")
+    cache = moe.slot_cache(slots, 256, state, policy=7)
+    cache.slot_stride = synth.blob_bytes(d.D, d.F) + 255 & ~255
+    ids = torch.zeros((1, d.K), dtype=torch.int32, device="cuda")
+    ps = torch.empty((1, d.K), dtype=torch.int32, device="cuda")
+    with pytest.raises(moe.MoeError):
+        moe.cache_plan(ctx, cache, ids, 1, 0, ps, None)
 
 
 def test_cache_plan_tiny_uniform(O):

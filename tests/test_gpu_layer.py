@@ -68,19 +68,19 @@ def test_batched_decode_resident(O, d, T):
     assert np.array_equal(yb.cpu().numpy().view(np.uint16), synth.to_bf16_bits(y_h))
 
 
-def _streaming(O, d, layers, tokens, S, check_y_every=1, T=1):
+def _streaming(O, d, layers, tokens, S, check_y_every=1, T=1, policy=0, period=0):
     Ls = [Layer(d, layer=l, seed=1, zipf_s=1.1, resident=False, pinned=True) for l in range(layers)]
     ctx = moe.Ctx.from_dims(d, max_tokens=T, S=S)
     caches, states, slotbufs = [], [], []
     for L in Ls:
         state = torch.empty(ctx.state_words(), dtype=torch.int32, device="cuda")
         slots = torch.empty((S, L.stride), dtype=torch.uint8, device="cuda")
-        c = moe.slot_cache(slots, L.stride, state, L.store_t, L.stride)
+        c = moe.slot_cache(slots, L.stride, state, L.store_t, L.stride, policy=policy, decay_period=period)
         moe.cache_reset(ctx, c)
         caches.append(c)
         states.append(state)
         slotbufs.append(slots)
-    ost = [oracle.LfuState(d.E, S) for _ in Ls]
+    ost = [oracle.LfuState(d.E, S, policy, period) for _ in Ls]
     y = torch.empty((T, d.D), dtype=torch.float32, device="cuda")
     ids = torch.empty((T, d.K), dtype=torch.int32, device="cuda")
     gw = torch.empty((T, d.K), dtype=torch.float32, device="cuda")
@@ -176,6 +176,14 @@ def test_resident_no_shared_expert(O):
     ctx.sync()
     for t in range(2):
         _check_token(O, L, xb[t], ids.cpu().numpy()[t], gw.cpu().numpy()[t], y.cpu().numpy()[t])
+
+
+@pytest.mark.parametrize("policy,period", [(moe.MOE_POLICY_LRU, 0), (moe.MOE_POLICY_LFU_DECAY, 5),
+                                           (moe.MOE_POLICY_LFU_IN_CACHE, 0)], ids=["lru", "decay5", "in-cache"])
+def test_streaming_decode_policies(O, policy, period):
+    """Whole streamed layers under the replacement-rule variants: traces,
+    slot contents and outputs against the oracle."""
+    _streaming(O, TINY, layers=2, tokens=30, S=6, policy=policy, period=period)
 
 
 def test_minimum_slots_equal_top_k(O):
