@@ -52,6 +52,9 @@ def parse_args():
     p.add_argument("--sweep-tokens", type=int, default=4096)
     p.add_argument("--batch", type=int, default=1)
     p.add_argument("--slots", type=int, default=16)
+    p.add_argument("--policy", choices=["lfu", "lru", "lfu_decay", "lfu_in_cache"], default="lfu",
+                   help="slot-cache replacement rule of the streamed workloads (default lfu, the pages' rule)")
+    p.add_argument("--decay-period", type=int, default=64, help="lfu_decay: halve the counts every N steps")
     p.add_argument("--zipf", type=float, default=None,
                    help="Zipf exponent of the router popularity bias (default 1.1; 0 = uniform router, "
                         "the default for decode_resident)")
@@ -229,7 +232,11 @@ class Model:
             self.store = store
             self.slots = [torch.empty((self.S, self.stride), dtype=torch.uint8, device=dev) for _ in range(self.L)]
             self.state = [torch.empty(self.ctx.state_words(), dtype=torch.int32, device=dev) for _ in range(self.L)]
-            self.caches = [moe.slot_cache(self.slots[l], self.stride, self.state[l], store[l], self.stride)
+            pol = {"lfu": moe.MOE_POLICY_LFU, "lru": moe.MOE_POLICY_LRU, "lfu_decay": moe.MOE_POLICY_LFU_DECAY,
+                   "lfu_in_cache": moe.MOE_POLICY_LFU_IN_CACHE}[getattr(args, "policy", "lfu")]
+            per = getattr(args, "decay_period", 0) if pol == moe.MOE_POLICY_LFU_DECAY else 0
+            self.caches = [moe.slot_cache(self.slots[l], self.stride, self.state[l], store[l], self.stride,
+                                          policy=pol, decay_period=per)
                            for l in range(self.L)]
             self.W = [moe.layer_weights(self.wq[l], self.ws[l], self.shared[l]) for l in range(self.L)]
         else:
@@ -384,7 +391,10 @@ class OracleDecoder:
                      for l in range(self.L)]
         self.shared = {}
         self.blobs = {}
-        self.lfu = [oracle.LfuState(dims.E, args.slots) for _ in range(self.L)]
+        pol = {"lfu": oracle.POLICY_LFU, "lru": oracle.POLICY_LRU, "lfu_decay": oracle.POLICY_LFU_DECAY,
+               "lfu_in_cache": oracle.POLICY_LFU_IN_CACHE}[getattr(args, "policy", "lfu")]
+        per = getattr(args, "decay_period", 0) if pol == oracle.POLICY_LFU_DECAY else 0
+        self.lfu = [oracle.LfuState(dims.E, args.slots, pol, per) for _ in range(self.L)]
         self.tok, self.layer = 0, 0
         self.x = synth.hidden(args.seed, 0, 0, dims.D)
         self.r = synth.bf16_bits_to_f32(self.x).astype(np.float64)
@@ -487,34 +497,44 @@ def run_sweep(args, dims, dist):
         blk = np.stack([synth.hidden(args.seed, tok, l, d.D) for l in range(args.layers)])
         xs_all[tok].copy_(torch.from_numpy(blk.view(np.int16)))
     gen_s = time.time() - t0
+    def plan_point(S, zs, policy=moe.MOE_POLICY_LFU, period=0):
+        """Router + cache plan over Tn tokens x all layers: hit rate and H2D bytes per token."""
+        ctx = moe.Ctx.from_dims(d, max_tokens=1, S=S)
+        bias = [torch.from_numpy(synth.zipf_bias(args.seed, l, d.E, s=zs)).cuda() for l in range(args.layers)]
+        states = [torch.empty(ctx.state_words(), dtype=torch.int32, device="cuda") for _ in range(args.layers)]
+        slots = torch.empty((S, 256), dtype=torch.uint8, device="cuda")  # plan only: never read
+        caches = []
+        for st in states:
+            c = moe.slot_cache(slots, (nb + 255) // 256 * 256, st, policy=policy, decay_period=period)
+            moe.cache_reset(ctx, c)
+            caches.append(c)
+        ids = torch.empty((1, d.K), dtype=torch.int32, device="cuda")
+        gw = torch.empty((1, d.K), dtype=torch.float32, device="cuda")
+        ps = torch.empty((1, d.K), dtype=torch.int32, device="cuda")
+        tr = moe.Trace(d.E)
+        hits = misses = 0
+        t0 = time.time()
+        for tok in range(Tn):
+            for l in range(args.layers):
+                moe.router_topk(ctx, xs_all[tok, l:l + 1], wq[l], ws[l], bias[l], 1, ids, gw)
+                moe.cache_plan(ctx, caches[l], ids, 1, tok, ps, tr)
+                r = tr.result()
+                misses += r["misses"]
+                hits += r["n_distinct"] - r["misses"]
+        ctx.sync()
+        ctx.close()
+        return {"slots": S, "zipf_s": zs, "hit_rate": hits / max(1, hits + misses),
+                "h2d_bytes_per_token": misses * nb / Tn, "plan_seconds": time.time() - t0}
+
     for S in (8, 16, 32, 64):
         for zs in (0.8, 1.1, 1.4):
-            ctx = moe.Ctx.from_dims(d, max_tokens=1, S=S)
-            bias = [torch.from_numpy(synth.zipf_bias(args.seed, l, d.E, s=zs)).cuda() for l in range(args.layers)]
-            states = [torch.empty(ctx.state_words(), dtype=torch.int32, device="cuda") for _ in range(args.layers)]
-            slots = torch.empty((S, 256), dtype=torch.uint8, device="cuda")  # plan only: never read
-            caches = []
-            for st in states:
-                c = moe.slot_cache(slots, (nb + 255) // 256 * 256, st)
-                moe.cache_reset(ctx, c)
-                caches.append(c)
-            ids = torch.empty((1, d.K), dtype=torch.int32, device="cuda")
-            gw = torch.empty((1, d.K), dtype=torch.float32, device="cuda")
-            ps = torch.empty((1, d.K), dtype=torch.int32, device="cuda")
-            tr = moe.Trace(d.E)
-            hits = misses = 0
-            t0 = time.time()
-            for tok in range(Tn):
-                for l in range(args.layers):
-                    moe.router_topk(ctx, xs_all[tok, l:l + 1], wq[l], ws[l], bias[l], 1, ids, gw)
-                    moe.cache_plan(ctx, caches[l], ids, 1, tok, ps, tr)
-                    r = tr.result()
-                    misses += r["misses"]
-                    hits += r["n_distinct"] - r["misses"]
-            ctx.sync()
-            results.append({"slots": S, "zipf_s": zs, "hit_rate": hits / max(1, hits + misses),
-                            "h2d_bytes_per_token": misses * nb / Tn, "plan_seconds": time.time() - t0})
-            ctx.close()
+            results.append(plan_point(S, zs))
+    # replacement-rule variants at Zipf 1.1 (hit rate and H2D bytes; tokens/s follows the bytes)
+    policies = []
+    for name, pol, per in (("lru", moe.MOE_POLICY_LRU, 0), ("lfu_decay_64", moe.MOE_POLICY_LFU_DECAY, 64),
+                           ("lfu_in_cache", moe.MOE_POLICY_LFU_IN_CACHE, 0)):
+        for S in (8, 16, 32):
+            policies.append({"policy": name, **plan_point(S, 1.1, pol, per)})
     # tokens/s at each point from a short streamed decode (one store for all)
     store = None
     for res in results:
@@ -538,8 +558,8 @@ def run_sweep(args, dims, dist):
                 "ms_per_step": 1e3 / base["tokens_per_s"], "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f32", "data": "synthetic",
                 "config": {"workload": "sweep", "layers": args.layers, "sweep_tokens": Tn,
-                           "value_point": "slots 16, zipf 1.1", "hidden_state_generation_s": gen_s},
-                "sweep": results}
+                           "value_point": "slots 16, zipf 1.1, LFU", "hidden_state_generation_s": gen_s},
+                "sweep": results, "policies": policies}
         print(json.dumps(line), flush=True)
     return 0
 
@@ -605,6 +625,8 @@ def main():
             "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic"}
     cfg = {"workload": args.workload, "layers": args.layers, "batch": T, "slots": args.slots if streaming else None,
+           "cache_policy": (args.policy + (f"_{args.decay_period}" if args.policy == "lfu_decay" else ""))
+           if streaming else None,
            "zipf_s": args.zipf, "tokens_per_rank": ntok * T, "parallelism": f"replicas x{dist.world}",
            "l2": ("working set > L2: 30 layers x (16 slots + shared) = 1.9 GB in HBM plus a 12.85 GB pinned store"
                   if streaming else "working set > L2: 12.85 GB of resident experts")}
