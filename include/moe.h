@@ -179,8 +179,9 @@ typedef struct moe_slot_cache {
 } moe_slot_cache;
 
 /* Replacement rules of the slot cache ("El milagro ...", "Mas inteligente
- * que tu RAM": a miss replaces the least frequently used resident expert; the
- * other rules are the variants compared against it).  All share the waves,
+ * que tu RAM": a miss replaces the least frequently used resident expert;
+ * "Gemma 4 26B en ~2 GB de RAM ...", "La parte que se gana la confianza":
+ * other cache policies were measured against it).  All share the waves,
  * the pinning of the current wave's experts and the empty-slot rule:
  *   LFU          victim = smallest (count, last_use, id); count = selections
  *                so far, kept across evictions

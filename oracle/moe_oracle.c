@@ -329,10 +329,10 @@ int orc_moe_token(int D, int E, int K, int F, int FS, int G,
  * 0 miss), u_victim (evicted expert or -1), u_wave.  *n_u = number of distinct
  * experts.  Returns the number of waves, or -1 on an out-of-range id.
  *
- * Replacement-policy variants (the pages report that several policies were
- * compared before LFU was kept; they do not define them, so these readings
- * are the plain ones), all with the same waves, pinning, empty-slot and
- * last_use rules:
+ * Replacement-policy variants ([yodev] "La parte que se gana la confianza":
+ * the project logged which cache policies lost to LFU, without defining
+ * them; these readings are the plain ones), all with the same waves,
+ * pinning, empty-slot and last_use rules:
  *   ORC_POLICY_LFU        the rule above;
  *   ORC_POLICY_LRU        victim = smallest (last_use, expert id);
  *   ORC_POLICY_LFU_DECAY  LFU whose counts are halved (integer shift) at the
