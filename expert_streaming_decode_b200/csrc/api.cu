@@ -21,6 +21,7 @@
 
 #include "common.cuh"
 #include "ffn.cuh"
+#include "filestore.cuh"
 #include "plan.cuh"
 #include <cstdlib>
 
@@ -78,6 +79,7 @@ struct moe_ctx {
     uint64_t launches = 0;
     size_t blob_routed = 0;
     size_t blob_shared = 0;
+    FileReader reader;  // file-backed stores: staging buffers and reader threads
     // instrumentation (moe_ctx_profile)
     struct Rec {
         int kind;
@@ -364,6 +366,26 @@ int fill_wave(moe_ctx* c, const moe_slot_cache* cache, int w, cudaEvent_t after,
     const size_t nb = c->blob_routed;
     if (cudaStreamWaitEvent(c->side, after, 0) != cudaSuccess) return MOE_ERR_CUDA;
     prof_mark(c, MOE_PROF_H2D, true, c->side);
+    if (cache->source == MOE_SOURCE_FILE) {
+        // read each missed blob (whole 4 KB pages, so O_DIRECT descriptors work)
+        // into a staging buffer, copy it to its slot as soon as it is read
+        const size_t len = (nb + 4095) / 4096 * 4096 <= cache->store_stride ? (nb + 4095) / 4096 * 4096 : nb;
+        std::vector<FileRead> reads;
+        for (int i = 0; i < mb->n_distinct; ++i) {
+            if (mb->wave[i] != w || mb->hit[i]) continue;
+            const int e = mb->expert[i], sl = mb->slot[i];
+            if (e < 0 || e >= c->d.n_experts || sl < 0 || sl >= c->d.n_slots) return MOE_ERR_RANGE;
+            reads.push_back(FileRead{cache->store_fd, cache->store_file_offset + uint64_t(e) * cache->store_stride, len,
+                                     nb, cache->slots + size_t(sl) * cache->slot_stride});
+        }
+        int r = c->reader.ensure((nb + 4095) / 4096 * 4096, c->d.n_slots < 16 ? c->d.n_slots : 16);
+        if (r == MOE_OK) r = c->reader.read_and_copy(reads, c->side, 10000, bytes);
+        if (r != MOE_OK) return r;
+        prof_mark(c, MOE_PROF_H2D, false, c->side);
+        if (cudaEventRecord(c->ev_fill, c->side) != cudaSuccess) return MOE_ERR_CUDA;
+        if (cudaStreamWaitEvent(s, c->ev_fill, 0) != cudaSuccess) return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
     for (int i = 0; i < mb->n_distinct; ++i) {
         if (mb->wave[i] != w || mb->hit[i]) continue;
         const int e = mb->expert[i], sl = mb->slot[i];
@@ -379,12 +401,18 @@ int fill_wave(moe_ctx* c, const moe_slot_cache* cache, int w, cudaEvent_t after,
     return MOE_OK;
 }
 
+// the cache has a backing store the misses are copied from
+bool has_store(const moe_slot_cache* cache) { return cache->store || cache->source == MOE_SOURCE_FILE; }
+
 int check_cache(const moe_ctx* c, const moe_slot_cache* cache) {
     if (!cache || !cache->slots || !cache->state) return MOE_ERR_ARG;
     if (!aligned(cache->slots, 256) || cache->slot_stride % 256 || cache->slot_stride < c->blob_routed) return MOE_ERR_ARG;
     if (!aligned(cache->state, 16)) return MOE_ERR_ARG;
     if (cache->store && cache->store_stride < c->blob_routed) return MOE_ERR_ARG;
     if (cache->policy < MOE_POLICY_LFU || cache->policy > MOE_POLICY_LFU_IN_CACHE) return MOE_ERR_ARG;
+    if (cache->source != MOE_SOURCE_HOST && cache->source != MOE_SOURCE_FILE) return MOE_ERR_ARG;
+    if (cache->source == MOE_SOURCE_FILE && (cache->store_fd < 0 || cache->store_stride < c->blob_routed))
+        return MOE_ERR_ARG;
     return MOE_OK;
 }
 
@@ -408,6 +436,7 @@ const char* moe_status_str(int s) {
         case MOE_ERR_STATE: return "invalid state";
         case MOE_ERR_NAN: return "NaN router logit";
         case MOE_ERR_RANGE: return "index out of range";
+        case MOE_ERR_IO: return "expert file read failed";
         default: return "unknown status";
     }
 }
@@ -580,12 +609,12 @@ int moe_cache_plan(moe_ctx* c, moe_slot_cache* cache, const int32_t* ids, int T,
     if (T < 1 || T > c->d.max_tokens) return MOE_ERR_ARG;
     int r = check_cache(c, cache);
     if (r != MOE_OK) return r;
-    const bool need_host = cache->store || trace;
+    const bool need_host = has_store(cache) || trace;
     int waves = 0;
     r = plan_call(c, cache, ids, T, step, pair_slot, need_host, &waves, s);
     if (r != MOE_OK) return r;
     uint64_t bytes = 0;
-    if (cache->store && waves == 1) {
+    if (has_store(cache) && waves == 1) {
         r = fill_wave(c, cache, 0, c->ev_plan, s, &bytes);
         if (r != MOE_OK) return r;
     }
@@ -714,7 +743,7 @@ int moe_layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache* ca
     uint64_t bytes = 0;
     for (int w = 0; w < waves; ++w) {
         if (one && c->mbox_host->n_misses == 0) break;  // everything hit: list A was the whole layer
-        if (cache->store) {
+        if (has_store(cache)) {
             // wave w's victims may be slots wave w-1 still reads: copy after it
             cudaEvent_t after = c->ev_plan;
             if (w > 0) {

@@ -21,6 +21,7 @@ if not os.path.exists(LIB_PATH):
 lib = C.CDLL(LIB_PATH)
 
 MOE_OK, MOE_ERR_ARG, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE_ERR_STATE, MOE_ERR_NAN, MOE_ERR_RANGE = 0, -1, -2, -3, -4, -5, -6
+MOE_ERR_IO = -7
 
 
 class MoeError(RuntimeError):
@@ -37,7 +38,11 @@ class moe_dims(C.Structure):
 class moe_slot_cache(C.Structure):
     _fields_ = [("slots", C.c_void_p), ("slot_stride", C.c_size_t), ("state", C.c_void_p),
                 ("store", C.c_void_p), ("store_stride", C.c_size_t), ("policy", C.c_int32),
-                ("decay_period", C.c_uint32)]
+                ("decay_period", C.c_uint32), ("source", C.c_int32), ("store_fd", C.c_int32),
+                ("store_file_offset", C.c_uint64)]
+
+
+MOE_SOURCE_HOST, MOE_SOURCE_FILE = 0, 1
 
 
 MOE_POLICY_LFU, MOE_POLICY_LRU, MOE_POLICY_LFU_DECAY, MOE_POLICY_LFU_IN_CACHE = 0, 1, 2, 3
@@ -184,11 +189,15 @@ def router_topk(ctx: Ctx, x, wq, ws, bias, T, ids, gate_w, stream=None):
 
 
 def slot_cache(slots, slot_stride, state, store=None, store_stride=0, policy=MOE_POLICY_LFU,
-               decay_period=0) -> moe_slot_cache:
+               decay_period=0, store_fd=None, store_file_offset=0) -> moe_slot_cache:
     """moe_slot_cache for torch tensors.  The struct keeps references to the
-    tensors, so their memory lives at least as long as the struct."""
+    tensors, so their memory lives at least as long as the struct.  With
+    store_fd (an open file descriptor) the misses are read from that file at
+    store_file_offset + e * store_stride instead of the pinned `store`."""
+    src = MOE_SOURCE_HOST if store_fd is None else MOE_SOURCE_FILE
     c = moe_slot_cache(slots.data_ptr(), slot_stride, state.data_ptr(),
-                       None if store is None else store.data_ptr(), store_stride, policy, decay_period)
+                       None if store is None else store.data_ptr(), store_stride, policy, decay_period,
+                       src, -1 if store_fd is None else store_fd, store_file_offset)
     c._keep = (slots, state, store)
     return c
 

@@ -60,6 +60,7 @@ extern "C" {
 #define MOE_ERR_STATE    -4  /* call not valid in the context's current state */
 #define MOE_ERR_NAN      -5  /* a router logit was NaN: no top-k order exists */
 #define MOE_ERR_RANGE    -6  /* an expert id or slot index out of range reached a kernel */
+#define MOE_ERR_IO       -7  /* reading an expert from a file-backed store failed or came up short */
 
 /* ------------------------------------------------------------------ shapes
  * Gemma 4 26B-A4B MoE layer: d_model 2816, 128 experts, top-8, expert FFN
@@ -167,7 +168,17 @@ int moe_router_topk(moe_ctx *ctx, const uint16_t *x, const int8_t *wq, const uin
  *   policy        replacement rule (MOE_POLICY_*; 0 = LFU, the pages' rule)
  *   decay_period  MOE_POLICY_LFU_DECAY: counts are halved at the start of
  *                 every call whose step is a positive multiple of it (0: never)
- * A zero-initialised struct field selects LFU without decay. */
+ *   source        MOE_SOURCE_HOST (the pinned `store` above) or
+ *                 MOE_SOURCE_FILE: expert e is read from file descriptor
+ *                 store_fd at byte store_file_offset + e*store_stride with
+ *                 positional reads, several in flight, into pinned staging
+ *                 buffers of the context, then copied to its slot ("Gemma 4
+ *                 26B en ~2 GB de RAM ...", "Por que pread y no mmap").  For a
+ *                 descriptor opened with O_DIRECT, store_stride and
+ *                 store_file_offset must be multiples of 4096.  The caller
+ *                 owns the descriptor; a read that fails or comes up short is
+ *                 MOE_ERR_IO.
+ * A zero-initialised struct's new fields select LFU, no decay, host store. */
 typedef struct moe_slot_cache {
     uint8_t *slots;
     size_t slot_stride;
@@ -176,7 +187,13 @@ typedef struct moe_slot_cache {
     size_t store_stride;
     int32_t policy;
     uint32_t decay_period;
+    int32_t source;
+    int32_t store_fd;
+    uint64_t store_file_offset;
 } moe_slot_cache;
+
+#define MOE_SOURCE_HOST 0
+#define MOE_SOURCE_FILE 1
 
 /* Replacement rules of the slot cache ("El milagro ...", "Mas inteligente
  * que tu RAM": a miss replaces the least frequently used resident expert;

@@ -6,6 +6,8 @@ batched decode, and a 128-token prefill chunk with cold caches.
 Inputs are seeded generator hidden states for every (token, layer), so the
 oracle and the GPU see identical inputs; ids and cache traces must match bit
 for bit, outputs within max|y - r| <= 2e-3 * max|r|."""
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -68,14 +70,28 @@ def test_batched_decode_resident(O, d, T):
     assert np.array_equal(yb.cpu().numpy().view(np.uint16), synth.to_bf16_bits(y_h))
 
 
-def _streaming(O, d, layers, tokens, S, check_y_every=1, T=1, policy=0, period=0):
+def _streaming(O, d, layers, tokens, S, check_y_every=1, T=1, policy=0, period=0, file_dir=None):
     Ls = [Layer(d, layer=l, seed=1, zipf_s=1.1, resident=False, pinned=True) for l in range(layers)]
     ctx = moe.Ctx.from_dims(d, max_tokens=T, S=S)
     caches, states, slotbufs = [], [], []
-    for L in Ls:
+    fds = []
+    for li, L in enumerate(Ls):
         state = torch.empty(ctx.state_words(), dtype=torch.int32, device="cuda")
         slots = torch.empty((S, L.stride), dtype=torch.uint8, device="cuda")
-        c = moe.slot_cache(slots, L.stride, state, L.store_t, L.stride, policy=policy, decay_period=period)
+        if file_dir is not None:
+            # the layer's experts in a file at a 4 KB-aligned stride, after a 4 KB header
+            fstride = (L.nb + 4095) // 4096 * 4096
+            path = os.path.join(file_dir, f"layer{li}.experts")
+            with open(path, "wb") as f:
+                f.write(b"\0" * 4096)
+                for e in range(d.E):
+                    f.write(L.blobs[e].tobytes() + b"\0" * (fstride - L.nb))
+            fd = os.open(path, os.O_RDONLY)
+            fds.append(fd)
+            c = moe.slot_cache(slots, L.stride, state, None, fstride, policy=policy, decay_period=period,
+                               store_fd=fd, store_file_offset=4096)
+        else:
+            c = moe.slot_cache(slots, L.stride, state, L.store_t, L.stride, policy=policy, decay_period=period)
         moe.cache_reset(ctx, c)
         caches.append(c)
         states.append(state)
@@ -113,6 +129,8 @@ def _streaming(O, d, layers, tokens, S, check_y_every=1, T=1, policy=0, period=0
                 for s_, e_ in enumerate(ost[l].expert_in):
                     if e_ >= 0:
                         assert np.array_equal(sl[s_, :L.nb], L.blobs[e_]), (step, l, s_, e_)
+    for fd in fds:
+        os.close(fd)
     return hits, misses
 
 
@@ -184,6 +202,42 @@ def test_streaming_decode_policies(O, policy, period):
     """Whole streamed layers under the replacement-rule variants: traces,
     slot contents and outputs against the oracle."""
     _streaming(O, TINY, layers=2, tokens=30, S=6, policy=policy, period=period)
+
+
+def test_streaming_decode_from_file(O, tmp_path):
+    """Misses read from per-layer expert files with positional reads into
+    pinned staging, then copied to the slots: traces, slot contents and
+    outputs as with the pinned host store."""
+    _streaming(O, TINY, layers=2, tokens=30, S=6, file_dir=str(tmp_path))
+    _streaming(O, FULL, layers=1, tokens=6, S=16, check_y_every=3, file_dir=str(tmp_path))
+
+
+def test_prefill_chunk_from_file(O, tmp_path):
+    """A 4-token batch through the file store with waves (more distinct experts than slots)."""
+    _streaming(O, TINY, layers=1, tokens=3, S=6, T=4, file_dir=str(tmp_path))
+
+
+def test_file_store_short_file_is_an_io_error(tmp_path):
+    d = TINY
+    L = Layer(d, layer=0, seed=1, zipf_s=1.1, resident=False, pinned=False)
+    ctx = moe.Ctx.from_dims(d, max_tokens=1, S=6)
+    state = torch.empty(ctx.state_words(), dtype=torch.int32, device="cuda")
+    slots = torch.empty((6, L.stride), dtype=torch.uint8, device="cuda")
+    path = os.path.join(str(tmp_path), "short.experts")
+    with open(path, "wb") as f:
+        f.write(b"\1" * 4096)            # far shorter than E blobs
+    fd = os.open(path, os.O_RDONLY)
+    try:
+        c = moe.slot_cache(slots, L.stride, state, None, L.stride, store_fd=fd)
+        moe.cache_reset(ctx, c)
+        x = bf16_tensor(synth.hidden(1, 0, 0, d.D)[None])
+        y = torch.empty((1, d.D), dtype=torch.float32, device="cuda")
+        with pytest.raises(moe.MoeError) as ei:
+            moe.layer_forward(ctx, L.weights(resident=False), c, x, 1, 0, L.bias_t, y)
+        assert ei.value.code == moe.MOE_ERR_IO
+    finally:
+        os.close(fd)
+    ctx.sync()
 
 
 def test_minimum_slots_equal_top_k(O):
