@@ -720,7 +720,8 @@ def main():
     line["roofline"] = {"bound": "hbm", "kernel": f"{kname} ({dom})",
                         "achieved": ach, "peak": hbm_peak,
                         "unit": "GB/s", "frac": ach / hbm_peak,
-                        "traffic": recorded_traffic(f"{args.workload}:{dom}"),
+                        # recorded for the one-token GEMV kernels only
+                        "traffic": recorded_traffic(f"{args.workload}:{dom}") if not gemm else None,
                         "traffic_unit": "DRAM bytes per layer-token (ncu, profiles/traffic.json)",
                         "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
                         else "fallback 6650 GB/s"}
