@@ -239,7 +239,7 @@ class Model:
             pol = {"lfu": moe.MOE_POLICY_LFU, "lru": moe.MOE_POLICY_LRU, "lfu_decay": moe.MOE_POLICY_LFU_DECAY,
                    "lfu_in_cache": moe.MOE_POLICY_LFU_IN_CACHE}[getattr(args, "policy", "lfu")]
             per = getattr(args, "decay_period", 0) if pol == moe.MOE_POLICY_LFU_DECAY else 0
-            self.fds = []
+            self.fds, self.files = [], []
             if getattr(args, "store_file", None):
                 # one file per layer, experts at a 4 KB-aligned stride (O_DIRECT-compatible)
                 fstride = (self.nb + 4095) // 4096 * 4096
@@ -252,6 +252,7 @@ class Model:
                         for e in range(dims.E):
                             f.write(view[l, e, :self.nb].tobytes())
                             f.write(pad)
+                    self.files.append(path)
                     flags = os.O_RDONLY | (os.O_DIRECT if args.direct else 0)
                     self.fds.append(os.open(path, flags))
                 self.caches = [moe.slot_cache(self.slots[l], self.stride, self.state[l], None, fstride,
@@ -268,6 +269,14 @@ class Model:
             self.caches = [None] * self.L
             self.W = [moe.layer_weights(self.wq[l], self.ws[l], self.shared[l], self.experts[l], self.stride)
                       for l in range(self.L)]
+
+    def close_files(self):
+        """Closes and deletes the expert files this run wrote (--store-file)."""
+        for fd in getattr(self, "fds", []):
+            os.close(fd)
+        for path in getattr(self, "files", []):
+            os.remove(path)
+        self.fds, self.files = [], []
 
     def reset(self):
         if self.streaming:
@@ -776,6 +785,7 @@ def main():
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
     model.ctx.close()
+    model.close_files()
     dist.close()
     return 0
 
