@@ -59,6 +59,8 @@ def parse_args():
                    help="streamed workloads: write each layer's experts to DIR/layerNN.experts and read misses "
                         "from those files with positional reads (the file-backed store)")
     p.add_argument("--direct", action="store_true", help="--store-file: open the files with O_DIRECT")
+    p.add_argument("--prefetch", type=int, default=0, metavar="P",
+                   help="decode_stream: stage up to P of the next layer's predicted misses (look-ahead; 0 = off)")
     p.add_argument("--zipf", type=float, default=None,
                    help="Zipf exponent of the router popularity bias (default 1.1; 0 = uniform router, "
                         "the default for decode_resident)")
@@ -70,6 +72,10 @@ def parse_args():
     a = p.parse_args()
     if a.zipf is None:
         a.zipf = 0.0 if a.workload == "decode_resident" else 1.1
+    if a.prefetch and (a.workload != "decode_stream" or a.batch != 1 or a.store_file):
+        p.error("--prefetch needs the one-token decode_stream workload with the pinned host store")
+    if not 0 <= a.prefetch <= 16:
+        p.error("--prefetch takes 0..16 buffers")
     return a
 
 
@@ -263,7 +269,15 @@ class Model:
                                               policy=pol, decay_period=per)
                                for l in range(self.L)]
             self.W = [moe.layer_weights(self.wq[l], self.ws[l], self.shared[l]) for l in range(self.L)]
+            self.nexts = None
+            if getattr(args, "prefetch", 0) > 0:
+                # layer l stages layer l+1's predicted misses; the last layer has
+                # no successor within the token
+                moe.prefetch_configure(self.ctx, args.prefetch)
+                self.nexts = [moe.next_layer(self.W[l + 1], self.caches[l + 1], self.bias[l + 1])
+                              for l in range(self.L - 1)] + [None]
         else:
+            self.nexts = None
             self.experts = store.to(dev)
             del store
             self.caches = [None] * self.L
@@ -297,6 +311,11 @@ class Model:
         return (self.d.D // 32) * (F // ks) * 18 * ks
 
 
+def moe_prefetch_stats(model):
+    """(issued, used) look-ahead bytes so far; zeros when prefetch is off."""
+    return model.moe.prefetch_stats(model.ctx) if model.nexts is not None else (0, 0)
+
+
 def decode_token(model, x0, r, x, y, T, tok, tr=None, trace_acc=None):
     """One decode step: T tokens through every layer (layer l+1 reads the
     residual stream after layer l, RMS-normalised)."""
@@ -304,7 +323,11 @@ def decode_token(model, x0, r, x, y, T, tok, tr=None, trace_acc=None):
     moe.bf16_to_f32(ctx, x0, r, T * d.D)
     cur = x0
     for l in range(model.L):
-        moe.layer_forward(ctx, model.W[l], model.caches[l], cur, T, tok, model.bias[l], y, trace=tr)
+        if model.nexts is not None and T == 1:
+            moe.layer_forward_next(ctx, model.W[l], model.caches[l], cur, T, tok, model.bias[l], y, model.nexts[l],
+                                   trace=tr)
+        else:
+            moe.layer_forward(ctx, model.W[l], model.caches[l], cur, T, tok, model.bias[l], y, trace=tr)
         if tr is not None:
             res = tr.c
             trace_acc["misses"] += res.n_misses
@@ -672,8 +695,10 @@ def main():
     if not args.profile:
         clocks.start()
     acc_t = {"misses": 0, "distinct": 0, "h2d": 0}
+    pf0 = moe_prefetch_stats(model)
     ms, launches = timed(dist, model, lambda: runner.run(x_dev, K, W, trace_acc=acc_t if streaming else None))
     clk = clocks.stop() if not args.profile else None
+    pf1 = moe_prefetch_stats(model)
 
     # ---- kernel timing pass: event pairs around every kernel (this serialises
     # the kernels, so it is kept out of the pass above)
@@ -697,6 +722,7 @@ def main():
     cfg = {"workload": args.workload, "layers": args.layers, "batch": T, "slots": args.slots if streaming else None,
            "cache_policy": (args.policy + (f"_{args.decay_period}" if args.policy == "lfu_decay" else ""))
            if streaming else None,
+           "prefetch_buffers": args.prefetch if streaming else None,
            "store": (("file, O_DIRECT" if args.direct else "file, page cache") if args.store_file else "pinned host memory")
            if streaming else None,
            "zipf_s": args.zipf, "tokens_per_rank": ntok * T, "parallelism": f"replicas x{dist.world}",
@@ -765,6 +791,14 @@ def main():
                                                 "4 threads" + (", O_DIRECT" if args.direct else ", page cache")}
         line["hit_rate"] = 1.0 - acc_t["misses"] / max(1, acc_t["distinct"])
         line["misses_per_token"] = acc_t["misses"] / (K * T)
+        if model.nexts is not None:
+            iss, used = pf1[0] - pf0[0], pf1[1] - pf0[1]
+            line["prefetch"] = {"buffers": args.prefetch, "issued_bytes_per_token": iss / (K * T),
+                                "used_bytes_per_token": used / (K * T),
+                                "wasted_bytes_per_token": (iss - used) / (K * T),
+                                "miss_bytes_served": used / max(1, acc_t["h2d"]),
+                                "note": "measured over the timed pass; the misses' trace bytes include the ones "
+                                        "filled from staged blobs (device-to-device)"}
     line["gpu_launches"] = int(dist.sum(launches))
     if clk:
         line["clocks"] = clk

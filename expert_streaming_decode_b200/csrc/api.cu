@@ -17,6 +17,7 @@
 #include <cstdio>
 #include <cstring>
 #include <new>
+#include <unordered_map>
 #include <vector>
 
 #include "common.cuh"
@@ -80,6 +81,25 @@ struct moe_ctx {
     size_t blob_routed = 0;
     size_t blob_shared = 0;
     FileReader reader;  // file-backed stores: staging buffers and reader threads
+    // look-ahead prefetch (moe_prefetch_configure / moe_layer_forward_next)
+    int pf_n = 0;                          // HBM blob buffers
+    uint8_t* pf_buf = nullptr;             // [pf_n][pf_stride]
+    size_t pf_stride = 0;
+    int32_t* pf_ids_host = nullptr;        // pinned mapped: the next layer's predicted ids
+    int32_t* pf_ids_dev = nullptr;
+    float* pf_gw = nullptr;                // device scratch: their gate weights
+    cudaStream_t pf_stream = nullptr;
+    cudaEvent_t ev_x = nullptr, ev_pred = nullptr;
+    struct Prefetched {
+        const int32_t* state;  // the cache the blob was fetched for
+        const uint8_t* store;  // and the store it was copied from
+        int expert, buf;
+    };
+    std::vector<Prefetched> pf_table;      // blobs now held by the buffers
+    uint64_t pf_issued = 0, pf_used = 0;   // bytes
+    // host mirror of each cache's residency (slot of expert e, -1: absent),
+    // kept from the plans the host reads; decides what is worth prefetching
+    std::unordered_map<const int32_t*, std::vector<int16_t>> mirror;
     // instrumentation (moe_ctx_profile)
     struct Rec {
         int kind;
@@ -119,6 +139,14 @@ cudaError_t dalloc(T** p, size_t n) {
 
 void free_ctx(moe_ctx* c) {
     if (!c) return;
+    if (c->pf_stream) cudaStreamSynchronize(c->pf_stream);
+    if (c->side) cudaStreamSynchronize(c->side);
+    cudaFree(c->pf_buf);
+    cudaFree(c->pf_gw);
+    if (c->pf_ids_host) cudaFreeHost(c->pf_ids_host);
+    if (c->ev_x) cudaEventDestroy(c->ev_x);
+    if (c->ev_pred) cudaEventDestroy(c->ev_pred);
+    if (c->pf_stream) cudaStreamDestroy(c->pf_stream);
     for (auto& r : c->recs) {
         cudaEventDestroy(r.a);
         cudaEventDestroy(r.b);
@@ -390,15 +418,41 @@ int fill_wave(moe_ctx* c, const moe_slot_cache* cache, int w, cudaEvent_t after,
         if (mb->wave[i] != w || mb->hit[i]) continue;
         const int e = mb->expert[i], sl = mb->slot[i];
         if (e < 0 || e >= c->d.n_experts || sl < 0 || sl >= c->d.n_slots) return MOE_ERR_RANGE;
-        if (cudaMemcpyAsync(cache->slots + size_t(sl) * cache->slot_stride, cache->store + size_t(e) * cache->store_stride,
-                            nb, cudaMemcpyHostToDevice, c->side) != cudaSuccess)
-            return MOE_ERR_CUDA;
+        uint8_t* dst = cache->slots + size_t(sl) * cache->slot_stride;
+        // a blob prefetched for this cache is moved from its HBM buffer (the
+        // prefetch copy is earlier on the same side stream)
+        int pb = -1;
+        for (const auto& f : c->pf_table)
+            if (f.state == cache->state && f.store == cache->store && f.expert == e) pb = f.buf;
+        const cudaError_t ce =
+            pb >= 0 ? cudaMemcpyAsync(dst, c->pf_buf + size_t(pb) * c->pf_stride, nb, cudaMemcpyDeviceToDevice, c->side)
+                    : cudaMemcpyAsync(dst, cache->store + size_t(e) * cache->store_stride, nb, cudaMemcpyHostToDevice,
+                                      c->side);
+        if (ce != cudaSuccess) return MOE_ERR_CUDA;
+        if (pb >= 0) c->pf_used += nb;
         *bytes += nb;
     }
     prof_mark(c, MOE_PROF_H2D, false, c->side);
     if (cudaEventRecord(c->ev_fill, c->side) != cudaSuccess) return MOE_ERR_CUDA;
     if (cudaStreamWaitEvent(s, c->ev_fill, 0) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
+}
+
+// Residency mirror of a cache, updated from a plan the host has read.
+std::vector<int16_t>& mirror_of(moe_ctx* c, const int32_t* state) {
+    auto& m = c->mirror[state];
+    if (m.empty()) m.assign(size_t(c->d.n_experts), int16_t(-1));
+    return m;
+}
+void mirror_update(moe_ctx* c, const moe_slot_cache* cache) {
+    auto& m = mirror_of(c, cache->state);
+    const PlanMailbox* mb = c->mbox_host;
+    for (int i = 0; i < mb->n_distinct; ++i) {
+        if (mb->hit[i]) continue;
+        const int e = mb->expert[i], v = mb->victim[i], sl = mb->slot[i];
+        if (v >= 0 && v < c->d.n_experts) m[size_t(v)] = -1;
+        if (e >= 0 && e < c->d.n_experts) m[size_t(e)] = int16_t(sl);
+    }
 }
 
 // the cache has a backing store the misses are copied from
@@ -577,6 +631,7 @@ int moe_router_topk(moe_ctx* c, const uint16_t* x, const int8_t* wq, const uint1
 
 int moe_cache_reset(moe_ctx* c, moe_slot_cache* cache, cudaStream_t s) {
     if (!c || !cache || !cache->state) return MOE_ERR_ARG;
+    mirror_of(c, cache->state).assign(size_t(c->d.n_experts), int16_t(-1));
     c->launches += 1;
     return cuda_status(launch_cache_reset(cache->state, c->d.n_experts, c->d.n_slots, c->pdl, s));
 }
@@ -614,6 +669,7 @@ int moe_cache_plan(moe_ctx* c, moe_slot_cache* cache, const int32_t* ids, int T,
     r = plan_call(c, cache, ids, T, step, pair_slot, need_host, &waves, s);
     if (r != MOE_OK) return r;
     uint64_t bytes = 0;
+    if (need_host) mirror_update(c, cache);
     if (has_store(cache) && waves == 1) {
         r = fill_wave(c, cache, 0, c->ev_plan, s, &bytes);
         if (r != MOE_OK) return r;
@@ -641,9 +697,12 @@ int moe_expert_ffn(moe_ctx* c, const uint16_t* x, int T, int top_k, const int32_
     return run_ffn(c, wa, x, T, y_in, y, y_bf16, s);
 }
 
-int moe_layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache* cache, const uint16_t* x, int T,
-                      uint32_t step, const float* bias, float* y, uint16_t* y_bf16, int32_t* ids, float* gate_w,
-                      moe_plan_trace* trace, cudaStream_t s) {
+}  // extern "C"
+
+// the layer; `next` (or null) asks for a look-ahead prefetch of the next layer
+static int layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache* cache, const uint16_t* x, int T,
+                         uint32_t step, const float* bias, float* y, uint16_t* y_bf16, int32_t* ids, float* gate_w,
+                         moe_plan_trace* trace, const moe_next_layer* next, cudaStream_t s) {
     if (!c || !W || !W->router_q || !W->router_s || !x || !y) return MOE_ERR_ARG;
     if (T < 1 || T > c->d.max_tokens) return MOE_ERR_ARG;
     if (!aligned(x, 16) || !aligned(y, 16)) return MOE_ERR_ARG;
@@ -670,6 +729,19 @@ int moe_layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache* ca
         c->launches += 1;
         if (e != cudaSuccess) return MOE_ERR_CUDA;
         return run_ffn_list(c, c->wl, c->entries, c->rows, x, 1, nullptr, y, y_bf16, s, W->shared_blob);
+    }
+    // look-ahead: the next layer's router on this layer's input, on its own
+    // stream, while this layer runs (one token, host stores, buffers configured)
+    const bool prefetch = next && T == 1 && c->pf_n > 0 && next->W && next->W->router_q && next->W->router_s &&
+                          next->cache && next->cache->source == MOE_SOURCE_HOST && next->cache->store;
+    if (prefetch) {
+        if (cudaEventRecord(c->ev_x, s) != cudaSuccess || cudaStreamWaitEvent(c->pf_stream, c->ev_x, 0) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        const cudaError_t pe = launch_router(x, next->W->router_q, next->W->router_s, next->bias, c->d.n_experts,
+                                             c->d.d_model, K, 1, c->pf_ids_dev, c->pf_gw, c->status, DecodeWLTarget{},
+                                             false, c->pf_stream);
+        c->launches += 1;
+        if (pe != cudaSuccess || cudaEventRecord(c->ev_pred, c->pf_stream) != cudaSuccess) return MOE_ERR_CUDA;
     }
     r = moe_router_topk(c, x, W->router_q, W->router_s, bias, T, id, gw, s);
     if (r != MOE_OK) return r;
@@ -739,6 +811,7 @@ int moe_layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache* ca
     }
     r = wait_mailbox(c, seq, 10000);
     if (r != MOE_OK) return r;
+    mirror_update(c, cache);
     const int waves = c->mbox_host->n_waves;
     uint64_t bytes = 0;
     for (int w = 0; w < waves; ++w) {
@@ -777,7 +850,82 @@ int moe_layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache* ca
         c->launches += 1;
         if (launch_f32_to_bf16(y, y_bf16, size_t(T) * c->d.d_model, c->pdl, s) != cudaSuccess) return MOE_ERR_CUDA;
     }
+    if (prefetch) {
+        // the next layer's predicted experts its cache does not hold, in
+        // logit order, after this layer's own copies on the side stream; the
+        // blobs the buffers held before are no longer wanted
+        if (cudaEventSynchronize(c->ev_pred) != cudaSuccess) return MOE_ERR_CUDA;
+        c->pf_table.clear();
+        const auto& m = mirror_of(c, next->cache->state);
+        for (int k = 0; k < K && int(c->pf_table.size()) < c->pf_n; ++k) {
+            const int e = c->pf_ids_host[k];
+            if (e < 0 || e >= c->d.n_experts || m[size_t(e)] >= 0) continue;
+            const int b = int(c->pf_table.size());
+            if (cudaMemcpyAsync(c->pf_buf + size_t(b) * c->pf_stride,
+                                next->cache->store + size_t(e) * next->cache->store_stride, c->blob_routed,
+                                cudaMemcpyHostToDevice, c->side) != cudaSuccess)
+                return MOE_ERR_CUDA;
+            c->pf_table.push_back({next->cache->state, next->cache->store, e, b});
+            c->pf_issued += c->blob_routed;
+        }
+    }
     copy_trace(c->mbox_host, trace, c->blob_routed, bytes);
+    return MOE_OK;
+}
+
+extern "C" {
+
+int moe_layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache* cache, const uint16_t* x, int T,
+                      uint32_t step, const float* bias, float* y, uint16_t* y_bf16, int32_t* ids, float* gate_w,
+                      moe_plan_trace* trace, cudaStream_t s) {
+    return layer_forward(c, W, cache, x, T, step, bias, y, y_bf16, ids, gate_w, trace, nullptr, s);
+}
+
+int moe_layer_forward_next(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache* cache, const uint16_t* x, int T,
+                           uint32_t step, const float* bias, float* y, uint16_t* y_bf16, int32_t* ids, float* gate_w,
+                           moe_plan_trace* trace, const moe_next_layer* next, cudaStream_t s) {
+    if (next && next->cache) {
+        const int r = check_cache(c, next->cache);
+        if (r != MOE_OK) return r;
+    }
+    return layer_forward(c, W, cache, x, T, step, bias, y, y_bf16, ids, gate_w, trace, next, s);
+}
+
+int moe_prefetch_configure(moe_ctx* c, int n_buffers) {
+    if (!c || n_buffers < 0 || n_buffers > 16) return MOE_ERR_ARG;
+    // drop the old buffers once nothing queued can still use them
+    if ((c->side && cudaStreamSynchronize(c->side) != cudaSuccess) ||
+        (c->pf_stream && cudaStreamSynchronize(c->pf_stream) != cudaSuccess))
+        return MOE_ERR_CUDA;
+    cudaFree(c->pf_buf);
+    c->pf_buf = nullptr;
+    c->pf_table.clear();
+    c->pf_n = 0;
+    if (n_buffers == 0) return MOE_OK;
+    bool ok = true;
+    if (!c->pf_stream) {
+        ok = ok && cudaStreamCreateWithFlags(&c->pf_stream, cudaStreamNonBlocking) == cudaSuccess;
+        ok = ok && cudaEventCreateWithFlags(&c->ev_x, cudaEventDisableTiming) == cudaSuccess;
+        ok = ok && cudaEventCreateWithFlags(&c->ev_pred, cudaEventDisableTiming) == cudaSuccess;
+        ok = ok && cudaHostAlloc(reinterpret_cast<void**>(&c->pf_ids_host), sizeof(int32_t) * size_t(c->d.top_k),
+                                 cudaHostAllocMapped) == cudaSuccess;
+        ok = ok && cudaHostGetDevicePointer(reinterpret_cast<void**>(&c->pf_ids_dev), c->pf_ids_host, 0) == cudaSuccess;
+        ok = ok && dalloc(&c->pf_gw, size_t(c->d.top_k)) == cudaSuccess;
+    }
+    c->pf_stride = (c->blob_routed + 255) / 256 * 256;
+    ok = ok && cudaMalloc(reinterpret_cast<void**>(&c->pf_buf), c->pf_stride * size_t(n_buffers)) == cudaSuccess;
+    if (!ok) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    c->pf_n = n_buffers;
+    return MOE_OK;
+}
+
+int moe_prefetch_stats(const moe_ctx* c, uint64_t* issued_bytes, uint64_t* used_bytes) {
+    if (!c) return MOE_ERR_ARG;
+    if (issued_bytes) *issued_bytes = c->pf_issued;
+    if (used_bytes) *used_bytes = c->pf_used;
     return MOE_OK;
 }
 

@@ -56,6 +56,10 @@ class moe_layer_weights(C.Structure):
 _I32P = C.POINTER(C.c_int32)
 
 
+class moe_next_layer(C.Structure):
+    _fields_ = [("W", C.POINTER(moe_layer_weights)), ("cache", C.POINTER(moe_slot_cache)), ("bias", C.c_void_p)]
+
+
 class moe_plan_trace(C.Structure):
     _fields_ = [("capacity", C.c_int32), ("n_distinct", C.c_int32), ("n_waves", C.c_int32),
                 ("n_misses", C.c_int32), ("h2d_bytes", C.c_uint64), ("expert", _I32P), ("slot", _I32P),
@@ -92,6 +96,14 @@ lib.moe_expert_ffn_noalloc.argtypes = [_i, _i, _i, _vp, _vp, _vp, _vp, _sz, _i, 
 lib.moe_layer_forward.restype = _i
 lib.moe_layer_forward.argtypes = [_vp, C.POINTER(moe_layer_weights), C.POINTER(moe_slot_cache), _vp, _i, _u32,
                                   _vp, _vp, _vp, _vp, _vp, C.POINTER(moe_plan_trace), _vp]
+lib.moe_layer_forward_next.restype = _i
+lib.moe_layer_forward_next.argtypes = [_vp, C.POINTER(moe_layer_weights), C.POINTER(moe_slot_cache), _vp, _i, _u32,
+                                       _vp, _vp, _vp, _vp, _vp, C.POINTER(moe_plan_trace), C.POINTER(moe_next_layer),
+                                       _vp]
+lib.moe_prefetch_configure.restype = _i
+lib.moe_prefetch_configure.argtypes = [_vp, _i]
+lib.moe_prefetch_stats.restype = _i
+lib.moe_prefetch_stats.argtypes = [_vp, C.POINTER(C.c_uint64), C.POINTER(C.c_uint64)]
 lib.moe_ctx_profile.restype = _i
 lib.moe_ctx_profile.argtypes = [_vp, _i]
 lib.moe_ctx_profile_read.restype = _i
@@ -261,6 +273,35 @@ def layer_forward(ctx: Ctx, W: moe_layer_weights, cache: moe_slot_cache | None, 
                                  _ptr(bias), _ptr(y), _ptr(y_bf16), _ptr(ids), _ptr(gate_w),
                                  None if trace is None else C.byref(trace.c), _stream(stream)),
            "moe_layer_forward")
+
+
+def next_layer(W: moe_layer_weights, cache: moe_slot_cache, bias=None):
+    """The layer after the one being run, for moe_layer_forward_next (keeps its
+    structures alive with it)."""
+    n = moe_next_layer(C.pointer(W), C.pointer(cache), _ptr(bias))
+    n._keep = (W, cache, bias)
+    return n
+
+
+def layer_forward_next(ctx: Ctx, W: moe_layer_weights, cache: moe_slot_cache, x, T, step, bias, y,
+                       next: moe_next_layer | None, y_bf16=None, ids=None, gate_w=None, trace: Trace | None = None,
+                       stream=None):
+    _check(lib.moe_layer_forward_next(ctx.h, C.byref(W), C.byref(cache), _ptr(x), T, step, _ptr(bias), _ptr(y),
+                                      _ptr(y_bf16), _ptr(ids), _ptr(gate_w),
+                                      None if trace is None else C.byref(trace.c),
+                                      None if next is None else C.byref(next), _stream(stream)),
+           "moe_layer_forward_next")
+
+
+def prefetch_configure(ctx: Ctx, n_buffers: int):
+    _check(lib.moe_prefetch_configure(ctx.h, n_buffers), "moe_prefetch_configure")
+
+
+def prefetch_stats(ctx: Ctx):
+    """(issued_bytes, used_bytes) of the look-ahead prefetch so far."""
+    a, b = C.c_uint64(0), C.c_uint64(0)
+    _check(lib.moe_prefetch_stats(ctx.h, C.byref(a), C.byref(b)), "moe_prefetch_stats")
+    return a.value, b.value
 
 
 def residual_rmsnorm(ctx: Ctx, r, y, x_next, T, stream=None):

@@ -336,6 +336,54 @@ int moe_layer_forward(moe_ctx *ctx, const moe_layer_weights *W, moe_slot_cache *
                       float *y, uint16_t *y_bf16, int32_t *ids, float *gate_w,
                       moe_plan_trace *trace, cudaStream_t stream);
 
+/* ------------------------------------------------- look-ahead prefetch
+ * Opt-in; off unless moe_prefetch_configure gave buffers.  The pages disagree
+ * on whether expert loads can be started a layer early: one says the router
+ * gives a layer of warning ("Gemma 4 26B en ~2 GB de RAM ...", section "Por
+ * que pread y no mmap"); the discussion threads judge speculative expert
+ * prefetch hard, because a layer's routing depends on the previous layers'
+ * output, and note that reading mispredicted experts costs the bandwidth the
+ * real misses need ("Show HN: Motor de codigo abierto ...", section
+ * "Direcciones futuras e ideas de investigacion"; "TurboFieldfare: motor open
+ * source ...", the comment thread).  This path makes the trade measurable:
+ * while layer l runs on x, layer l+1's router is evaluated on the same x on a
+ * separate stream; after layer l's own miss copies, up to n_buffers of its
+ * predicted experts that layer l+1's cache does not hold (as far as the host
+ * has seen from the plans it read) are copied from layer l+1's host store into
+ * HBM staging buffers.  When layer l+1 runs, a miss whose blob is staged is
+ * filled by a device-to-device copy instead of a host copy.  The cache plan,
+ * the trace and the outputs are exactly those of moe_layer_forward; only
+ * where a missed blob is copied from changes.
+ *
+ * Sets the number of HBM staging buffers (0..16; 0 turns prefetch off and
+ * frees them), one expert blob each.  Waits for the context's copy streams.
+ * MOE_ERR_ARG (count out of range), MOE_ERR_CUDA (allocation failed). */
+int moe_prefetch_configure(moe_ctx *ctx, int n_buffers);
+
+/* Bytes copied into the staging buffers so far, and the part of them later
+ * used to fill a miss; issued - used is the bandwidth spent on wrong guesses. */
+int moe_prefetch_stats(const moe_ctx *ctx, uint64_t *issued_bytes, uint64_t *used_bytes);
+
+/* The layer after the one being run: its weights, its cache (which must have
+ * a host store, source MOE_SOURCE_HOST) and its router bias (or NULL). */
+typedef struct moe_next_layer {
+    const moe_layer_weights *W;
+    moe_slot_cache *cache;
+    const float *bias;
+} moe_next_layer;
+
+/* moe_layer_forward, plus the look-ahead prefetch of `next` when T = 1, buffers
+ * are configured and next->cache has a host store; otherwise (next NULL or any
+ * of these missing) exactly moe_layer_forward.  The staged blobs are matched to
+ * a later miss by (cache state, store, expert); a later call that issues new
+ * prefetches drops the old ones.  The host waits for the prediction router
+ * (issued before this layer's own router) after queueing this layer's copies.
+ * Errors: those of moe_layer_forward, and next->cache is checked as any cache. */
+int moe_layer_forward_next(moe_ctx *ctx, const moe_layer_weights *W, moe_slot_cache *cache,
+                           const uint16_t *x, int T, uint32_t step, const float *bias,
+                           float *y, uint16_t *y_bf16, int32_t *ids, float *gate_w,
+                           moe_plan_trace *trace, const moe_next_layer *next, cudaStream_t stream);
+
 /* ------------------------------------------------------ instrumentation */
 #define MOE_PROF_ROUTER    0   /* moe_router_topk kernel */
 #define MOE_PROF_PLAN      1   /* cache-plan kernel */

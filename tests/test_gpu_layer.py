@@ -70,7 +70,8 @@ def test_batched_decode_resident(O, d, T):
     assert np.array_equal(yb.cpu().numpy().view(np.uint16), synth.to_bf16_bits(y_h))
 
 
-def _streaming(O, d, layers, tokens, S, check_y_every=1, T=1, policy=0, period=0, file_dir=None):
+def _streaming(O, d, layers, tokens, S, check_y_every=1, T=1, policy=0, period=0, file_dir=None, prefetch=0,
+               same_x=False, stats=None):
     Ls = [Layer(d, layer=l, seed=1, zipf_s=1.1, resident=False, pinned=True) for l in range(layers)]
     ctx = moe.Ctx.from_dims(d, max_tokens=T, S=S)
     caches, states, slotbufs = [], [], []
@@ -102,11 +103,22 @@ def _streaming(O, d, layers, tokens, S, check_y_every=1, T=1, policy=0, period=0
     gw = torch.empty((T, d.K), dtype=torch.float32, device="cuda")
     tr = moe.Trace(d.E)
     hits = misses = 0
+    if prefetch:
+        moe.prefetch_configure(ctx, prefetch)
+        nexts = [moe.next_layer(Ls[l + 1].weights(resident=False), caches[l + 1], Ls[l + 1].bias_t)
+                 for l in range(layers - 1)] + [None]
+        later_misses = 0  # misses of layers 1.. (the ones a prefetch can serve)
     for step in range(tokens):
         for l, L in enumerate(Ls):
-            xb = synth.hidden_batch(1, range(step * T, step * T + T), l, d.D)
-            moe.layer_forward(ctx, L.weights(resident=False), caches[l], bf16_tensor(xb), T, step, L.bias_t, y,
-                              ids=ids, gate_w=gw, trace=tr)
+            # same_x: every layer of a token sees one input, so the look-ahead
+            # router predicts the next layer's experts exactly
+            xb = synth.hidden_batch(1, range(step * T, step * T + T), 0 if same_x else l, d.D)
+            if prefetch:
+                moe.layer_forward_next(ctx, L.weights(resident=False), caches[l], bf16_tensor(xb), T, step,
+                                       L.bias_t, y, nexts[l], ids=ids, gate_w=gw, trace=tr)
+            else:
+                moe.layer_forward(ctx, L.weights(resident=False), caches[l], bf16_tensor(xb), T, step, L.bias_t, y,
+                                  ids=ids, gate_w=gw, trace=tr)
             ctx.sync()
             got = tr.result()
             ids_h = ids.cpu().numpy()
@@ -120,6 +132,8 @@ def _streaming(O, d, layers, tokens, S, check_y_every=1, T=1, policy=0, period=0
             assert got["misses"] == nmiss and got["h2d_bytes"] == nmiss * L.nb
             hits += int(want["hit"].sum())
             misses += nmiss
+            if prefetch and l > 0:
+                later_misses += nmiss
             if step % check_y_every == 0:
                 for t in range(T):
                     _check_token(O, L, xb[t], ids_h[t], gw.cpu().numpy()[t], y.cpu().numpy()[t])
@@ -131,6 +145,9 @@ def _streaming(O, d, layers, tokens, S, check_y_every=1, T=1, policy=0, period=0
                         assert np.array_equal(sl[s_, :L.nb], L.blobs[e_]), (step, l, s_, e_)
     for fd in fds:
         os.close(fd)
+    if prefetch and stats is not None:
+        stats["issued"], stats["used"] = moe.prefetch_stats(ctx)
+        stats["later_misses"], stats["nb"] = later_misses, Ls[0].nb
     return hits, misses
 
 
@@ -202,6 +219,29 @@ def test_streaming_decode_policies(O, policy, period):
     """Whole streamed layers under the replacement-rule variants: traces,
     slot contents and outputs against the oracle."""
     _streaming(O, TINY, layers=2, tokens=30, S=6, policy=policy, period=period)
+
+
+@pytest.mark.parametrize("d,layers,tokens,S,every", [(TINY, 3, 30, 6, 1), (FULL, 3, 8, 16, 4)],
+                         ids=["tiny", "full"])
+def test_streaming_decode_lookahead_exact(O, d, layers, tokens, S, every):
+    """Look-ahead prefetch with one input per token for every layer: the
+    prediction is then exact, so every miss of layers 1.. is filled from a
+    staged blob and nothing staged is wasted; traces, slot contents and outputs
+    are still those of the oracle."""
+    st = {}
+    _streaming(O, d, layers=layers, tokens=tokens, S=S, check_y_every=every, prefetch=d.K, same_x=True, stats=st)
+    assert st["later_misses"] > 0
+    assert st["issued"] == st["used"] == st["later_misses"] * st["nb"]
+
+
+def test_streaming_decode_lookahead_mispredicted(O):
+    """Look-ahead prefetch with unrelated inputs per layer (mostly wrong
+    guesses, fewer buffers than K): same traces, slots and outputs; the used
+    bytes never exceed the issued ones."""
+    st = {}
+    _streaming(O, TINY, layers=3, tokens=30, S=6, prefetch=3, stats=st)
+    assert 0 < st["issued"] and st["used"] <= st["issued"]
+    assert st["used"] <= st["later_misses"] * st["nb"]
 
 
 def test_streaming_decode_from_file(O, tmp_path):
