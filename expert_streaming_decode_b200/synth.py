@@ -14,6 +14,8 @@ Distributions (the pages' model shape with synthetic values):
   hidden state  bfloat16 (round to nearest even) of N(0, 1)
   Zipf bias     bias_e = -lam * s * ln(1 + pi(e)), pi a seeded per-layer
                 permutation of 0..E-1 (popular experts repeat, as in decode)
+  attention     decode query bfloat16 of N(0, 1) [Hq][hd]; KV cache binary16 of
+                N(0, 1), [Hkv][capacity][hd] for keys and for values
 
 Expert blob layout (the kernel-ready layout both sides read):
   an expert with width D and FFN width F is one contiguous blob of two sections
@@ -36,7 +38,7 @@ import os
 import numpy as np
 
 # draw kinds (part of the seed key)
-_ROUTED, _SHARED, _ROUTER, _HIDDEN, _ZIPF, _IDS = 1, 2, 3, 4, 5, 6
+_ROUTED, _SHARED, _ROUTER, _HIDDEN, _ZIPF, _IDS, _ATTN = 1, 2, 3, 4, 5, 6, 7
 
 
 @dataclasses.dataclass(frozen=True)
@@ -218,3 +220,35 @@ def random_ids(seed, T, K, E, index=0) -> np.ndarray:
     """T rows of K distinct expert ids (for cache-plan tests)."""
     r = _rng(seed, _IDS, 0, index)
     return np.stack([r.choice(E, size=K, replace=False) for _ in range(T)]).astype(np.int32)
+
+
+@dataclasses.dataclass(frozen=True)
+class AttnDims:
+    """Decode-attention shape.  The pages give the layer mix (25 sliding-window
+    layers with a ring KV cache, 5 full-attention layers with linear storage,
+    a 4K context) but no head counts; the head counts, head width and window
+    here are chosen, not taken from the pages."""
+    Hq: int = 16        # query heads
+    Hkv: int = 8        # KV heads (query heads h*Hq/Hkv .. share KV head h)
+    hd: int = 256       # head width
+    window: int = 1024  # ring capacity of a sliding-window layer
+    context: int = 4096  # tokens in the context (linear capacity of a full layer)
+    sliding: int = 25
+    full: int = 5
+
+
+GEMMA4_ATTN = AttnDims()
+
+
+def attn_query(seed, token, layer, Hq, hd) -> np.ndarray:
+    """bf16 bits [Hq][hd] of N(0, 1)."""
+    r = _rng(seed, _ATTN, layer, 2 * token)
+    return to_bf16_bits(r.standard_normal((Hq, hd)).astype(np.float32))
+
+
+def attn_kv(seed, layer, Hkv, cap, hd):
+    """binary16 bits of N(0, 1): (k, v), each [Hkv][cap][hd]."""
+    r = _rng(seed, _ATTN, layer, -1 & 0x7FFFFFFF)
+    k = r.standard_normal((Hkv, cap, hd)).astype(np.float16).view(np.uint16)
+    v = r.standard_normal((Hkv, cap, hd)).astype(np.float16).view(np.uint16)
+    return k, v

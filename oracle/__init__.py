@@ -79,6 +79,8 @@ class Oracle:
         L.orc_group_by_expert.restype = C.c_int
         L.orc_group_by_expert.argtypes = [C.c_void_p, C.c_int, C.c_int, C.c_int,
                                           C.c_void_p, C.c_void_p]
+        L.orc_attn_decode.restype = C.c_int
+        L.orc_attn_decode.argtypes = [C.c_void_p] * 3 + [C.c_int] * 5 + [C.c_double, C.c_void_p]
 
     # scalar helpers -------------------------------------------------------
     def f16_to_f64(self, h: int) -> float:
@@ -198,6 +200,21 @@ class Oracle:
         if rc != 0:
             raise ValueError("oracle: expert id out of range")
         return off, pairs
+
+    def attn_decode(self, q_bf16, k_f16, v_f16, cap: int, n: int, scale: float) -> np.ndarray:
+        """Decode attention of one token: q bf16 bits [Hq][hd], k/v binary16
+        bits [Hkv][cap][hd]; returns fp64 [Hq][hd]."""
+        q = np.ascontiguousarray(q_bf16, dtype=np.uint16)
+        k = np.ascontiguousarray(k_f16, dtype=np.uint16)
+        v = np.ascontiguousarray(v_f16, dtype=np.uint16)
+        Hq, hd = q.shape
+        Hkv = k.shape[0]
+        if k.shape != (Hkv, cap, hd) or v.shape != k.shape:
+            raise ValueError("oracle: k/v must be [Hkv][cap][hd]")
+        o = np.empty((Hq, hd), dtype=np.float64)
+        if self.lib.orc_attn_decode(_p(q), _p(k), _p(v), Hq, Hkv, hd, cap, n, float(scale), _p(o)) != 0:
+            raise ValueError("oracle: bad attention sizes")
+        return o
 
 
 POLICY_LFU, POLICY_LRU, POLICY_LFU_DECAY, POLICY_LFU_IN_CACHE = 0, 1, 2, 3

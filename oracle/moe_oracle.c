@@ -446,3 +446,60 @@ int orc_group_by_expert(const int32_t *ids, int T, int K, int E,
     offsets[E] = pos;
     return 0;
 }
+
+/* ------------------------------------------------ decode attention
+ * The other per-token kernel of the layer loop ([hada] "Proceso de generacion
+ * de tokens": decode attention is an exact split-K/V method; the fp16 KV cache
+ * is a bounded ring for the 25 sliding-window layers and linear storage for the
+ * 5 full-attention layers, as also in [yodev] "Por que funciona: el A4B del
+ * nombre").  "Exact" means that splitting the keys and values into parts and
+ * merging them changes nothing but rounding, so the oracle is softmax attention
+ * itself, written out:
+ *   o[h] = sum_p w[h][p] * v[g][slot(p)],
+ *   w[h] = softmax over p of (scale * q[h] . k[g][slot(p)]),  g = h / (Hq / Hkv).
+ * Readings where the pages are silent: a cache of capacity cap holds position p
+ * in slot p mod cap (a ring; a linear cache has cap >= n, so its slot is p);
+ * the token at position n-1 attends to positions max(0, n - cap) .. n-1, its
+ * own key included (the window is the ring's capacity); query heads that share
+ * a KV head are consecutive.  Layouts: q bf16 [Hq][hd]; k, v binary16
+ * [Hkv][cap][hd]; o fp64 [Hq][hd].  Arithmetic in fp64; the largest score is
+ * subtracted before exponentiating, which leaves the softmax unchanged.
+ * Returns 0, or -1 on bad sizes (n < 1, cap < 1, Hq not a multiple of Hkv). */
+int orc_attn_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                    int Hq, int Hkv, int hd, int cap, int n, double scale, double *o)
+{
+    if (n < 1 || cap < 1 || Hkv < 1 || hd < 1 || Hq < Hkv || Hq % Hkv != 0) return -1;
+    const int grp = Hq / Hkv;
+    const int first = n > cap ? n - cap : 0;
+    const int np = n - first;
+    double *w = (double *)malloc(sizeof(double) * (size_t)np);
+    if (!w) return -1;
+    for (int h = 0; h < Hq; ++h) {
+        const int g = h / grp;
+        const uint16_t *kg = k + (size_t)g * (size_t)cap * (size_t)hd;
+        const uint16_t *vg = v + (size_t)g * (size_t)cap * (size_t)hd;
+        double mx = -INFINITY, z = 0.0;
+        for (int i = 0; i < np; ++i) {
+            const size_t slot = (size_t)((first + i) % cap);
+            double a = 0.0;
+            for (int d = 0; d < hd; ++d)
+                a += (double)orc_bf16_to_f32(q[(size_t)h * hd + d]) * orc_f16_to_f64(kg[slot * hd + d]);
+            w[i] = scale * a;
+            if (w[i] > mx) mx = w[i];
+        }
+        for (int i = 0; i < np; ++i) {
+            w[i] = exp(w[i] - mx);
+            z += w[i];
+        }
+        for (int d = 0; d < hd; ++d) {
+            double acc = 0.0;
+            for (int i = 0; i < np; ++i) {
+                const size_t slot = (size_t)((first + i) % cap);
+                acc += w[i] * orc_f16_to_f64(vg[slot * hd + d]);
+            }
+            o[(size_t)h * hd + d] = acc / z;
+        }
+    }
+    free(w);
+    return 0;
+}

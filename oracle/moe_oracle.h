@@ -48,4 +48,7 @@ int orc_lfu_plan(int E, int S, uint32_t *count, uint32_t *last_use,
 
 int orc_group_by_expert(const int32_t *ids, int T, int K, int E,
                         int32_t *offsets, int32_t *pairs);
+
+int orc_attn_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                    int Hq, int Hkv, int hd, int cap, int n, double scale, double *o);
 #endif

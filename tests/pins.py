@@ -391,7 +391,92 @@ def pin_group_by_expert(O):
         assert np.array_equal(off, np.searchsorted(flat[want], np.arange(E + 1)))
 
 
+# ------------------------------------------------------------ decode attention
+def _attn_case(rng, Hq, Hkv, hd, cap):
+    q = synth.to_bf16_bits(rng.standard_normal((Hq, hd)).astype(np.float32))
+    k = rng.standard_normal((Hkv, cap, hd)).astype(np.float16).view(np.uint16)
+    v = rng.standard_normal((Hkv, cap, hd)).astype(np.float16).view(np.uint16)
+    return q, k, v
+
+
+def _attn_torch(q, k, v, cap, n, scale):
+    """torch's own attention routine on the attended rows, gathered by
+    position (p = max(0, n - cap) .. n - 1 in slot p mod cap), in fp64, with
+    each KV head repeated for its consecutive query heads."""
+    Hq, Hkv = q.shape[0], k.shape[0]
+    pos = np.arange(max(0, n - cap), n)
+    kk = torch.from_numpy(k.view(np.float16)[:, pos % cap].astype(np.float64))
+    vv = torch.from_numpy(v.view(np.float16)[:, pos % cap].astype(np.float64))
+    qq = torch.from_numpy(synth.bf16_bits_to_f32(q).astype(np.float64))
+    kk = kk.repeat_interleave(Hq // Hkv, dim=0)
+    vv = vv.repeat_interleave(Hq // Hkv, dim=0)
+    o = torch.nn.functional.scaled_dot_product_attention(qq[:, None, :], kk, vv, scale=scale)
+    return o[:, 0, :].numpy()
+
+
+def pin_attn_library(O):
+    """Against torch's scaled_dot_product_attention on the explicitly gathered
+    window: GQA head mapping, scale, window bounds, ring slots, normalisation."""
+    rng = np.random.default_rng(11)
+    for Hq, Hkv, hd, cap, n in [(4, 2, 8, 7, 1), (4, 2, 8, 7, 5), (4, 2, 8, 7, 7), (4, 2, 8, 7, 12),
+                                (6, 3, 16, 5, 23), (8, 8, 4, 9, 9), (8, 1, 8, 4, 6), (4, 4, 32, 16, 100)]:
+        q, k, v = _attn_case(rng, Hq, Hkv, hd, cap)
+        scale = 1.0 / math.sqrt(hd) * float(rng.uniform(0.5, 2.0))
+        got = O.attn_decode(q, k, v, cap, n, scale)
+        want = _attn_torch(q, k, v, cap, n, scale)
+        assert np.allclose(got, want, rtol=1e-12, atol=1e-12), (Hq, Hkv, hd, cap, n)
+
+
+def pin_attn_closed_forms(O):
+    rng = np.random.default_rng(12)
+    Hq, Hkv, hd, cap = 4, 2, 8, 6
+    q, k, v = _attn_case(rng, Hq, Hkv, hd, cap)
+    vf = v.view(np.float16).astype(np.float64)
+    kf = k.view(np.float16).astype(np.float64)
+    qf = synth.bf16_bits_to_f32(q).astype(np.float64)
+    # one position: the output is that value row, exactly
+    o = O.attn_decode(q, k, v, cap, 1, 0.3)
+    for h in range(Hq):
+        assert np.array_equal(o[h], vf[h // 2, 0])
+    # a zero query weighs every attended position equally: the mean of the rows
+    z = np.zeros_like(q)
+    o = O.attn_decode(z, k, v, cap, 4, 0.3)
+    for h in range(Hq):
+        assert np.allclose(o[h], vf[h // 2, :4].mean(axis=0), rtol=0, atol=1e-15)
+    # two positions: weight of the newer one = logistic(scale * q . (k1 - k0))
+    o = O.attn_decode(q, k, v, cap, 2, 0.3)
+    for h in range(Hq):
+        g = h // 2
+        a = 1.0 / (1.0 + math.exp(-0.3 * float(qf[h] @ (kf[g, 1] - kf[g, 0]))))
+        assert np.allclose(o[h], (1 - a) * vf[g, 0] + a * vf[g, 1], rtol=0, atol=1e-13)
+    # a ring after wrap-around attends to exactly its cap newest positions: the
+    # same result as a linear cache holding those positions in order
+    n = 3 * cap + 2
+    pos = np.arange(n - cap, n)
+    k_lin = np.ascontiguousarray(k[:, pos % cap])
+    v_lin = np.ascontiguousarray(v[:, pos % cap])
+    ring = O.attn_decode(q, k, v, cap, n, 0.3)
+    lin = O.attn_decode(q, k_lin, v_lin, cap, cap, 0.3)
+    assert np.allclose(ring, lin, rtol=0, atol=1e-13)
+    # one dominant key: its value row, up to exp(-gap)
+    kk = np.zeros((Hkv, cap, hd), dtype=np.float16)
+    kk[:, 2, 0] = 64.0
+    qq = np.zeros((Hq, hd), dtype=np.float32)
+    qq[:, 0] = 1.0
+    o = O.attn_decode(synth.to_bf16_bits(qq), kk.view(np.uint16), v, cap, 5, 1.0)
+    for h in range(Hq):
+        assert np.allclose(o[h], vf[h // 2, 2], rtol=0, atol=1e-20 + 4 * math.exp(-64) * np.abs(vf).max())
+    # sizes the definition rejects: no attended position, an empty cache
+    try:
+        O.attn_decode(q, k, v, cap, 0, 0.3)
+    except ValueError:
+        pass
+    else:
+        raise AssertionError("n < 1 accepted")
+    assert O.lib.orc_attn_decode(None, None, None, Hq, Hkv, hd, 0, 1, 0.3, None) == -1
+
+
 ALL_PINS = [pin_binary16, pin_bf16, pin_layout_points, pin_packer_points, pin_dequant_random,
             pin_router_exact, pin_router_random, pin_topk, pin_gate_weights, pin_gelu, pin_ffn,
             pin_layer, pin_lfu_naive, pin_cache_policies_naive, pin_cache_policies_cases, pin_lfu_invariants,
-            pin_group_by_expert]
+            pin_group_by_expert, pin_attn_library, pin_attn_closed_forms]

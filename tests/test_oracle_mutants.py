@@ -50,6 +50,12 @@ MUTANTS = {
                             "if (policy == ORC_POLICY_LFU_IN_CACHE) count[victim] = count[victim];"),
     "group_unstable": ("        for (int p = 0; p < T * K; ++p)\n            if (ids[p] == e) pairs[pos++] = p;",
                        "        for (int p = T * K - 1; p >= 0; --p)\n            if (ids[p] == e) pairs[pos++] = p;"),
+    "attn_gqa_modulo": ("const int g = h / grp;", "const int g = h % Hkv;"),
+    "attn_scale_dropped": ("w[i] = scale * a;", "w[i] = a;"),
+    "attn_window_short": ("const int first = n > cap ? n - cap : 0;", "const int first = n > cap ? n - cap + 1 : 0;"),
+    "attn_not_normalised": ("o[(size_t)h * hd + d] = acc / z;", "o[(size_t)h * hd + d] = acc;"),
+    "attn_value_slot_linear": ("acc += w[i] * orc_f16_to_f64(vg[slot * hd + d]);",
+                               "acc += w[i] * orc_f16_to_f64(vg[(size_t)i * hd + d]);"),
 }
 
 
