@@ -104,6 +104,10 @@ lib.moe_prefetch_configure.restype = _i
 lib.moe_prefetch_configure.argtypes = [_vp, _i]
 lib.moe_prefetch_stats.restype = _i
 lib.moe_prefetch_stats.argtypes = [_vp, C.POINTER(C.c_uint64), C.POINTER(C.c_uint64)]
+lib.moe_attn_workspace_bytes.restype = _sz
+lib.moe_attn_workspace_bytes.argtypes = [_i, _i]
+lib.moe_attn_decode.restype = _i
+lib.moe_attn_decode.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, C.c_float, _vp, _vp, _sz, _vp]
 lib.moe_ctx_profile.restype = _i
 lib.moe_ctx_profile.argtypes = [_vp, _i]
 lib.moe_ctx_profile_read.restype = _i
@@ -302,6 +306,21 @@ def prefetch_stats(ctx: Ctx):
     a, b = C.c_uint64(0), C.c_uint64(0)
     _check(lib.moe_prefetch_stats(ctx.h, C.byref(a), C.byref(b)), "moe_prefetch_stats")
     return a.value, b.value
+
+
+def attn_workspace_bytes(n_heads_q: int, head_dim: int) -> int:
+    return int(lib.moe_attn_workspace_bytes(n_heads_q, head_dim))
+
+
+def attn_decode(q, k_cache, v_cache, n_heads_q, n_heads_kv, head_dim, capacity, n_tokens, scale, o, workspace,
+                stream=None):
+    """Decode attention of one token (moe_attn_decode).  `workspace` is a
+    zero-initialised device byte tensor of at least attn_workspace_bytes."""
+    _check(lib.moe_attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), n_heads_q, n_heads_kv, head_dim, capacity,
+                               n_tokens, float(scale), _ptr(o), _ptr(workspace),
+                               0 if workspace is None else workspace.numel() * workspace.element_size(),
+                               _stream(stream)),
+           "moe_attn_decode")
 
 
 def residual_rmsnorm(ctx: Ctx, r, y, x_next, T, stream=None):

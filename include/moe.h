@@ -384,6 +384,45 @@ int moe_layer_forward_next(moe_ctx *ctx, const moe_layer_weights *W, moe_slot_ca
                            float *y, uint16_t *y_bf16, int32_t *ids, float *gate_w,
                            moe_plan_trace *trace, const moe_next_layer *next, cudaStream_t stream);
 
+/* ------------------------------------------------------ decode attention
+ * The other per-token kernel of the layer loop ("TurboFieldfare: motor open
+ * source ...", section "Proceso de generacion de tokens": decode attention is an
+ * exact split-K/V method over an fp16 KV cache held as a bounded ring for the
+ * sliding-window layers and as linear storage for the full-attention layers;
+ * "Gemma 4 26B en ~2 GB de RAM ...", section "Por que funciona: el A4B del
+ * nombre", the same cache).  For one token:
+ *   o[h] = sum_p softmax_p(scale * q[h] . k[g][slot(p)]) v[g][slot(p)],
+ *   g = h / (n_heads_q / n_heads_kv) (consecutive query heads share a KV head),
+ * over the cache's newest min(n_tokens, capacity) positions, position p held in
+ * slot p mod capacity (a ring; a linear cache has capacity >= n_tokens, so the
+ * attended slots are 0 .. n_tokens-1).  Since attention does not depend on the
+ * order of the positions, the call attends to slots 0 .. min(n_tokens,
+ * capacity)-1.  The slots are split into parts across CTAs; each part keeps
+ * its maximum, exponential sum and unnormalised value sum, and the parts are
+ * merged exactly (by rescaling), in a fixed order, so results are
+ * reproducible bit for bit.
+ *   q        dev bf16 [n_heads_q][head_dim]
+ *   k_cache  dev binary16 [n_heads_kv][capacity][head_dim]; v_cache likewise
+ *   o        dev fp32 [n_heads_q][head_dim] out
+ *   scale    the score scale (e.g. 1/sqrt(head_dim)), finite and > 0
+ *   workspace dev, >= moe_attn_workspace_bytes(n_heads_q, head_dim) bytes,
+ *            ZEROED by the caller before its first use; each call leaves it
+ *            ready for the next one.  Calls sharing a workspace must not overlap
+ *            on the GPU (issue them on one stream).
+ * Supported: head_dim in {64, 128, 256, 512}; n_heads_q / n_heads_kv in
+ * {1, 2, 4, 8} with (head_dim / 32) * group <= 32; n_heads_kv <= 64; every
+ * pointer 16-byte aligned.  One launch, no host synchronisation, capturable in a
+ * CUDA graph.  Errors: MOE_ERR_ARG (sizes, n_tokens < 1, pointers, alignment,
+ * workspace too small), MOE_ERR_CUDA (launch failed). */
+int moe_attn_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                    int n_heads_q, int n_heads_kv, int head_dim, int capacity, int n_tokens,
+                    float scale, float *o, void *workspace, size_t workspace_bytes,
+                    cudaStream_t stream);
+
+/* Workspace bytes moe_attn_decode needs for these sizes (a per-KV-head ticket
+ * and each part's partial results); 0 for sizes below 1.  Host-only. */
+size_t moe_attn_workspace_bytes(int n_heads_q, int head_dim);
+
 /* ------------------------------------------------------ instrumentation */
 #define MOE_PROF_ROUTER    0   /* moe_router_topk kernel */
 #define MOE_PROF_PLAN      1   /* cache-plan kernel */

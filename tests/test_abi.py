@@ -47,3 +47,30 @@ def test_header_documents_every_entry_point():
         # each declaration is preceded by a comment block
         m = re.search(r"\*/\s*(?:[\w\s\*]+?)\b" + name + r"\s*\(", src)
         assert m, name
+
+
+def test_attn_host_side_checks_without_a_gpu():
+    """Workspace sizing is host arithmetic; argument checks of the decode
+    attention entry point answer before any CUDA call."""
+    # ticket block + per (query head, part) an (m, l) pair and head_dim partial sums
+    assert moe.attn_workspace_bytes(16, 256) == 256 + 16 * 64 * 8 + 16 * 64 * 256 * 4
+    assert moe.attn_workspace_bytes(0, 256) == 0
+    L = moe.lib
+    ok = dict(q=16, k=16, v=16, hq=4, hkv=2, hd=64, cap=8, n=4, scale=0.1, o=16, ws=16, wsb=1 << 20)
+
+    def call(**kw):
+        a = {**ok, **kw}
+        return L.moe_attn_decode(a["q"], a["k"], a["v"], a["hq"], a["hkv"], a["hd"], a["cap"], a["n"], a["scale"],
+                                 a["o"], a["ws"], a["wsb"], None)
+
+    # fake (aligned, never dereferenced) addresses: each case fails a check first
+    assert call(q=None) == moe.MOE_ERR_ARG
+    assert call(n=0) == moe.MOE_ERR_ARG
+    assert call(cap=0) == moe.MOE_ERR_ARG
+    assert call(hd=96) == moe.MOE_ERR_ARG
+    assert call(hq=6, hkv=4) == moe.MOE_ERR_ARG
+    assert call(hq=32, hkv=2) == moe.MOE_ERR_ARG
+    assert call(hd=512, hq=8, hkv=2) == moe.MOE_ERR_ARG   # group 4 at width 512: too many registers
+    assert call(scale=-1.0) == moe.MOE_ERR_ARG
+    assert call(q=18) == moe.MOE_ERR_ARG                  # not 16-byte aligned
+    assert call(wsb=100) == moe.MOE_ERR_ARG
