@@ -97,17 +97,18 @@ def csrc_sha256(files=TRAFFIC_SOURCES):
     return h.hexdigest()
 
 
-def recorded_traffic(key):
-    """DRAM bytes (read + write) per layer-token of one kernel on one workload,
-    from one ncu capture (profiles/traffic.json), or None when absent or taken
-    on other kernel sources."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
+def recorded_traffic(key, name="traffic.json", table="bytes_per_layer_token"):
+    """DRAM bytes (read + write) of one kernel on one workload from one ncu
+    capture (profiles/<name>): per layer-token for the expert GEMV kernels,
+    per step for decode attention.  None when absent or taken on other kernel
+    sources."""
+    p = os.path.join(ROOT, "profiles", name)
     if not os.path.exists(p):
         return None
     rec = json.load(open(p))
     if rec.get("source_sha256") != csrc_sha256(tuple(rec.get("sources", TRAFFIC_SOURCES))):
         return None
-    return rec.get("bytes_per_layer_token", {}).get(key)
+    return rec.get(table, {}).get(key)
 
 
 def peaks():
@@ -789,9 +790,10 @@ def run_attn(args, dist):
     kern = {k: {"ms_total": v[0], "launches": v[1], "bytes_per_launch": v[2] / max(1, v[1]),
                 "us_per_launch": 1e3 * v[0] / max(1, v[1]), "gbs": v[2] / (v[0] * 1e-3) / 1e9}
             for k, v in kinds.items() if v[1]}
-    tot_ms = sum(v[0] for v in kinds.values())
-    tot_b = sum(v[2] for v in kinds.values())
-    ach = tot_b / (tot_ms * 1e-3) / 1e9
+    # every kernel of the timed region is this one: its average duration there
+    # is the step time over the step's launches (the step's query copy, a few
+    # microseconds, is included, so this understates the kernel)
+    ach = step_bytes / (ms / Ks * 1e-3) / 1e9
 
     tokens_all = dist.sum(Ks)
     line = {"metric": METRIC_ATTN, "value": tokens_all / (ms * 1e-3), "unit": "tokens/s", "n_gpus": dist.world,
@@ -805,10 +807,13 @@ def run_attn(args, dist):
                        "input_generation_s": gen_s},
             "roofline": {"bound": "hbm", "kernel": "attn_decode_kernel (all 30 launches of a step)",
                          "achieved": ach, "peak": hbm_peak, "unit": "GB/s", "frac": ach / hbm_peak,
-                         "traffic": None, "peak_source": f"{peak_kind} hbm_gbs",
-                         "bytes_per_step": step_bytes,
-                         "note": "achieved = algorithmic bytes of the timed launches / their summed event durations"},
+                         "traffic": recorded_traffic("attn_decode", "traffic_attn.json", "bytes_per_step"),
+                         "traffic_unit": "DRAM bytes per step (ncu)",
+                         "peak_source": f"{peak_kind} hbm_gbs", "bytes_per_step": step_bytes,
+                         "note": "achieved = algorithmic bytes per step / device time per step in the timed region"},
             "kernels": kern,
+            "kernels_note": f"per-launch times from a separate pass of {kp} steps with an event pair around every "
+                            "launch (serialised: no overlap between launches)",
             "gpu_launches": int(dist.sum(nl * Ks))}
     if clk:
         line["clocks"] = clk

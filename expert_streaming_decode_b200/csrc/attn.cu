@@ -123,7 +123,29 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_decode_kernel(AttnArgs A
     const uint16_t* kh = A.k + size_t(h) * A.cap * HD;
     const uint16_t* vh = A.v + size_t(h) * A.cap * HD;
 
-    // the group's queries, pre-scaled so that exp(scale*q.k) = 2^(q'.k)
+    // Start this part's rows streaming into L2 (a hint: no data is read and
+    // nothing waits on it), then wait for the preceding kernel in the stream.
+    // Everything the kernel reads or writes comes after the wait, so with
+    // programmatic dependent launch the next layer's rows stream in while
+    // this kernel's last parts merge.
+    if (warp == 0) {
+        const size_t off = size_t(p0) * HD, bytes = size_t(p1 - p0) * HD * sizeof(uint16_t);
+        bulk_prefetch_l2(kh + off, bytes, lane, 32);
+        bulk_prefetch_l2(vh + off, bytes, lane, 32);
+    }
+    pdl_wait();
+    pdl_trigger();
+
+    // the warp's first rows, then the group's queries (pre-scaled so that
+    // exp(scale*q.k) = 2^(q'.k)) while those rows are in flight
+    RowPiece<DPL> kr[U], vr[U];
+    int p = p0 + warp * U;
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+        if (p + u < p1) {
+            kr[u] = load_piece<DPL>(kh + size_t(p + u) * HD, lane);
+            vr[u] = load_piece<DPL>(vh + size_t(p + u) * HD, lane);
+        }
     float qr[G][DPL];
 #pragma unroll
     for (int g = 0; g < G; ++g)
@@ -140,14 +162,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_decode_kernel(AttnArgs A
         for (int j = 0; j < DPL; ++j) acc[g][j] = 0.f;
     }
 
-    for (int p = p0 + warp * U; p < p1; p += kAttnWarps * U) {
-        RowPiece<DPL> kr[U], vr[U];
-#pragma unroll
-        for (int u = 0; u < U; ++u)
-            if (p + u < p1) kr[u] = load_piece<DPL>(kh + size_t(p + u) * HD, lane);
-#pragma unroll
-        for (int u = 0; u < U; ++u)
-            if (p + u < p1) vr[u] = load_piece<DPL>(vh + size_t(p + u) * HD, lane);
+    for (; p < p1; p += kAttnWarps * U) {
         float s[U][G];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
@@ -199,6 +214,14 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_decode_kernel(AttnArgs A
                 }
             }
         }
+        // the warp's next rows (the registers are free again)
+        const int pn = p + kAttnWarps * U;
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            if (pn + u < p1) {
+                kr[u] = load_piece<DPL>(kh + size_t(pn + u) * HD, lane);
+                vr[u] = load_piece<DPL>(vh + size_t(pn + u) * HD, lane);
+            }
     }
 
     // warps -> this part
@@ -237,29 +260,38 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_decode_kernel(AttnArgs A
     if (!s_last) return;
     __threadfence();
     if (warp < G) {
+        // per part j (lanes j and j + 32): its factor 2^(m_j - M) and the
+        // normaliser sum_j 2^(m_j - M) l_j, reduced in a fixed order
         const int g = warp;
-        float M = -INFINITY;
-        for (int j = lane; j < S; j += 32) M = fmaxf(M, __ldcg(A.part_ml + (size_t(h) * kAttnMaxSplits + j) * G + g).x);
+        const float2* ml = A.part_ml + size_t(h) * kAttnMaxSplits * G + g;
+        const float2 a0 = lane < S ? __ldcg(ml + size_t(lane) * G) : make_float2(-INFINITY, 0.f);
+        const float2 a1 = lane + 32 < S ? __ldcg(ml + size_t(lane + 32) * G) : make_float2(-INFINITY, 0.f);
+        float M = fmaxf(a0.x, a1.x);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-        for (int j = lane; j < S; j += 32) {
-            const float2 ml = __ldcg(A.part_ml + (size_t(h) * kAttnMaxSplits + j) * G + g);
-            s_f[g][j] = exp2f(ml.x - M);
-        }
-        __syncwarp();
-        if (lane == 0) {
-            float den = 0.f;
-            for (int j = 0; j < S; ++j)
-                den = fmaf(s_f[g][j], __ldcg(A.part_ml + (size_t(h) * kAttnMaxSplits + j) * G + g).y, den);
-            s_den[g] = den;
-        }
+        const float f0 = lane < S ? exp2f(a0.x - M) : 0.f;
+        const float f1 = lane + 32 < S ? exp2f(a1.x - M) : 0.f;
+        s_f[g][lane] = f0;
+        s_f[g][lane + 32] = f1;
+        float den = fmaf(f0, a0.y, f1 * a1.y);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
+        if (lane == 0) s_den[g] = den;
     }
     __syncthreads();
+    // each output element: all parts' partial sums loaded together, then summed in part order
+    constexpr int kBatch = 16;
     for (int i = tid; i < G * HD; i += kAttnThreads) {
         const int g = i / HD, d = i % HD;
+        const float* po = A.part_o + (size_t(h) * kAttnMaxSplits * G + g) * HD + d;
         float num = 0.f;
-        for (int j = 0; j < S; ++j)
-            num = fmaf(s_f[g][j], __ldcg(A.part_o + ((size_t(h) * kAttnMaxSplits + j) * G + g) * HD + d), num);
+        for (int j0 = 0; j0 < S; j0 += kBatch) {
+            float t[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) t[u] = j0 + u < S ? __ldcg(po + size_t(j0 + u) * G * HD) : 0.f;
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) num = fmaf(s_f[g][(j0 + u) & (kAttnMaxSplits - 1)], t[u], num);
+        }
         A.o[size_t(h * G + g) * HD + d] = num / s_den[g];
     }
     if (tid == 0) atomicExch(A.tickets + h, 0);  // ready for the next call
@@ -267,7 +299,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_decode_kernel(AttnArgs A
 
 template <int DPL, int G>
 cudaError_t launch_attn(const AttnArgs& a, dim3 grid, cudaStream_t s) {
-    return launch_kernel(attn_decode_kernel<DPL, G>, grid, dim3(kAttnThreads), 0, s, false, 1, a);
+    return launch_kernel(attn_decode_kernel<DPL, G>, grid, dim3(kAttnThreads), 0, s, true, 1, a);
 }
 
 template <int DPL>
