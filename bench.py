@@ -712,6 +712,45 @@ def attn_cpu_baseline(A, seed, budget_s=20.0):
                       f"single-threaded C oracle (fp64), {ts + tf:.1f} s"}
 
 
+def run_reference_attn(args, dist):
+    """The reference arm for decode attention: the oracle, one (token, layer)
+    per step over the same 30-layer mix, on one host core."""
+    if dist.rank != 0:
+        return 0
+    import oracle
+    from expert_streaming_decode_b200 import synth
+    O = oracle.get()
+    A = synth.GEMMA4_ATTN
+    layers = _attn_layers(A)
+    nl = len(layers)
+    kv = [synth.attn_kv(args.seed, l, A.Hkv, cap, A.hd) for l, (cap, _) in enumerate(layers)]
+    scale = 1.0 / math.sqrt(A.hd)
+
+    def step(i):
+        t, l = divmod(i, nl)
+        cap, n = layers[l]
+        O.attn_decode(synth.attn_query(args.seed, t, l, A.Hq, A.hd), kv[l][0], kv[l][1], cap, n, scale)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.warmup, args.warmup + args.steps):
+        step(i)
+    el = time.perf_counter() - t0
+    v = args.steps / nl / el
+    line = {"impl": "reference", "metric": METRIC_ATTN, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": el * 1e3 / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "attn_decode", "layers": nl, "heads_q": A.Hq, "heads_kv": A.Hkv,
+                       "head_dim": A.hd, "window": A.window, "context": A.context,
+                       "step": "one (token, layer) of the 30-layer mix"},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{args.steps} (token, layer) steps after {args.warmup} warm-up steps"},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_attn(args, dist):
     """Decode attention for every layer of one token per step, from resident
     KV caches (378 MB, larger than L2), replayed as a CUDA graph."""
@@ -854,7 +893,7 @@ def main():
     dist = Dist()
     if args.impl == "reference":
         dist.init("gloo")
-        rc = run_reference(args, dims, dist)
+        rc = run_reference_attn(args, dist) if args.workload == "attn_decode" else run_reference(args, dims, dist)
         dist.close()
         return rc
 

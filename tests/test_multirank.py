@@ -61,3 +61,19 @@ def test_reference_arm_two_ranks():
     j = json.loads(lines[0])
     assert j["impl"] == "reference" and j["unit"] == "tokens/s" and j["value"] > 0
     assert j["cpu_baseline"]["kind"] == "oracle" and j["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_attention_reference_arm_two_ranks():
+    """The decode-attention reference arm under a 2-rank torchrun: rank 0
+    alone times the oracle and prints one line; the other rank exits 0."""
+    port = _free_port()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
+           "--impl", "reference", "--workload", "attn_decode", "--gpus", "2", "--steps", "3", "--warmup", "0"]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    j = json.loads(lines[0])
+    assert j["impl"] == "reference" and j["config"]["workload"] == "attn_decode" and j["value"] > 0
+    assert j["cpu_baseline"]["kind"] == "oracle" and j["e2e"]["d2h_bytes_per_step"] == 0
