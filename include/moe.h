@@ -340,7 +340,7 @@ int moe_layer_forward(moe_ctx *ctx, const moe_layer_weights *W, moe_slot_cache *
  * Opt-in; off unless moe_prefetch_configure gave buffers.  The pages disagree
  * on whether expert loads can be started a layer early: one says the router
  * gives a layer of warning ("Gemma 4 26B en ~2 GB de RAM ...", section "Por
- * que pread y no mmap"); the discussion threads judge speculative expert
+ * que pread y no mmap"); the discussion threads consider speculative expert
  * prefetch hard, because a layer's routing depends on the previous layers'
  * output, and note that reading mispredicted experts costs the bandwidth the
  * real misses need ("Show HN: Motor de codigo abierto ...", section
