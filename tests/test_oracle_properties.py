@@ -53,3 +53,37 @@ def test_plan_equals_naive_simulator(case):
             if e_ >= 0:
                 assert st_.slot_of[e_] == s_
         assert (st_.slot_of >= 0).sum() == (st_.expert_in >= 0).sum()
+
+
+@st.composite
+def attn_case(draw):
+    Hkv = draw(st.integers(1, 4))
+    G = draw(st.sampled_from([1, 2, 3, 4]))
+    hd = draw(st.integers(1, 40))
+    cap = draw(st.integers(1, 30))
+    n = draw(st.integers(1, 4 * cap + 3))
+    scale = draw(st.floats(0.01, 3.0))
+    seed = draw(st.integers(0, 2 ** 31 - 1))
+    return Hkv * G, Hkv, hd, cap, n, scale, seed
+
+
+@settings(max_examples=150, deadline=None)
+@given(attn_case())
+def test_attention_equals_library_routine(case):
+    """Decode attention for random head counts, widths, ring capacities and
+    token counts (wrapped or not) equals torch's attention routine applied to
+    the explicitly gathered newest positions, and it is a convex combination
+    of the attended value rows (each output lies within their range)."""
+    import pins
+    Hq, Hkv, hd, cap, n, scale, seed = case
+    rng = np.random.default_rng(seed)
+    q, k, v = pins._attn_case(rng, Hq, Hkv, hd, cap)
+    O = oracle.get()
+    got = O.attn_decode(q, k, v, cap, n, scale)
+    want = pins._attn_torch(q, k, v, cap, n, scale)
+    assert np.allclose(got, want, rtol=1e-11, atol=1e-11)
+    pos = np.arange(max(0, n - cap), n) % cap
+    vf = v.view(np.float16).astype(np.float64)[:, pos]
+    for h in range(Hq):
+        rows = vf[h // (Hq // Hkv)]
+        assert (got[h] >= rows.min(axis=0) - 1e-12).all() and (got[h] <= rows.max(axis=0) + 1e-12).all()
