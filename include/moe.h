@@ -345,7 +345,7 @@ int moe_layer_forward(moe_ctx *ctx, const moe_layer_weights *W, moe_slot_cache *
  * output, and note that reading mispredicted experts costs the bandwidth the
  * real misses need ("Show HN: Motor de codigo abierto ...", section
  * "Direcciones futuras e ideas de investigacion"; "TurboFieldfare: motor open
- * source ...", the comment thread).  This path makes the trade measurable:
+ * source ...", section "Comentarios de Hacker News").  This path makes the trade measurable:
  * while layer l runs on x, layer l+1's router is evaluated on the same x on a
  * separate stream; after layer l's own miss copies, up to n_buffers of its
  * predicted experts that layer l+1's cache does not hold (as far as the host
