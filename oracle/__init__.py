@@ -76,6 +76,10 @@ class Oracle:
         L.orc_cache_plan.restype = C.c_int
         L.orc_cache_plan.argtypes = ([C.c_int, C.c_int, C.c_int, C.c_uint32] + [C.c_void_p] * 5
                                      + [C.c_int, C.c_int, C.c_uint32] + [C.c_void_p] * 7)
+        L.orc_f64_to_bf16.restype = C.c_uint16
+        L.orc_f64_to_bf16.argtypes = [C.c_double]
+        L.orc_residual_rmsnorm.restype = None
+        L.orc_residual_rmsnorm.argtypes = [C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p]
         L.orc_group_by_expert.restype = C.c_int
         L.orc_group_by_expert.argtypes = [C.c_void_p, C.c_int, C.c_int, C.c_int,
                                           C.c_void_p, C.c_void_p]
@@ -190,6 +194,20 @@ class Oracle:
         n = nu.value
         return dict(pair_slot=pair_slot, expert=ue[:n].copy(), slot=us[:n].copy(),
                     hit=uh[:n].copy(), victim=uv[:n].copy(), wave=uw[:n].copy(), waves=waves)
+
+    # layer chaining (test and benchmark harness, not the MoE layer) ---------
+    def f64_to_bf16(self, v: float) -> int:
+        return int(self.lib.orc_f64_to_bf16(float(v)))
+
+    def residual_rmsnorm(self, r_in, y):
+        """(r_out fp64 [D], x_next bf16 bits [D]) for one token."""
+        r_in = np.ascontiguousarray(r_in, dtype=np.float64)
+        y = np.ascontiguousarray(y, dtype=np.float64)
+        D = r_in.size
+        r_out = np.empty(D, dtype=np.float64)
+        x = np.empty(D, dtype=np.uint16)
+        self.lib.orc_residual_rmsnorm(_p(r_in), _p(y), D, _p(r_out), _p(x))
+        return r_out, x
 
     def group_by_expert(self, ids, E: int):
         ids = np.ascontiguousarray(ids, dtype=np.int32)

@@ -425,6 +425,54 @@ int orc_lfu_plan(int E, int S, uint32_t *count, uint32_t *last_use,
                           pair_slot, u_expert, u_slot, u_hit, u_victim, u_wave, n_u);
 }
 
+/* --------------------------------------------------- layer chaining step
+ * Not a step of the MoE layer itself: what the tests and the benchmark put
+ * between two MoE layers so that layer l+1 is routed on layer l's output.
+ * The pages run the routed layers in order, token by token ([hada] "Proceso
+ * de generacion de tokens": the routed-layer loop repeats for every token;
+ * [yodev] "Por que funciona": per layer the router, the fetch plan, the reads
+ * and the combine), so a layer's experts are only known once the layers below
+ * it have run; the rest of the model between two MoE layers is out of scope
+ * and stood in for by a residual stream and an RMS normalisation without a
+ * weight (a stated choice, not the model's own block):
+ *   r_out = r_in + y,   x_next = bf16( r_out / sqrt(mean(r_out^2) + 1e-6) ).
+ * fp64 arithmetic; bf16 rounding is round to nearest, ties to even, straight
+ * from the double value (orc_f64_to_bf16). */
+
+/* bfloat16 (1 sign, 8 exponent bits with bias 127, 7 fraction bits) nearest
+ * to v, ties to the even pattern; beyond the largest finite value (half an
+ * ulp past it) the result is infinity.  NaN gives the quiet NaN 0x7FC0. */
+uint16_t orc_f64_to_bf16(double v)
+{
+    uint16_t sign = signbit(v) ? 0x8000u : 0u;
+    double a = fabs(v), q;
+    int e;
+    if (isnan(v)) return 0x7FC0u;
+    if (a == 0.0) return sign;
+    frexp(a, &e);                       /* a = m * 2^e, 0.5 <= m < 1 */
+    if (e < -125) e = -125;             /* subnormal range: spacing 2^-133 */
+    q = rint(ldexp(a, 8 - e));          /* significand in units of the spacing 2^(e-8), ties to even */
+    a = ldexp(q, e - 8);
+    if (a >= ldexp(1.0, 128)) return (uint16_t)(sign | 0x7F80u);
+    {
+        float f = (float)a;             /* exact: at most 8 significant bits */
+        uint32_t u;
+        memcpy(&u, &f, sizeof u);
+        return (uint16_t)(sign | (u >> 16));
+    }
+}
+
+void orc_residual_rmsnorm(const double *r_in, const double *y, int D, double *r_out, uint16_t *x_next)
+{
+    double ss = 0.0, rms;
+    for (int i = 0; i < D; ++i) {
+        r_out[i] = r_in[i] + y[i];
+        ss += r_out[i] * r_out[i];
+    }
+    rms = sqrt(ss / (double)D + 1e-6);
+    for (int i = 0; i < D; ++i) x_next[i] = orc_f64_to_bf16(r_out[i] / rms);
+}
+
 /* ------------------------------------------------ prefill token grouping
  * Prefill chunk ([hada] "Proceso de generacion de tokens": the prompt is
  * prefilled in chunks of up to 128 tokens so that an expert fetched once

@@ -46,6 +46,9 @@ int orc_lfu_plan(int E, int S, uint32_t *count, uint32_t *last_use,
                  int32_t *pair_slot, int32_t *u_expert, int32_t *u_slot,
                  int32_t *u_hit, int32_t *u_victim, int32_t *u_wave, int *n_u);
 
+uint16_t orc_f64_to_bf16(double v);
+void orc_residual_rmsnorm(const double *r_in, const double *y, int D, double *r_out, uint16_t *x_next);
+
 int orc_group_by_expert(const int32_t *ids, int T, int K, int E,
                         int32_t *offsets, int32_t *pairs);
 

@@ -476,7 +476,59 @@ def pin_attn_closed_forms(O):
     assert O.lib.orc_attn_decode(None, None, None, Hq, Hkv, hd, 0, 1, 0.3, None) == -1
 
 
+# ------------------------------------------------- layer chaining (harness)
+def pin_bf16_round(O):
+    """Rounding to bfloat16: hand-derived golden cases (ties to even,
+    subnormals, overflow), then torch's float32 -> bfloat16 conversion (a
+    library routine, round to nearest even) on random float32 values."""
+    for v, bits in _golden_rows("bf16_round.txt"):
+        got = O.f64_to_bf16(float.fromhex(v))
+        assert got == int(bits, 16), (v, hex(got), bits)
+    rng = np.random.default_rng(21)
+    f = (rng.standard_normal(5000) * np.exp2(rng.integers(-30, 30, 5000))).astype(np.float32)
+    ref = torch.from_numpy(f).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    for v, r in zip(f, ref):
+        assert O.f64_to_bf16(float(v)) == int(r), (float(v), int(r))
+
+
+def pin_residual_rmsnorm(O):
+    """The chaining step r += y; x = bf16(r / sqrt(mean(r^2) + 1e-6)), pinned
+    by cases whose result is fixed without evaluating that expression:
+    the residual sum of float32 values is exact in double; a constant vector
+    of 1e-3 has mean square equal to the 1e-6 term, so every output is
+    1/sqrt(2) -> bf16 0x3F35; a large constant gives 1.0 exactly after
+    rounding; a single non-zero entry 8 in 64 has mean square 1 (the mean, not
+    the sum), so it maps to 8 -> 0x4100; the zero vector stays zero; negating
+    the input flips only the sign bits; and for random rows the bf16 outputs
+    have mean square 1 to within the rounding."""
+    rng = np.random.default_rng(22)
+    D = 512
+    r0 = rng.standard_normal(D).astype(np.float32).astype(np.float64)
+    y = rng.standard_normal(D).astype(np.float32).astype(np.float64)
+    r1, x = O.residual_rmsnorm(r0, y)
+    assert np.array_equal(r1, (r0.astype(np.float32) + y.astype(np.float32)).astype(np.float64)) or \
+        np.array_equal(r1 - y, r0)
+    assert np.array_equal(r1 - r0, y)
+    _, x = O.residual_rmsnorm(np.zeros(D), np.full(D, 1e-3))
+    assert np.all(x == 0x3F35), hex(int(x[0]))
+    _, x = O.residual_rmsnorm(np.full(D, 1000.0), np.zeros(D))
+    assert np.all(x == 0x3F80)
+    one = np.zeros(64)
+    one[5] = 8.0
+    _, x = O.residual_rmsnorm(np.zeros(64), one)
+    assert x[5] == 0x4100 and np.all(np.delete(x, 5) == 0), hex(int(x[5]))
+    r_out, x = O.residual_rmsnorm(np.zeros(D), np.zeros(D))
+    assert np.all(x == 0) and np.all(r_out == 0)
+    v = rng.standard_normal(D) * 5
+    _, xp = O.residual_rmsnorm(v, np.zeros(D))
+    _, xn = O.residual_rmsnorm(-v, np.zeros(D))
+    assert np.array_equal(xn, xp ^ np.uint16(0x8000))
+    xf = synth.bf16_bits_to_f32(xp).astype(np.float64)
+    assert abs(np.mean(xf * xf) - 1.0) < 2.0 ** -7
+
+
 ALL_PINS = [pin_binary16, pin_bf16, pin_layout_points, pin_packer_points, pin_dequant_random,
             pin_router_exact, pin_router_random, pin_topk, pin_gate_weights, pin_gelu, pin_ffn,
             pin_layer, pin_lfu_naive, pin_cache_policies_naive, pin_cache_policies_cases, pin_lfu_invariants,
-            pin_group_by_expert, pin_attn_library, pin_attn_closed_forms]
+            pin_group_by_expert, pin_attn_library, pin_attn_closed_forms, pin_bf16_round,
+            pin_residual_rmsnorm]

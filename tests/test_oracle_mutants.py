@@ -56,6 +56,12 @@ MUTANTS = {
     "attn_not_normalised": ("o[(size_t)h * hd + d] = acc / z;", "o[(size_t)h * hd + d] = acc;"),
     "attn_value_slot_linear": ("acc += w[i] * orc_f16_to_f64(vg[slot * hd + d]);",
                                "acc += w[i] * orc_f16_to_f64(vg[(size_t)i * hd + d]);"),
+    "bf16_truncates": ("q = rint(ldexp(a, 8 - e));", "q = floor(ldexp(a, 8 - e));"),
+    "bf16_ties_away": ("q = rint(ldexp(a, 8 - e));", "q = round(ldexp(a, 8 - e));"),
+    "bf16_no_subnormal_clamp": ("if (e < -125) e = -125;", "(void)0;"),
+    "rms_eps_dropped": ("rms = sqrt(ss / (double)D + 1e-6);", "rms = sqrt(ss / (double)D);"),
+    "rms_sum_not_mean": ("rms = sqrt(ss / (double)D + 1e-6);", "rms = sqrt(ss + 1e-6);"),
+    "residual_dropped": ("r_out[i] = r_in[i] + y[i];", "r_out[i] = y[i];"),
 }
 
 
