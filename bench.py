@@ -66,6 +66,9 @@ def parse_args():
     p.add_argument("--zipf", type=float, default=None,
                    help="Zipf exponent of the router popularity bias (default 1.1; 0 = uniform router, "
                         "the default for decode_resident)")
+    p.add_argument("--zipf-lambda", type=float, default=synth_default_lambda(),
+                   help="strength of the Zipf popularity bias: bias_e = -lambda * s * ln(1 + rank_e); "
+                        "calibrated so the chained 16-slot decode lands in the pages' 60-70%% hit-rate band")
     p.add_argument("--layers", type=int, default=30)
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--no-e2e", action="store_true")
@@ -84,6 +87,11 @@ def parse_args():
 
 
 # --------------------------------------------------------------- helpers
+def synth_default_lambda():
+    from expert_streaming_decode_b200 import synth
+    return synth.ZIPF_LAMBDA
+
+
 # sources of the one-token expert GEMV kernels whose DRAM traffic profiles/traffic.json records
 TRAFFIC_SOURCES = ("ffn.cu", "ffn.cuh", "common.cuh", "decode_wl.cuh", "launch.cuh")
 
@@ -234,7 +242,7 @@ class Model:
             wq, ws = synth.router_weights(args.seed, l, dims.E, dims.D)
             self.wq.append(torch.from_numpy(wq).to(dev))
             self.ws.append(torch.from_numpy(ws.view(np.int16)).to(dev))
-            b = synth.zipf_bias(args.seed, l, dims.E, s=args.zipf) if args.zipf > 0 else None
+            b = synth.zipf_bias(args.seed, l, dims.E, s=args.zipf, lam=args.zipf_lambda) if args.zipf > 0 else None
             self.bias.append(None if b is None else torch.from_numpy(b).to(dev))
             self.shared.append(torch.from_numpy(synth.expert_blob(args.seed, l, 0, dims.D, dims.FS, shared=True)).to(dev))
         t0 = time.time()
@@ -321,23 +329,39 @@ def moe_prefetch_stats(model):
     return model.moe.prefetch_stats(model.ctx) if model.nexts is not None else (0, 0)
 
 
-def decode_token(model, x0, r, x, y, T, tok, tr=None, trace_acc=None):
+def decode_token(model, x0, r, x, y, T, tok, tr=None, trace_acc=None, on_layer=None, ids=None, gate_w=None):
     """One decode step: T tokens through every layer (layer l+1 reads the
-    residual stream after layer l, RMS-normalised)."""
+    residual stream after layer l, RMS-normalised).  on_layer(l, x_l, y, r),
+    if given, runs after layer l's call and before the residual step (tests
+    use it to read each layer's input and output); ids / gate_w receive the
+    layer's routing when given."""
     moe, d, ctx = model.moe, model.d, model.ctx
     moe.bf16_to_f32(ctx, x0, r, T * d.D)
     cur = x0
     for l in range(model.L):
         if model.nexts is not None and T == 1:
             moe.layer_forward_next(ctx, model.W[l], model.caches[l], cur, T, tok, model.bias[l], y, model.nexts[l],
-                                   trace=tr)
+                                   ids=ids, gate_w=gate_w, trace=tr)
         else:
-            moe.layer_forward(ctx, model.W[l], model.caches[l], cur, T, tok, model.bias[l], y, trace=tr)
+            moe.layer_forward(ctx, model.W[l], model.caches[l], cur, T, tok, model.bias[l], y, ids=ids,
+                              gate_w=gate_w, trace=tr)
         if tr is not None:
             res = tr.c
             trace_acc["misses"] += res.n_misses
             trace_acc["distinct"] += res.n_distinct
             trace_acc["h2d"] += int(res.h2d_bytes)
+            if T == 1:
+                # expert repeats across consecutive tokens of this layer
+                sel = set(int(e) for e in tr.arrays["expert"][:res.n_distinct])
+                hist = trace_acc.setdefault("hist", {}).setdefault(l, [])
+                if len(hist) == 2:
+                    trace_acc["rep_n"] = trace_acc.get("rep_n", 0) + len(sel)
+                    trace_acc["rep1"] = trace_acc.get("rep1", 0) + len(sel & hist[-1])
+                    trace_acc["rep2"] = trace_acc.get("rep2", 0) + len(sel & (hist[-1] | hist[-2]))
+                hist.append(sel)
+                del hist[:-2]
+        if on_layer is not None:
+            on_layer(l, cur, y, r)
         if l + 1 < model.L:
             moe.residual_rmsnorm(ctx, r, y, x, T)
             cur = x
@@ -485,8 +509,8 @@ class OracleDecoder:
         self.O, self.synth, self.d, self.args = oracle.get(), synth, dims, args
         self.L = args.layers
         self.routers = [synth.router_weights(args.seed, l, dims.E, dims.D) for l in range(self.L)]
-        self.bias = [synth.zipf_bias(args.seed, l, dims.E, s=args.zipf) if args.zipf > 0 else None
-                     for l in range(self.L)]
+        self.bias = [synth.zipf_bias(args.seed, l, dims.E, s=args.zipf, lam=args.zipf_lambda) if args.zipf > 0
+                     else None for l in range(self.L)]
         self.shared = {}
         self.blobs = {}
         pol = {"lfu": oracle.POLICY_LFU, "lru": oracle.POLICY_LRU, "lfu_decay": oracle.POLICY_LFU_DECAY,
@@ -949,7 +973,9 @@ def main():
     value = tokens_all / (ms * 1e-3)
     line = {"metric": METRIC_PREFILL if args.workload == "prefill" else METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": dist.world, "steps": K, "warmup": W,
-            "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": ("fp16 tcgen05 MMA on dequantised int4 tiles, fp32 accumulation" if T >= 2 else
+                      "int4 weights x 16-bit fixed-point activations (dp4a), fp32 accumulation"),
             "data": "synthetic"}
     cfg = {"workload": args.workload, "layers": args.layers, "batch": T, "slots": args.slots if streaming else None,
            "cache_policy": (args.policy + (f"_{args.decay_period}" if args.policy == "lfu_decay" else ""))
@@ -957,7 +983,8 @@ def main():
            "prefetch_buffers": args.prefetch if streaming else None,
            "store": (("file, O_DIRECT" if args.direct else "file, page cache") if args.store_file else "pinned host memory")
            if streaming else None,
-           "zipf_s": args.zipf, "tokens_per_rank": ntok * T, "parallelism": f"replicas x{dist.world}",
+           "zipf_s": args.zipf, "zipf_lambda": args.zipf_lambda if args.zipf > 0 else None,
+           "tokens_per_rank": ntok * T, "parallelism": f"replicas x{dist.world}",
            "l2": ("working set > L2: 30 layers x (16 slots + shared) = 1.9 GB in HBM plus a 12.85 GB pinned store"
                   if streaming else "working set > L2: 12.85 GB of resident experts")}
     line["config"] = cfg
@@ -996,7 +1023,8 @@ def main():
         # the grouped GEMM's FLOPs: 2 * pairs * (3 * F * D) routed + 2 * T * (3 * FS * D) shared per layer
         flop_layer = 2.0 * T * dims.K * 3 * dims.F * dims.D + 2.0 * T * 3 * dims.FS * dims.D
         gemm_ms = kern["gate_up"]["ms_total"] + kern["down"]["ms_total"]
-        tf = flop_layer * n_layer_tok / T / (gemm_ms * 1e-3) / 1e12
+        # n_layer_tok counts layer-steps of T tokens each, and flop_layer already covers the T tokens
+        tf = flop_layer * n_layer_tok / (gemm_ms * 1e-3) / 1e12
         pk = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["bf16_tflops"] if peak_kind == "measured" else 1590.0
         line["tensor"] = {"achieved_tflops": tf, "peak_tflops": pk, "frac": tf / pk,
                           "note": "fp16 tcgen05 MMAs (peak: measured bf16 dense, same rate as fp16); "
@@ -1037,6 +1065,19 @@ def main():
                                                 "4 threads" + (", O_DIRECT" if args.direct else ", page cache")}
         line["hit_rate"] = 1.0 - acc_t["misses"] / max(1, acc_t["distinct"])
         line["misses_per_token"] = acc_t["misses"] / (K * T)
+        if T == 1:
+            # the identity miss bytes = (1 - hit) x layers x top-k x blob for one-token steps,
+            # and the pages' repeat statistics of the routing (40 % / 57 %)
+            line["miss_bytes_check"] = {
+                "measured": acc_t["h2d"] / K,
+                "from_hit_rate": (1.0 - line["hit_rate"]) * args.layers * dims.K * model.nb,
+                "holds": abs(acc_t["h2d"] / K - (1.0 - line["hit_rate"]) * args.layers * dims.K * model.nb) < 1.0}
+            n_rep = max(1, acc_t.get("rep_n", 0))
+            line["expert_repeat"] = {"next_token": acc_t.get("rep1", 0) / n_rep,
+                                     "within_two_tokens": acc_t.get("rep2", 0) / n_rep,
+                                     "pages": {"next_token": 0.40, "within_two_tokens": 0.57},
+                                     "note": "share of a token's selected experts (per layer) also selected by the "
+                                             "previous token / one of the two previous tokens, over the timed tokens"}
         if model.nexts is not None:
             iss, used = pf1[0] - pf0[0], pf1[1] - pf0[1]
             line["prefetch"] = {"buffers": args.prefetch, "issued_bytes_per_token": iss / (K * T),
@@ -1058,7 +1099,8 @@ def main():
         ms2, _ = timed(dist, model, lambda: runner.run(None, K, W, host_io=(xh, yh)))
         line["e2e"] = {"value": dist.sum(K * T) / (ms2 * 1e-3), "unit": "tokens/s",
                        "h2d_bytes_per_step": T * dims.D * 2, "d2h_bytes_per_step": T * dims.D * 4,
-                       "api": "moe_layer_forward x 30 per step, input bf16 copied from pinned host, output fp32 copied back"}
+                       "api": ("moe_layer_forward_next" if model.nexts is not None else "moe_layer_forward")
+                              + f" x {args.layers} per step, input bf16 copied from pinned host, output fp32 copied back"}
 
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu and not args.profile and args.workload == "decode_stream":
         line["cpu_baseline"] = cpu_baseline(args, dims)

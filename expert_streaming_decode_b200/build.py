@@ -5,6 +5,7 @@ library next to this file, so the built library travels with the source tree.
 """
 from __future__ import annotations
 
+import concurrent.futures
 import glob
 import os
 import subprocess
@@ -34,7 +35,7 @@ def build(verbose: bool = False, ptxas_info: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
     sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     headers = sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + [os.path.join(INCLUDE, "moe.h")]
-    objs = []
+    objs, cmds = [], []
     for src in sources:
         obj = os.path.join(BUILD, os.path.basename(src) + ".o")
         objs.append(obj)
@@ -44,7 +45,13 @@ def build(verbose: bool = False, ptxas_info: bool = False) -> str:
                 cmd.insert(1, "-Xptxas=-v")
             if verbose:
                 print(" ".join(cmd), flush=True)
-            subprocess.run(cmd, check=True)
+            cmds.append(cmd)
+    # the translation units are independent: compile them in parallel
+    with concurrent.futures.ThreadPoolExecutor(max(1, min(len(cmds), os.cpu_count() or 4))) as ex:
+        for r in ex.map(lambda c: subprocess.run(c, capture_output=True, text=True), cmds):
+            if r.stdout or r.stderr:
+                print(r.stdout + r.stderr, end="", flush=True)
+            r.check_returncode()
     if _stale(LIB, objs):
         cmd = [NVCC, *ARCH, "-shared", "-o", LIB, *objs, "-lcudart"]
         if verbose:

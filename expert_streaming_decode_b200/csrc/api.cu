@@ -632,6 +632,10 @@ int moe_router_topk(moe_ctx* c, const uint16_t* x, const int8_t* wq, const uint1
 int moe_cache_reset(moe_ctx* c, moe_slot_cache* cache, cudaStream_t s) {
     if (!c || !cache || !cache->state) return MOE_ERR_ARG;
     mirror_of(c, cache->state).assign(size_t(c->d.n_experts), int16_t(-1));
+    // staged look-ahead blobs fetched for this cache no longer match its state
+    for (size_t i = 0; i < c->pf_table.size();)
+        if (c->pf_table[i].state == cache->state) c->pf_table.erase(c->pf_table.begin() + long(i));
+        else ++i;
     c->launches += 1;
     return cuda_status(launch_cache_reset(cache->state, c->d.n_experts, c->d.n_slots, c->pdl, s));
 }

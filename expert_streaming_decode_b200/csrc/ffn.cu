@@ -28,6 +28,7 @@
 //     w * (partial dot) per (entry, tile segment) and the last CTA of each
 //     32-row output tile sums y_in and every entry in list order.
 #include "common.cuh"
+#include "decode_wl.cuh"
 #include "ffn.cuh"
 #include "launch.cuh"
 
@@ -1018,7 +1019,8 @@ cudaError_t launch_ffn(const GemvLaunch& L, cudaStream_t s, void (*hook)(void*, 
 }
 
 // ------------------------------------------------------ work-list builder
-// Groups the call's (token, k) pairs by expert slot (ascending slot, pairs in
+// One token (GEMV mode): one entry per selection in k order.  Otherwise:
+// groups the call's (token, k) pairs by expert slot (ascending slot, pairs in
 // ascending index inside a slot), splits each group into entries of at most
 // kMaxRows rows (kGemmMaxRows in GEMM mode), puts the shared expert (all
 // tokens) first, and computes each entry's first gate/up and down unit.  One
@@ -1060,6 +1062,40 @@ __global__ void __launch_bounds__(kWlThreads) build_worklist_kernel(WorkListArgs
     __shared__ int s_maxr;
     pdl_wait();
     pdl_trigger();
+    if (a.T == 1 && !a.gemm) {
+        // one token: one entry per selection, in k order, as the router and
+        // plan kernels write it; a slot named twice is streamed twice (each
+        // selection carries its own gate weight)
+        if (threadIdx.x < 32) {
+            const int lane = threadIdx.x;
+            int sl = 0;
+            float w = 0.f;
+            bool take = false;
+            if (lane < a.K) {
+                take = !a.pair_wave || a.pair_wave[lane] == a.wave;
+                sl = a.pair_slot[lane];
+                if (sl < 0 || sl >= a.n_slot_range) {
+                    if (take) set_status(a.status, MOE_ERR_RANGE);
+                    sl = 0;
+                }
+                w = a.gate_w[lane];
+            }
+            DecodeWLTarget t;
+            t.wl = a.wl;
+            t.entries = a.entries;
+            t.rows = a.rows;
+            t.slot_base = a.slot_base;
+            t.slot_stride = a.slot_stride;
+            t.shared_blob = a.shared_blob;
+            t.F = a.F;
+            t.FS = a.FS;
+            t.D = a.D;
+            t.h_shared_off = a.h_shared_off;
+            t.blob_bytes = 0;
+            write_decode_worklist(t, a.K, sl, w, take);
+        }
+        return;
+    }
     const int np = a.T * a.K;
     const int S = a.n_slot_range;
     auto slot_of = [&](int p) -> int {  // -1: not in this wave

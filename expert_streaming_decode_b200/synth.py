@@ -187,8 +187,15 @@ def router_weights(seed, layer, E, D, G=64):
     return wq, ws
 
 
-def zipf_bias(seed, layer, E, s=1.1, lam=0.75):
-    """Per-expert popularity bias, float32 [E]."""
+# Strength of the popularity bias (see zipf_bias): chosen so that the chained
+# 30-layer decode (residual stream between layers) with 16 LFU slots and
+# Zipf s = 1.1 lands in the pages' 60-70 % hit-rate band.
+ZIPF_LAMBDA = 0.75
+
+
+def zipf_bias(seed, layer, E, s=1.1, lam=None):
+    """Per-expert popularity bias, float32 [E]: -lam * s * ln(1 + pi(e))."""
+    lam = ZIPF_LAMBDA if lam is None else lam
     r = _rng(seed, _ZIPF, layer, 0)
     rank = r.permutation(E).astype(np.float64) + 1.0
     return (-lam * s * np.log(rank)).astype(np.float32)

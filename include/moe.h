@@ -216,6 +216,7 @@ typedef struct moe_slot_cache {
 size_t moe_cache_state_words(const moe_dims *dims);
 
 /* Cold start: counts and last-use 0, nothing resident, all slots empty.
+ * Also drops any look-ahead blob staged for this cache (moe_layer_forward_next).
  * Enqueued on `stream`. */
 int moe_cache_reset(moe_ctx *ctx, moe_slot_cache *cache, cudaStream_t stream);
 
@@ -268,7 +269,8 @@ int moe_cache_plan(moe_ctx *ctx, moe_slot_cache *cache, const int32_t *ids, int 
  *   y_in       dev fp32 [T][D] or NULL; y dev fp32 [T][D] out (may equal y_in)
  *   y_bf16     dev bf16 bits [T][D] out, or NULL
  * 1 <= T <= 32 (dequantising GEMV kernels; moe_layer_forward runs batches on
- * the grouped tensor-core path instead).
+ * the grouped tensor-core path instead).  With T = 1 a slot may appear more
+ * than once in pair_slot (each selection is computed with its own weight).
  * Slot indices outside [0, n_slot_range) are clamped and MOE_ERR_RANGE is
  * recorded.  Uses context scratch; calls on one context must not overlap. */
 int moe_expert_ffn(moe_ctx *ctx, const uint16_t *x, int T, int top_k, const int32_t *pair_slot,
@@ -289,8 +291,9 @@ int moe_expert_ffn(moe_ctx *ctx, const uint16_t *x, int T, int top_k, const int3
  * pair_slot dev int32 [top_k], gate_w dev fp32 [top_k], slot_base/slot_stride/
  * n_slot_range as there, y_in/y dev fp32 [d_model], y_bf16 dev bf16 or NULL).
  * Limits of the fixed scratch: d_model <= 2816 (multiple of 256), d_ff <= 2112,
- * top_k <= 8; larger sizes return MOE_ERR_ARG before any CUDA call.  Slots of
- * one token must be distinct.
+ * top_k <= 8; larger sizes return MOE_ERR_ARG before any CUDA call.  A slot
+ * may appear more than once in pair_slot: each selection is computed with its
+ * own gate weight (the blob is streamed once per selection).
  * Scratch: a 4 MiB file-scope device array inside libmoe.so, present on every
  * GPU that loads the library until the process exits.  The FIRST call on each
  * device sets up that device (looks up the array's device address and the
@@ -355,8 +358,14 @@ int moe_layer_forward(moe_ctx *ctx, const moe_layer_weights *W, moe_slot_cache *
  * the trace and the outputs are exactly those of moe_layer_forward; only
  * where a missed blob is copied from changes.
  *
+ * A staged blob is a copy of the host store taken when it was prefetched: the
+ * store must not be rewritten while buffers are configured, or the caller must
+ * drop the staged blobs first (moe_prefetch_configure, or moe_cache_reset of
+ * the cache they were fetched for).
+ *
  * Sets the number of HBM staging buffers (0..16; 0 turns prefetch off and
- * frees them), one expert blob each.  Waits for the context's copy streams.
+ * frees them), one expert blob each, and drops every staged blob.  Waits for
+ * the context's copy streams.
  * MOE_ERR_ARG (count out of range), MOE_ERR_CUDA (allocation failed). */
 int moe_prefetch_configure(moe_ctx *ctx, int n_buffers);
 

@@ -1,0 +1,159 @@
+"""GPU parity of the chained decode: the benchmark's own token loop
+(bench.decode_token), where layer l+1's input is the residual stream after
+layer l, RMS-normalised, so every layer's routing depends on the layers below
+it, as in the pages' token loop ("TurboFieldfare: motor open source ...",
+section "Proceso de generacion de tokens": the routed-layer loop repeats token
+by token; "Gemma 4 26B en ~2 GB de RAM ...", section "Por que funciona").
+
+The oracle is teacher-forced on the GPU's own bf16 input of every (token,
+layer): its router, top-K, LFU plan (one state per layer, carried across the
+tokens) and layer output are compared with the GPU's at every step, and its
+chaining step (residual + RMS, fp64) with the harness kernel's.  Ids, gate
+weights, plan traces and slot contents bit for bit (gate weights within 1e-5);
+outputs within max|y - r| <= 2e-3 max|r|; the chained bf16 input within one
+bf16 unit in the last place of the oracle's rounding of the fp64 value."""
+import argparse
+
+import numpy as np
+import pytest
+import torch
+
+import bench
+import oracle
+from expert_streaming_decode_b200 import synth
+from gpu_data import GATE_TOL, TOL, rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def O():
+    return oracle.get()
+
+
+def _args(layers, slots, prefetch, seed=0):
+    return argparse.Namespace(layers=layers, slots=slots, seed=seed, zipf=1.1, zipf_lambda=synth.ZIPF_LAMBDA,
+                              policy="lfu", decay_period=0, store_file=None, direct=False, prefetch=prefetch)
+
+
+def _bf16_ulp_diff(a, b):
+    """|a - b| in bf16 units in the last place (same-sign finite values)."""
+    fa = synth.bf16_bits_to_f32(a).astype(np.float64)
+    fb = synth.bf16_bits_to_f32(b).astype(np.float64)
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(fb), 2.0 ** -126))) - 7)
+    return np.abs(fa - fb) / ulp
+
+
+def _chain(O, d, layers, tokens, slots, prefetch, y_samples):
+    args = _args(layers, slots, prefetch)
+    model = bench.Model(args, synth.Dims(**{**d.as_dict(), "L": layers, "S": slots}), max_tokens=1, streaming=True)
+    moe = model.moe
+    nb = model.nb
+    store = model.store.numpy()
+    routers = [synth.router_weights(args.seed, l, d.E, d.D) for l in range(layers)]
+    biases = [synth.zipf_bias(args.seed, l, d.E, s=args.zipf, lam=args.zipf_lambda) for l in range(layers)]
+    shared = [synth.expert_blob(args.seed, l, 0, d.D, d.FS, shared=True) for l in range(layers)]
+    ost = [oracle.LfuState(d.E, slots) for _ in range(layers)]
+    dev = torch.device("cuda")
+    x0 = torch.empty((1, d.D), dtype=torch.int16, device=dev)
+    x = torch.empty((1, d.D), dtype=torch.int16, device=dev)
+    r = torch.empty((1, d.D), dtype=torch.float32, device=dev)
+    y = torch.empty((1, d.D), dtype=torch.float32, device=dev)
+    ids = torch.empty((1, d.K), dtype=torch.int32, device=dev)
+    gw = torch.empty((1, d.K), dtype=torch.float32, device=dev)
+    tr = moe.Trace(d.E)
+    acc = {"misses": 0, "distinct": 0, "h2d": 0}
+    model.reset()
+    stats = {"ids": 0, "plans": 0, "outputs": 0, "chained": 0, "slots": 0, "ulp1": 0, "misses": 0}
+    for t in range(tokens):
+        xb0 = synth.hidden(args.seed + 17, t, 0, d.D)
+        x0.copy_(torch.from_numpy(xb0.view(np.int16)[None].copy()))
+        prev = {}
+
+        def on_layer(l, cur, y_t, r_t):
+            torch.cuda.synchronize()
+            model.ctx.sync()
+            xl = cur.cpu().numpy().view(np.uint16)[0].copy()
+            yl = y_t.cpu().numpy()[0].astype(np.float64)
+            rl = r_t.cpu().numpy()[0].astype(np.float64)
+            got_ids, got_w = ids.cpu().numpy()[0], gw.cpu().numpy()[0]
+            plan = tr.result()
+            # the chained input: layer 0 reads the token's state; layer l > 0
+            # reads the oracle's chaining step applied to the GPU's r and y of l - 1
+            if l == 0:
+                assert np.array_equal(xl, xb0)
+                assert np.array_equal(rl, synth.bf16_bits_to_f32(xb0).astype(np.float64))
+            else:
+                r_want, x_want = O.residual_rmsnorm(prev["r"], prev["y"])
+                # fp32 residual add on the GPU: within half an fp32 ulp of the exact sum
+                assert np.all(np.abs(rl - r_want) <= np.abs(r_want) * 2.0 ** -24 + 1e-30), (t, l)
+                du = _bf16_ulp_diff(xl, x_want)
+                assert du.max() <= 1.0, (t, l, du.max())
+                stats["ulp1"] += int((du > 0).sum())
+                stats["chained"] += 1
+            wq, ws = routers[l]
+            lg = O.router_logits(xl, wq, ws, biases[l], d.E, d.D, d.G)
+            want_ids = O.topk(lg, d.K)
+            assert np.array_equal(got_ids, want_ids), (t, l, got_ids, want_ids)
+            assert np.max(np.abs(got_w - O.gate_weights(lg, want_ids))) <= GATE_TOL, (t, l)
+            stats["ids"] += 1
+            want = O.lfu_plan(ost[l], want_ids[None], t)
+            for key in ("expert", "slot", "hit", "victim", "wave"):
+                assert np.array_equal(plan[key], want[key]), (t, l, key)
+            nmiss = int((want["hit"] == 0).sum())
+            assert plan["misses"] == nmiss and plan["h2d_bytes"] == nmiss * nb, (t, l)
+            stats["plans"] += 1
+            stats["misses"] += nmiss
+            if (t, l) in y_samples:
+                _, _, _, want_y = O.moe_token(d.as_dict(), xl, wq, ws, biases[l], shared[l],
+                                              [store[l, e, :nb] for e in range(d.E)])
+                err = rel_err(yl, want_y)
+                assert err <= TOL, (t, l, err)
+                stats["outputs"] += 1
+            if t % 4 == 3:
+                sl = model.slots[l].cpu().numpy()
+                for s_, e_ in enumerate(ost[l].expert_in):
+                    if e_ >= 0:
+                        assert np.array_equal(sl[s_, :nb], store[l, e_, :nb]), (t, l, s_, e_)
+                stats["slots"] += 1
+            prev["r"], prev["y"] = rl, yl
+
+        bench.decode_token(model, x0, r, x, y, 1, t, tr=tr, trace_acc=acc, on_layer=on_layer, ids=ids, gate_w=gw)
+    torch.cuda.synchronize()
+    model.ctx.sync()
+    if prefetch:
+        issued, used = moe.prefetch_stats(model.ctx)
+        stats["pf_issued"], stats["pf_used"] = issued, used
+        assert used <= issued
+    model.ctx.close()
+    assert stats["ids"] == stats["plans"] == tokens * layers
+    assert stats["chained"] == tokens * (layers - 1)
+    assert stats["outputs"] == len(y_samples)
+    return stats
+
+
+@pytest.mark.parametrize("prefetch", [0, 2], ids=["no-lookahead", "lookahead-2"])
+def test_chained_decode_tiny_30_layers(O, prefetch):
+    """30 chained layers of the scaled-down shape (6 slots), 24 tokens: every
+    (token, layer) checked, outputs too."""
+    d = synth.TINY
+    samples = {(t, l) for t in range(24) for l in range(30)}
+    st = _chain(O, d, layers=30, tokens=24, slots=6, prefetch=prefetch, y_samples=samples)
+    assert st["misses"] > 0
+    if prefetch:
+        assert st["pf_used"] > 0
+
+
+@pytest.mark.parametrize("prefetch", [0, 1], ids=["no-lookahead", "lookahead-1"])
+def test_chained_decode_full_shape(O, prefetch):
+    """8 chained layers of the 26B-A4B shape, 16 slots, Zipf(1.1), 16 tokens:
+    ids, gate weights, plans, chained inputs at every (token, layer), slot
+    contents every 4th token, outputs on a sample spread over tokens and
+    layers (the oracle's fp64 layer takes about a second each)."""
+    d = synth.GEMMA4_26B
+    samples = {(0, 0), (0, 7), (1, 3), (3, 1), (5, 6), (7, 2), (8, 5), (10, 0), (11, 4), (13, 7), (15, 1),
+               (15, 6)}
+    st = _chain(O, d, layers=8, tokens=16, slots=16, prefetch=prefetch, y_samples=samples)
+    assert st["misses"] > 0
+    if prefetch:
+        assert st["pf_issued"] > 0
