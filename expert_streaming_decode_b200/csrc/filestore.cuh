@@ -10,6 +10,8 @@
 
 namespace moe {
 
+class ReadPool;
+
 // One miss: read [offset, offset + len) of fd (at least `need` bytes must
 // exist) and copy the first `need` bytes to the device address dst.
 struct FileRead {
@@ -33,12 +35,13 @@ public:
     // reads every entry with up to `buffers` reads in flight and issues its
     // copy on `side` as soon as it is read; returns MOE_OK, MOE_ERR_IO (read
     // failed or file too short), MOE_ERR_TIMEOUT (a read took longer than
-    // timeout_ms) or MOE_ERR_CUDA.  Adds the copied bytes to *bytes.
+    // timeout_ms), MOE_ERR_STATE (a read of an earlier failed call is still
+    // running: its buffer is not free yet) or MOE_ERR_CUDA.  Adds the copied
+    // bytes to *bytes.
     int read_and_copy(const std::vector<FileRead>& reads, cudaStream_t side, int timeout_ms, uint64_t* bytes);
 
 private:
-    struct Impl;
-    Impl* impl_ = nullptr;
+    ReadPool* pool_ = nullptr;
     std::vector<uint8_t*> bufs_;
     std::vector<cudaEvent_t> events_;
     size_t buf_bytes_ = 0;
