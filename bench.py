@@ -60,9 +60,13 @@ def parse_args():
                    help="streamed workloads: write each layer's experts to DIR/layerNN.experts and read misses "
                         "from those files with positional reads (the file-backed store)")
     p.add_argument("--direct", action="store_true", help="--store-file: open the files with O_DIRECT")
+    p.add_argument("--fill", choices=["direct", "copy"], default="direct",
+                   help="streamed workloads with the pinned store: how one-token misses reach their slots -- "
+                        "'direct': the layer kernel reads them from pinned host memory as it computes (default); "
+                        "'copy': the host reads the plan and the copy engine copies them")
     p.add_argument("--prefetch", type=int, default=None, metavar="P",
-                   help="decode_stream: stage up to P of the next layer's predicted misses (look-ahead; 0 = off; "
-                        "default 1 for the one-token decode_stream workload with the pinned store, else 0)")
+                   help="decode_stream with --fill copy: stage up to P of the next layer's predicted misses "
+                        "(look-ahead; 0 = off, the default)")
     p.add_argument("--zipf", type=float, default=None,
                    help="Zipf exponent of the router popularity bias (default 1.1; 0 = uniform router, "
                         "the default for decode_resident)")
@@ -78,9 +82,9 @@ def parse_args():
     if a.zipf is None:
         a.zipf = 0.0 if a.workload == "decode_resident" else 1.1
     if a.prefetch is None:
-        a.prefetch = 1 if (a.workload == "decode_stream" and a.batch == 1 and not a.store_file) else 0
-    if a.prefetch and (a.workload != "decode_stream" or a.batch != 1 or a.store_file):
-        p.error("--prefetch needs the one-token decode_stream workload with the pinned host store")
+        a.prefetch = 0
+    if a.prefetch and (a.workload != "decode_stream" or a.batch != 1 or a.store_file or a.fill != "copy"):
+        p.error("--prefetch needs the one-token decode_stream workload with the pinned host store and --fill copy")
     if not 0 <= a.prefetch <= 16:
         p.error("--prefetch takes 0..16 buffers")
     return a
@@ -185,6 +189,7 @@ class Dist:
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.local_world = int(os.environ.get("LOCAL_WORLD_SIZE", "1"))
         self.pg = None
 
     def init(self, backend):
@@ -220,13 +225,100 @@ class Dist:
             self.pg.destroy_process_group()
 
 
+# ------------------------------------------------------- the host store
+def mem_available() -> int:
+    """Bytes the kernel reports as available for new allocations."""
+    with open("/proc/meminfo") as f:
+        for line in f:
+            if line.startswith("MemAvailable:"):
+                return int(line.split()[1]) * 1024
+    return 0
+
+
+class HostStore:
+    """Every routed expert of every layer in host memory, [L][E][stride] uint8.
+
+    One process per GPU on a node: the local ranks share ONE copy, a POSIX
+    shared-memory segment that local rank 0 creates and fills and the others
+    map; each rank then page-locks the mapping for its own GPU, so eight
+    replicas hold one 12.85 GB store instead of eight.  A single process uses
+    ordinary pinned memory.  Both refuse up front, with the numbers, when the
+    host cannot hold the store (rather than failing half-way through pinning).
+    `pin` False keeps the memory pageable (CPU tests)."""
+
+    SHM_DIR = "/dev/shm"
+
+    def __init__(self, shape, fill, dist, pin=True, tag="moe_store", avail=None):
+        import mmap
+
+        import torch
+        self.shape, self.nbytes = tuple(shape), int(np.prod(shape))
+        self._mm, self._path, self.registered = None, None, False
+        avail = mem_available() if avail is None else avail
+        if dist.local_world <= 1:
+            if self.nbytes > 0.9 * avail:
+                raise RuntimeError(f"host store of {self.nbytes / 1e9:.2f} GB does not fit: "
+                                   f"{avail / 1e9:.2f} GB available")
+            self.tensor = torch.empty(self.shape, dtype=torch.uint8, pin_memory=pin)
+            fill(self.tensor.numpy())
+            self.shared = False
+            return
+        st = os.statvfs(self.SHM_DIR)
+        shm_free = st.f_bavail * st.f_frsize
+        if self.nbytes > shm_free or self.nbytes > 0.9 * avail:
+            raise RuntimeError(f"{dist.local_world} local ranks share one host store of {self.nbytes / 1e9:.2f} GB, "
+                               f"but {self.SHM_DIR} has {shm_free / 1e9:.2f} GB free and the host "
+                               f"{avail / 1e9:.2f} GB available")
+        self._path = os.path.join(self.SHM_DIR, f"{tag}_{os.environ.get('MASTER_PORT', '0')}")
+        if dist.local == 0:
+            fd = os.open(self._path, os.O_CREAT | os.O_EXCL | os.O_RDWR, 0o600)
+            try:
+                os.ftruncate(fd, self.nbytes)
+                self._mm = mmap.mmap(fd, self.nbytes)
+            finally:
+                os.close(fd)
+            fill(np.frombuffer(self._mm, dtype=np.uint8).reshape(self.shape))
+        dist.barrier()
+        if dist.local != 0:
+            fd = os.open(self._path, os.O_RDWR)
+            try:
+                self._mm = mmap.mmap(fd, self.nbytes)
+            finally:
+                os.close(fd)
+        dist.barrier()
+        if dist.local == 0:
+            os.unlink(self._path)  # every rank holds a mapping; the name is no longer needed
+        self._path = None
+        self.tensor = torch.from_numpy(np.frombuffer(self._mm, dtype=np.uint8).reshape(self.shape))
+        self.shared = True
+        if pin:
+            # page-locked for this rank's GPU; mapped, so kernels can read it
+            rc = torch.cuda.cudart().cudaHostRegister(self.tensor.data_ptr(), self.nbytes, 3)
+            if int(rc) != 0:
+                raise RuntimeError(f"cudaHostRegister of the shared host store failed ({int(rc)})")
+            self.registered = True
+
+    def close(self):
+        if self.registered:
+            import torch
+            torch.cuda.cudart().cudaHostUnregister(self.tensor.data_ptr())
+            self.registered = False
+        self.tensor = None
+        if self._mm is not None:
+            try:
+                self._mm.close()
+            except BufferError:
+                pass  # views still alive; the mapping goes with the process
+            self._mm = None
+
+
 # ------------------------------------------------------------- the model
 class Model:
     """30 MoE layers of synthetic weights: routers, shared experts and the
     routed expert blobs, either streamed (pinned host store + HBM slot
     caches) or resident in HBM."""
 
-    def __init__(self, args, dims, max_tokens, streaming, store=None):
+    def __init__(self, args, dims, max_tokens, streaming, store=None, dist=None):
         import torch
 
         from expert_streaming_decode_b200 import moe, synth
@@ -246,10 +338,18 @@ class Model:
             self.bias.append(None if b is None else torch.from_numpy(b).to(dev))
             self.shared.append(torch.from_numpy(synth.expert_blob(args.seed, l, 0, dims.D, dims.FS, shared=True)).to(dev))
         t0 = time.time()
+        self.host_store = None
         if store is None:
-            store = torch.empty((self.L, dims.E, self.stride), dtype=torch.uint8, pin_memory=streaming)
-            view = store.numpy()
-            synth.fill_store(view[:, :, :self.nb], args.seed, synth.Dims(**{**dims.as_dict(), "L": self.L}))
+            sd = synth.Dims(**{**dims.as_dict(), "L": self.L})
+
+            def fill(view):
+                synth.fill_store(view[:, :, :self.nb], args.seed, sd)
+            if streaming:
+                self.host_store = HostStore((self.L, dims.E, self.stride), fill, dist or Dist())
+                store = self.host_store.tensor
+            else:
+                store = torch.empty((self.L, dims.E, self.stride), dtype=torch.uint8)
+                fill(store.numpy())
         self.gen_s = time.time() - t0
         if streaming:
             self.store = store
@@ -279,7 +379,8 @@ class Model:
                                for l in range(self.L)]
             else:
                 self.caches = [moe.slot_cache(self.slots[l], self.stride, self.state[l], store[l], self.stride,
-                                              policy=pol, decay_period=per)
+                                              policy=pol, decay_period=per,
+                                              direct=getattr(args, "fill", "copy") == "direct")
                                for l in range(self.L)]
             self.W = [moe.layer_weights(self.wq[l], self.ws[l], self.shared[l]) for l in range(self.L)]
             self.nexts = None
@@ -546,9 +647,7 @@ class OracleDecoder:
         blobs = Lazy()
         _, _, _, y = self.O.moe_token(d.as_dict(), self.x, wq, ws, self.bias[l], self.shared[l],
                                       [blobs[e] if e in ids else np.zeros(1, np.uint8) for e in range(d.E)])
-        self.r = self.r + y
-        rms = np.sqrt(np.mean(self.r * self.r) + 1e-6)
-        self.x = self.synth.to_bf16_bits((self.r / rms).astype(np.float32))
+        self.r, self.x = self.O.residual_rmsnorm(self.r, y)
         self.layer += 1
         if self.layer == self.L:
             self.layer = 0
@@ -936,13 +1035,14 @@ def main():
     if args.workload == "prefill" and args.steps == 240 and args.warmup == 16:
         args.steps, args.warmup = 4, 1  # a chunk is ~9 GB of cold fills: keep the default run short
     streaming = args.workload in ("decode_stream", "prefill")
-    model = Model(args, dims, max_tokens=T, streaming=streaming)
+    model = Model(args, dims, max_tokens=T, streaming=streaming, dist=dist)
     W, K = args.warmup, args.steps
     ntok = W + K
     xs = np.stack([synth.hidden_batch(args.seed + 17, range(i * T, i * T + T), 0, dims.D) for i in range(ntok)])
     x_dev = torch.from_numpy(xs.view(np.int16)).cuda()
 
-    # ---- timed pass: inputs resident in HBM, no instrumentation
+    # ---- timed pass: inputs resident in HBM, no instrumentation; the cache
+    # counters are read on the device (no host round trip per layer)
     runner = Runner(model, T, graph=not streaming)
     runner.cold_each_step = args.workload == "prefill"
     model.reset()
@@ -950,11 +1050,12 @@ def main():
     clocks = ClockSampler(dist.local)
     if not args.profile:
         clocks.start()
-    acc_t = {"misses": 0, "distinct": 0, "h2d": 0}
+    st0 = model.ctx.stats() if streaming else None
     pf0 = moe_prefetch_stats(model)
-    ms, launches = timed(dist, model, lambda: runner.run(x_dev, K, W, trace_acc=acc_t if streaming else None))
+    ms, launches = timed(dist, model, lambda: runner.run(x_dev, K, W))
     clk = clocks.stop() if not args.profile else None
     pf1 = moe_prefetch_stats(model)
+    st1 = model.ctx.stats() if streaming else None
 
     # ---- kernel timing pass: event pairs around every kernel (this serialises
     # the kernels, so it is kept out of the pass above)
@@ -964,13 +1065,13 @@ def main():
     runner_p.cold_each_step = args.workload == "prefill"
     runner_p.run(x_dev, min(W, 2), 0)
     model.ctx.profile(True)
-    acc_p = {"misses": 0, "distinct": 0, "h2d": 0}
-    ms_p, _ = timed(dist, model, lambda: runner_p.run(x_dev, kp, W, trace_acc=acc_p if streaming else None))
+    ms_p, _ = timed(dist, model, lambda: runner_p.run(x_dev, kp, W))
     model.ctx.profile(False)
     prof = model.ctx.profile_read()
 
     tokens_all = dist.sum(K * T)
     value = tokens_all / (ms * 1e-3)
+    layer_kernel = prof["layer"][1] > 0
     line = {"metric": METRIC_PREFILL if args.workload == "prefill" else METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": dist.world, "steps": K, "warmup": W,
             "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -980,6 +1081,8 @@ def main():
     cfg = {"workload": args.workload, "layers": args.layers, "batch": T, "slots": args.slots if streaming else None,
            "cache_policy": (args.policy + (f"_{args.decay_period}" if args.policy == "lfu_decay" else ""))
            if streaming else None,
+           "miss_fill": (("layer kernel reads pinned host memory" if args.fill == "direct" and T == 1
+                          else "copy engine") if streaming and not args.store_file else None),
            "prefetch_buffers": args.prefetch if streaming else None,
            "store": (("file, O_DIRECT" if args.direct else "file, page cache") if args.store_file else "pinned host memory")
            if streaming else None,
@@ -989,36 +1092,43 @@ def main():
                   if streaming else "working set > L2: 12.85 GB of resident experts")}
     line["config"] = cfg
 
-    # ---- rooflines from the live kernel timings
+    # ---- kernel rooflines from the live kernel timings
     hbm_peak, peak_kind = peaks()
     n_layer_tok = kp * args.layers
-    if T == 1:
-        distinct = float(dims.K)
-    else:
-        distinct = (acc_p["distinct"] / max(1, n_layer_tok)) if streaming else dims.E * (1 - (1 - dims.K / dims.E) ** T)
+    distinct = float(dims.K) if T == 1 else dims.E * (1 - (1 - dims.K / dims.E) ** T)
     gu_b, dn_b, router_b = model.token_bytes_hbm(distinct)
     kern = {}
-    for kind, byts in (("gate_up", gu_b), ("down", dn_b), ("router", router_b)):
+    kinds = (("layer", gu_b + dn_b + router_b),) if layer_kernel else \
+        (("gate_up", gu_b), ("down", dn_b), ("router", router_b))
+    for kind, byts in kinds:
         tms, cnt = prof[kind]
         if cnt:
             kern[kind] = {"ms_total": tms, "launches": cnt, "bytes_per_layer_token": byts,
+                          "us_per_launch": 1e3 * tms / cnt,
                           "gbs": byts * n_layer_tok / (tms * 1e-3) / 1e9}
     for kind in ("plan", "worklist", "harness"):
         tms, cnt = prof[kind]
         if cnt:
             kern[kind] = {"ms_total": tms, "launches": cnt}
-    dom = max(("gate_up", "down"), key=lambda k: kern[k]["ms_total"])
+    dom = "layer" if layer_kernel else max(("gate_up", "down"), key=lambda k: kern[k]["ms_total"])
     ach = kern[dom]["gbs"]
     gemm = T >= model.moe.lib.moe_gemm_min_tokens()
-    kname = "grouped_gemm_kernel (tcgen05)" if gemm else "gemv_decode_kernel" if T == 1 else "stream_gemv_kernel"
-    line["roofline"] = {"bound": "hbm", "kernel": f"{kname} ({dom})",
-                        "achieved": ach, "peak": hbm_peak,
-                        "unit": "GB/s", "frac": ach / hbm_peak,
-                        # recorded for the one-token GEMV kernels only
-                        "traffic": recorded_traffic(f"{args.workload}:{dom}") if not gemm else None,
-                        "traffic_unit": "DRAM bytes per layer-token (ncu, profiles/traffic.json)",
-                        "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
-                        else "fallback 6650 GB/s"}
+    kname = ("layer_decode_kernel (one launch per layer)" if layer_kernel else
+             "grouped_gemm_kernel (tcgen05)" if gemm else "gemv_decode_kernel" if T == 1 else "stream_gemv_kernel")
+    hbm_roof = {"bound": "hbm", "kernel": kname if layer_kernel else f"{kname} ({dom})",
+                "achieved": ach, "peak": hbm_peak, "unit": "GB/s", "frac": ach / hbm_peak,
+                "traffic": (recorded_traffic(f"{args.workload}:{dom}") if not gemm else None),
+                "traffic_unit": "DRAM bytes per layer-token (ncu, profiles/traffic.json)",
+                "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
+                else "fallback 6650 GB/s",
+                "measured_in": f"a separate pass of {kp} steps with an event pair around every kernel launch"}
+    if not streaming and T == 1:
+        # the step-level rate of the timed pass (the graph keeps launches chained)
+        step_bytes = args.layers * (gu_b + dn_b + router_b)
+        hbm_roof["step_level"] = {"achieved": step_bytes / (ms / K * 1e-3) / 1e9,
+                                  "frac": step_bytes / (ms / K * 1e-3) / 1e9 / hbm_peak,
+                                  "bytes_per_step": step_bytes}
+    line["roofline"] = hbm_roof
     if gemm:
         # the grouped GEMM's FLOPs: 2 * pairs * (3 * F * D) routed + 2 * T * (3 * FS * D) shared per layer
         flop_layer = 2.0 * T * dims.K * 3 * dims.F * dims.D + 2.0 * T * 3 * dims.FS * dims.D
@@ -1033,59 +1143,60 @@ def main():
     line["kernels_note"] = (f"per-kernel times from a separate pass of {kp} steps with an event pair around every "
                             "kernel (serialised: no overlap between kernels)")
     if streaming:
-        h2d_ms, h2d_n = prof["h2d"]
-        peak_h2d = h2d_peak_gbs(torch)
-        got = acc_p["h2d"] / (h2d_ms * 1e-3) / 1e9 if h2d_ms > 0 else 0.0
-        # host->device bytes per token: the misses not served from a staged
-        # blob plus the look-ahead copies (wrong guesses included)
+        d_st = {k: st1[k] - st0[k] for k in st1}
+        planned = max(1, d_st["planned"])
+        miss_tok = d_st["miss_bytes"] / (K * T)
         pf_iss, pf_used = pf1[0] - pf0[0], pf1[1] - pf0[1]
-        pcie_tok = (acc_t["h2d"] - pf_used + pf_iss) / (K * T)
-        avg = pcie_tok * (value / dist.world) / 1e9  # each rank has its own link
-        line["h2d"] = {"achieved": got, "peak": peak_h2d, "unit": "GB/s", "frac": got / peak_h2d if peak_h2d else None,
-                       "peak_source": "measured in this run: 256 MiB pinned->device cudaMemcpyAsync, best of 6",
-                       "bytes_per_token": pcie_tok, "miss_bytes_per_token": acc_t["h2d"] / (K * T),
-                       "copy_batches": h2d_n,
-                       "average": avg, "average_frac": avg / peak_h2d if peak_h2d else None,
-                       "measured_in": "achieved: the kernel timing pass (miss copy batches bracketed by events on the "
-                                      "side stream); average: host->device bytes per token x tokens/s of the timed pass"}
-        if model.nexts is not None:
-            # staged blobs reach their slots device-to-device inside the bracketed
-            # batches, so only the time-averaged rate is a host->device figure
-            line["h2d"].update(achieved=avg, frac=avg / peak_h2d if peak_h2d else None,
-                               measured_in="time-averaged over the timed pass: host->device bytes per token "
-                                           "(misses not served from staged blobs + look-ahead copies) x tokens/s")
+        link_tok = miss_tok + (pf_iss - pf_used) / (K * T)  # bytes that crossed the host link per token
+        peak_h2d = h2d_peak_gbs(torch)
+        useful = miss_tok * (value / dist.world) / 1e9      # every missed expert crosses the link once
+        line["hit_rate"] = 1.0 - d_st["misses"] / planned
+        line["misses_per_token"] = d_st["misses"] / (K * T)
+        line["miss_bytes_per_token"] = miss_tok
+        if T == 1:
+            # the identity miss bytes = (1 - hit) x layers x top-k x blob for one-token steps,
+            # and the pages' repeat statistics of the routing (40 % / 57 %)
+            want = (1.0 - line["hit_rate"]) * args.layers * dims.K * model.nb
+            line["miss_bytes_check"] = {"measured": miss_tok, "from_hit_rate": want,
+                                        "holds": abs(miss_tok - want) < 1.0}
+            line["expert_repeat"] = {"next_token": d_st["repeat_prev"] / planned,
+                                     "within_two_tokens": d_st["repeat_prev2"] / planned,
+                                     "pages": {"next_token": 0.40, "within_two_tokens": 0.57},
+                                     "note": "share of a token's selected experts (per layer) also selected by the "
+                                             "previous token / one of the two previous tokens, over the timed tokens"}
+        pcie = {"bound": "pcie", "achieved": useful, "peak": peak_h2d, "unit": "GB/s",
+                "frac": useful / peak_h2d if peak_h2d else None, "traffic": link_tok,
+                "traffic_unit": "bytes over the host link per token (misses not served from staged blobs + "
+                                "look-ahead copies)",
+                "peak_source": "measured in this run: 256 MiB pinned->device cudaMemcpyAsync, best of 6",
+                "measured_in": "timed pass: missed-expert bytes per token (device counters) x tokens/s"}
+        if args.workload == "decode_stream" and not args.store_file:
+            # the miss path bounds the streamed decode: the link is the primary
+            # roofline, the layer's HBM kernel the secondary
+            line["roofline"] = {**pcie, "hbm_kernel": hbm_roof}
+        else:
+            line["pcie"] = pcie
+        h2d_ms, h2d_n = prof["h2d"]
+        if h2d_n:
+            line["copy_batches"] = {"count": h2d_n, "ms_total": h2d_ms,
+                                    "note": "batches of miss copies on the side stream, kernel timing pass"}
         if args.store_file:
             fstride = (model.nb + 4095) // 4096 * 4096
             paths = [os.path.join(args.store_file, f"layer{l:02d}.experts") for l in range(model.L)]
             fpk = file_read_peak_gbs(paths, fstride, args.direct)
-            line["h2d"]["note"] = ("misses are read from the expert files (positional reads into pinned staging, "
-                                   "4 in flight) and then copied: achieved covers read + copy")
-            line["file_read"] = {"achieved": got, "peak": fpk, "unit": "GB/s", "frac": got / fpk if fpk else None,
+            line["file_read"] = {"achieved": useful, "peak": fpk, "unit": "GB/s",
+                                 "frac": useful / fpk if fpk else None,
                                  "peak_source": "measured in this run: 512 MiB of expert-sized positional reads, "
-                                                "4 threads" + (", O_DIRECT" if args.direct else ", page cache")}
-        line["hit_rate"] = 1.0 - acc_t["misses"] / max(1, acc_t["distinct"])
-        line["misses_per_token"] = acc_t["misses"] / (K * T)
-        if T == 1:
-            # the identity miss bytes = (1 - hit) x layers x top-k x blob for one-token steps,
-            # and the pages' repeat statistics of the routing (40 % / 57 %)
-            line["miss_bytes_check"] = {
-                "measured": acc_t["h2d"] / K,
-                "from_hit_rate": (1.0 - line["hit_rate"]) * args.layers * dims.K * model.nb,
-                "holds": abs(acc_t["h2d"] / K - (1.0 - line["hit_rate"]) * args.layers * dims.K * model.nb) < 1.0}
-            n_rep = max(1, acc_t.get("rep_n", 0))
-            line["expert_repeat"] = {"next_token": acc_t.get("rep1", 0) / n_rep,
-                                     "within_two_tokens": acc_t.get("rep2", 0) / n_rep,
-                                     "pages": {"next_token": 0.40, "within_two_tokens": 0.57},
-                                     "note": "share of a token's selected experts (per layer) also selected by the "
-                                             "previous token / one of the two previous tokens, over the timed tokens"}
+                                                "4 threads" + (", O_DIRECT" if args.direct else ", page cache"),
+                                 "note": "misses are read from the expert files (positional reads into pinned "
+                                         "staging, 4 in flight) and then copied"}
         if model.nexts is not None:
-            iss, used = pf1[0] - pf0[0], pf1[1] - pf0[1]
-            line["prefetch"] = {"buffers": args.prefetch, "issued_bytes_per_token": iss / (K * T),
-                                "used_bytes_per_token": used / (K * T),
-                                "wasted_bytes_per_token": (iss - used) / (K * T),
-                                "miss_bytes_served": used / max(1, acc_t["h2d"]),
-                                "note": "measured over the timed pass; the misses' trace bytes include the ones "
-                                        "filled from staged blobs (device-to-device)"}
+            line["prefetch"] = {"buffers": args.prefetch, "issued_bytes_per_token": pf_iss / (K * T),
+                                "used_bytes_per_token": pf_used / (K * T),
+                                "wasted_bytes_per_token": (pf_iss - pf_used) / (K * T),
+                                "miss_bytes_served": pf_used / max(1, d_st["miss_bytes"]),
+                                "note": "measured over the timed pass; staged blobs reach their slots device to "
+                                        "device"}
     line["gpu_launches"] = int(dist.sum(launches))
     if clk:
         line["clocks"] = clk

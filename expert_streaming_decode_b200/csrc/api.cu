@@ -23,6 +23,7 @@
 #include "common.cuh"
 #include "ffn.cuh"
 #include "filestore.cuh"
+#include "layer.cuh"
 #include "plan.cuh"
 #include <cstdlib>
 
@@ -100,6 +101,17 @@ struct moe_ctx {
     // host mirror of each cache's residency (slot of expert e, -1: absent),
     // kept from the plans the host reads; decides what is worth prefetching
     std::unordered_map<const int32_t*, std::vector<int16_t>> mirror;
+    // one-token layer kernel (layer.cu): grid, support for the dims, scratch
+    int layer_G = 0;
+    bool layer_ok = false;
+    bool layer_on = true;
+    bool layer_pdl = true;
+    int layer_hvals = 0;
+    float* layer_logits = nullptr;
+    float* layer_partials = nullptr;  // [4 * G][32]: gate/up then down
+    unsigned* layer_bar = nullptr;    // [4]
+    uint64_t* stats = nullptr;        // [MOE_STATS] device counters
+    std::unordered_map<const void*, const uint8_t*> direct_store;  // host store -> device-accessible address
     // instrumentation (moe_ctx_profile)
     struct Rec {
         int kind;
@@ -153,6 +165,10 @@ void free_ctx(moe_ctx* c) {
     }
     for (auto e : c->pool) cudaEventDestroy(e);
     cudaFree(c->status);
+    cudaFree(c->layer_logits);
+    cudaFree(c->layer_partials);
+    cudaFree(c->layer_bar);
+    cudaFree(c->stats);
     cudaFree(c->wl);
     cudaFree(c->entries);
     cudaFree(c->rows);
@@ -464,7 +480,11 @@ int check_cache(const moe_ctx* c, const moe_slot_cache* cache) {
     if (!aligned(cache->state, 16)) return MOE_ERR_ARG;
     if (cache->store && cache->store_stride < c->blob_routed) return MOE_ERR_ARG;
     if (cache->policy < MOE_POLICY_LFU || cache->policy > MOE_POLICY_LFU_IN_CACHE) return MOE_ERR_ARG;
-    if (cache->source != MOE_SOURCE_HOST && cache->source != MOE_SOURCE_FILE) return MOE_ERR_ARG;
+    if (cache->source != MOE_SOURCE_HOST && cache->source != MOE_SOURCE_FILE && cache->source != MOE_SOURCE_HOST_DIRECT)
+        return MOE_ERR_ARG;
+    if (cache->source == MOE_SOURCE_HOST_DIRECT &&
+        (!cache->store || !aligned(cache->store, 16) || cache->store_stride % 16))
+        return MOE_ERR_ARG;
     if (cache->source == MOE_SOURCE_FILE && (cache->store_fd < 0 || cache->store_stride < c->blob_routed))
         return MOE_ERR_ARG;
     return MOE_OK;
@@ -544,6 +564,18 @@ int moe_ctx_create(const moe_dims* dims, int device, moe_ctx** out) {
     ok = ok && dalloc(&c->gate_w, pairs) == cudaSuccess;
     ok = ok && dalloc(&c->pair_slot, pairs) == cudaSuccess;
     ok = ok && dalloc(&c->pair_wave, pairs) == cudaSuccess;
+    ok = ok && layer_grid(device, &c->layer_G) == cudaSuccess;
+    if (ok) {
+        c->layer_ok = layer_supported(d.d_model, d.n_experts, d.top_k, d.d_ff, d.d_ff_shared, d.n_slots, c->layer_G);
+        c->layer_hvals = layer_hvals(d.d_model, d.top_k, d.d_ff, d.d_ff_shared, c->layer_G);
+        if (const char* v = std::getenv("MOE_LAYER_KERNEL")) c->layer_on = !(v[0] == '0');
+    }
+    ok = ok && dalloc(&c->layer_logits, size_t(d.n_experts)) == cudaSuccess;
+    ok = ok && dalloc(&c->layer_partials, size_t(4) * c->layer_G * 32) == cudaSuccess;
+    ok = ok && dalloc(&c->layer_bar, 4) == cudaSuccess;
+    ok = ok && dalloc(&c->stats, MOE_STATS) == cudaSuccess;
+    ok = ok && cudaMemset(c->layer_bar, 0, 4 * sizeof(unsigned)) == cudaSuccess;
+    ok = ok && cudaMemset(c->stats, 0, MOE_STATS * sizeof(uint64_t)) == cudaSuccess;
     ok = ok && cudaMemset(c->status, 0, sizeof(int)) == cudaSuccess;
     ok = ok && cudaMemset(c->counters_gu, 0, tiles_gu * sizeof(int)) == cudaSuccess;
     ok = ok && cudaMemset(c->counters_dn, 0, size_t(d.d_model / kChunkRows) * sizeof(int)) == cudaSuccess;
@@ -649,7 +681,7 @@ static int plan_call(moe_ctx* c, moe_slot_cache* cache, const int32_t* ids, int 
     cudaError_t e = launch_plan(ids, T * c->d.top_k, c->d.n_experts, c->d.n_slots, cache->policy, cache->decay_period,
                                 cache->state, step, pair_slot,
                                 c->pair_wave, need_host ? c->mbox_dev : nullptr, seq, c->status, nullptr,
-                                DecodeWLTarget{}, DecodeWLTarget{}, c->pdl, s);
+                                DecodeWLTarget{}, DecodeWLTarget{}, c->stats, c->blob_routed, c->pdl, s);
     prof_mark(c, MOE_PROF_PLAN, false, s);
     c->launches += 1;
     if (e != cudaSuccess) return MOE_ERR_CUDA;
@@ -703,6 +735,92 @@ int moe_expert_ffn(moe_ctx* c, const uint16_t* x, int T, int top_k, const int32_
 
 }  // extern "C"
 
+// Device-accessible address of a pinned host store (the kernels read missed
+// experts from it directly); null when the memory is not pinned and mapped.
+static const uint8_t* direct_store(moe_ctx* c, const uint8_t* store) {
+    auto it = c->direct_store.find(store);
+    if (it != c->direct_store.end()) return it->second;
+    cudaPointerAttributes pa;
+    if (cudaPointerGetAttributes(&pa, store) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    if (pa.type != cudaMemoryTypeHost || !pa.devicePointer) return nullptr;
+    const uint8_t* dp = static_cast<const uint8_t*>(pa.devicePointer);
+    c->direct_store[store] = dp;
+    return dp;
+}
+
+// One token through the whole layer in one launch (layer.cu): experts
+// resident (cache == null) or served from the slot cache with misses read
+// straight from the pinned host store by the kernel.
+static int run_layer_kernel(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache* cache, const uint16_t* x,
+                            uint32_t step, const float* bias, float* y, uint16_t* y_bf16, int32_t* ids, float* gate_w,
+                            moe_plan_trace* trace, cudaStream_t s) {
+    if (!aligned(W->router_q, 16) || !aligned(W->router_s, 4)) return MOE_ERR_ARG;
+    LayerArgs a{};
+    a.x = x;
+    a.wq = W->router_q;
+    a.ws = W->router_s;
+    a.bias = bias;
+    a.shared_blob = W->shared_blob;
+    if (!cache) {
+        a.experts = W->experts;
+        a.expert_stride = W->expert_stride;
+    } else {
+        a.slots = cache->slots;
+        a.slot_stride = cache->slot_stride;
+        a.state = cache->state;
+        a.store = direct_store(c, cache->store);
+        if (!a.store) return MOE_ERR_ARG;
+        a.store_stride = cache->store_stride;
+        a.policy = cache->policy;
+        a.decay_period = cache->decay_period;
+    }
+    a.step = step;
+    a.D = c->d.d_model;
+    a.E = c->d.n_experts;
+    a.K = c->d.top_k;
+    a.F = c->d.d_ff;
+    a.FS = W->shared_blob ? c->d.d_ff_shared : 0;
+    a.S = c->d.n_slots;
+    a.blob_bytes = c->blob_routed;
+    a.hvals = c->layer_hvals;
+    a.y = y;
+    a.y_bf16 = y_bf16;
+    a.ids = ids;
+    a.gate_w = gate_w;
+    a.mailbox = (cache && trace) ? c->mbox_dev : nullptr;
+    a.seq = ++c->seq;
+    a.stats = cache ? c->stats : nullptr;
+    a.logits = c->layer_logits;
+    a.h = c->h;
+    a.partials_gu = c->layer_partials;
+    a.partials_dn = c->layer_partials + size_t(2) * c->layer_G * 32;
+    a.counters_gu = c->counters_gu;
+    a.counters_dn = c->counters_dn;
+    a.bar = c->layer_bar;
+    a.status = c->status;
+    prof_mark(c, MOE_PROF_LAYER, true, s);
+    cudaError_t e = launch_layer(a, c->layer_G, c->pdl && c->layer_pdl, s);
+    if (e != cudaSuccess && c->pdl && c->layer_pdl) {
+        // a cooperative launch the driver will not chain programmatically
+        cudaGetLastError();
+        c->layer_pdl = false;
+        e = launch_layer(a, c->layer_G, false, s);
+    }
+    prof_mark(c, MOE_PROF_LAYER, false, s);
+    c->launches += 1;
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    if (cache && trace) {
+        const int r = wait_mailbox(c, a.seq, 10000);
+        if (r != MOE_OK) return r;
+        mirror_update(c, cache);
+        copy_trace(c->mbox_host, trace, c->blob_routed, uint64_t(c->mbox_host->n_misses) * c->blob_routed);
+    }
+    return MOE_OK;
+}
+
 // the layer; `next` (or null) asks for a look-ahead prefetch of the next layer
 static int layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache* cache, const uint16_t* x, int T,
                          uint32_t step, const float* bias, float* y, uint16_t* y_bf16, int32_t* ids, float* gate_w,
@@ -722,6 +840,12 @@ static int layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache*
     float* gw = gate_w ? gate_w : c->gate_w;
     const int K = c->d.top_k;
     int r;
+    // look-ahead: the next layer's router on this layer's input, on its own
+    // stream, while this layer runs (one token, host stores, buffers configured)
+    const bool prefetch = next && T == 1 && c->pf_n > 0 && next->W && next->W->router_q && next->W->router_s &&
+                          next->cache && next->cache->source == MOE_SOURCE_HOST && next->cache->store;
+    if (T == 1 && c->layer_ok && c->layer_on && !prefetch && (!cache || cache->source == MOE_SOURCE_HOST_DIRECT))
+        return run_layer_kernel(c, W, cache, x, step, bias, y, y_bf16, id, gw, trace, s);
     if (T == 1 && !cache) {
         // one token, resident: the router writes the work list itself
         const DecodeWLTarget t = decode_target(c, c->wl, c->entries, c->rows, W->experts, W->expert_stride,
@@ -734,10 +858,6 @@ static int layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache*
         if (e != cudaSuccess) return MOE_ERR_CUDA;
         return run_ffn_list(c, c->wl, c->entries, c->rows, x, 1, nullptr, y, y_bf16, s, W->shared_blob);
     }
-    // look-ahead: the next layer's router on this layer's input, on its own
-    // stream, while this layer runs (one token, host stores, buffers configured)
-    const bool prefetch = next && T == 1 && c->pf_n > 0 && next->W && next->W->router_q && next->W->router_s &&
-                          next->cache && next->cache->source == MOE_SOURCE_HOST && next->cache->store;
     if (prefetch) {
         if (cudaEventRecord(c->ev_x, s) != cudaSuccess || cudaStreamWaitEvent(c->pf_stream, c->ev_x, 0) != cudaSuccess)
             return MOE_ERR_CUDA;
@@ -779,7 +899,8 @@ static int layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache*
     prof_mark(c, MOE_PROF_PLAN, true, s);
     cudaError_t e = launch_plan(id, T * K, c->d.n_experts, c->d.n_slots, cache->policy, cache->decay_period,
                                 cache->state, step, c->pair_slot,
-                                c->pair_wave, c->mbox_dev, seq, c->status, gw, t_sh, t_rt, c->pdl, s);
+                                c->pair_wave, c->mbox_dev, seq, c->status, gw, t_sh, t_rt, c->stats, c->blob_routed,
+                                c->pdl, s);
     prof_mark(c, MOE_PROF_PLAN, false, s);
     c->launches += 1;
     if (e != cudaSuccess) return MOE_ERR_CUDA;
@@ -931,6 +1052,18 @@ int moe_prefetch_stats(const moe_ctx* c, uint64_t* issued_bytes, uint64_t* used_
     if (issued_bytes) *issued_bytes = c->pf_issued;
     if (used_bytes) *used_bytes = c->pf_used;
     return MOE_OK;
+}
+
+int moe_ctx_stats(moe_ctx* c, cudaStream_t s, uint64_t* out) {
+    if (!c || !out) return MOE_ERR_ARG;
+    if (cudaMemcpyAsync(out, c->stats, MOE_STATS * sizeof(uint64_t), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return cudaStreamSynchronize(s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_ctx_stats_reset(moe_ctx* c, cudaStream_t s) {
+    if (!c) return MOE_ERR_ARG;
+    return cuda_status(cudaMemsetAsync(c->stats, 0, MOE_STATS * sizeof(uint64_t), s));
 }
 
 int moe_residual_rmsnorm(moe_ctx* c, float* r, const float* y, uint16_t* x_next, int T, cudaStream_t s) {

@@ -66,11 +66,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Bounded wait for the phase with the given parity to complete.  Returns false
-// (after recording MOE_ERR_TIMEOUT) if it never does.
+// Nanoseconds of the GPU's global timer.
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+// Longest legitimate wait of any barrier here: copies and peer CTAs finish in
+// microseconds (a missed expert read over the host link in well under 1 ms).
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+
+// Bounded wait for the phase with the given parity to complete: gives up
+// after kWaitLimitNs of global time or kSpinLimit tries, whichever comes
+// first, and returns false after recording MOE_ERR_TIMEOUT.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
-    for (uint32_t i = 0; i < kSpinLimit; ++i)
+    unsigned long long t0 = 0;
+    for (uint32_t i = 0; i < kSpinLimit; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 255) == 255) {
+            const unsigned long long t = global_ns();
+            if (t0 == 0) t0 = t;
+            else if (t - t0 > kWaitLimitNs) break;
+        }
+    }
     set_status(status, MOE_ERR_TIMEOUT);
     return false;
 }

@@ -35,7 +35,8 @@ __global__ void __launch_bounds__(kPlanThreads) cache_plan_kernel(
     const int32_t* __restrict__ ids, int npairs, int E, int S, int policy, uint32_t decay_period,
     int32_t* __restrict__ state, uint32_t step,
     int32_t* __restrict__ pair_slot, int32_t* __restrict__ pair_wave, PlanMailbox* mailbox, uint32_t seq,
-    int* status, const float* __restrict__ gate_w, DecodeWLTarget wl_shared, DecodeWLTarget wl_routed) {
+    int* status, const float* __restrict__ gate_w, DecodeWLTarget wl_shared, DecodeWLTarget wl_routed,
+    uint64_t* stats, uint64_t blob_bytes) {
     extern __shared__ int32_t psm[];
     uint32_t* mult = reinterpret_cast<uint32_t*>(psm);   // [E] selections in this call
     uint32_t* count = mult + E;                           // [E]
@@ -97,7 +98,19 @@ __global__ void __launch_bounds__(kPlanThreads) cache_plan_kernel(
             n += __popc(b);
         }
         __syncwarp();
-        int n_miss = 0;
+        int n_miss = 0, rep1 = 0, rep2 = 0;
+        // experts also chosen by the previous call (last_use == step) or by
+        // one of the two previous calls (last_use >= step - 1), before update
+        for (int i = lane; i < n; i += 32) {
+            const uint32_t lu = last[ulist[i]];
+            rep1 += (lu != 0u && lu == step);
+            rep2 += (lu != 0u && lu + 1u >= step);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            rep1 += __shfl_xor_sync(0xffffffffu, rep1, off);
+            rep2 += __shfl_xor_sync(0xffffffffu, rep2, off);
+        }
         const int waves = (n + S - 1) / S;
         for (int w = 0; w < waves; ++w) {
             const int lo = w * S, hi = min(n, (w + 1) * S);
@@ -184,6 +197,15 @@ __global__ void __launch_bounds__(kPlanThreads) cache_plan_kernel(
         }
         if (lane == 0) {
             s_n = n;
+            if (stats) {
+                stats[0] += 1;
+                stats[1] += uint64_t(n - n_miss);
+                stats[2] += uint64_t(n_miss);
+                stats[3] += uint64_t(n_miss) * blob_bytes;
+                stats[4] += uint64_t(rep1);
+                stats[5] += uint64_t(rep2);
+                stats[6] += uint64_t(n);
+            }
             if (mailbox) {
                 mailbox->n_distinct = n;
                 mailbox->n_waves = waves;
@@ -245,7 +267,7 @@ cudaError_t launch_plan(const int32_t* ids, int npairs, int E, int S, int policy
                         int32_t* state, uint32_t step,
                         int32_t* pair_slot, int32_t* pair_wave, PlanMailbox* mailbox, uint32_t seq, int* status,
                         const float* gate_w, const DecodeWLTarget& wl_shared, const DecodeWLTarget& wl_routed,
-                        bool pdl, cudaStream_t s) {
+                        uint64_t* stats, uint64_t blob_bytes, bool pdl, cudaStream_t s) {
     static thread_local int attr_set_for = -1;  // device whose attribute this thread last set
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -258,7 +280,7 @@ cudaError_t launch_plan(const int32_t* ids, int npairs, int E, int S, int policy
     }
     return launch_kernel(cache_plan_kernel, dim3(1), dim3(kPlanThreads), plan_smem_bytes(E, S), s, pdl, 1, ids, npairs,
                          E, S, policy, decay_period, state, step, pair_slot, pair_wave, mailbox, seq, status, gate_w,
-                         wl_shared, wl_routed);
+                         wl_shared, wl_routed, stats, blob_bytes);
 }
 
 __global__ void cache_reset_kernel(int32_t* state, int E, int S) {

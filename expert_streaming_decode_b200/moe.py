@@ -42,7 +42,9 @@ class moe_slot_cache(C.Structure):
                 ("store_file_offset", C.c_uint64)]
 
 
-MOE_SOURCE_HOST, MOE_SOURCE_FILE = 0, 1
+MOE_SOURCE_HOST, MOE_SOURCE_FILE, MOE_SOURCE_HOST_DIRECT = 0, 1, 2
+STAT_NAMES = ("calls", "hits", "misses", "miss_bytes", "repeat_prev", "repeat_prev2", "planned")
+MOE_STATS = 8
 
 
 MOE_POLICY_LFU, MOE_POLICY_LRU, MOE_POLICY_LFU_DECAY, MOE_POLICY_LFU_IN_CACHE = 0, 1, 2, 3
@@ -112,6 +114,10 @@ lib.moe_ctx_profile.restype = _i
 lib.moe_ctx_profile.argtypes = [_vp, _i]
 lib.moe_ctx_profile_read.restype = _i
 lib.moe_ctx_profile_read.argtypes = [_vp, C.POINTER(C.c_double), C.POINTER(C.c_uint64)]
+lib.moe_ctx_stats.restype = _i
+lib.moe_ctx_stats.argtypes = [_vp, _vp, C.POINTER(C.c_uint64)]
+lib.moe_ctx_stats_reset.restype = _i
+lib.moe_ctx_stats_reset.argtypes = [_vp, _vp]
 lib.moe_residual_rmsnorm.restype = _i
 lib.moe_residual_rmsnorm.argtypes = [_vp, _vp, _vp, _vp, _i, _vp]
 lib.moe_bf16_to_f32.restype = _i
@@ -183,7 +189,7 @@ class Ctx:
     def launches(self) -> int:
         return int(lib.moe_ctx_launches(self.h))
 
-    PROF_KINDS = ("router", "plan", "worklist", "gate_up", "down", "harness", "h2d")
+    PROF_KINDS = ("router", "plan", "worklist", "gate_up", "down", "harness", "h2d", "layer")
 
     def profile(self, enable: bool):
         _check(lib.moe_ctx_profile(self.h, int(enable)), "moe_ctx_profile")
@@ -195,6 +201,15 @@ class Ctx:
         _check(lib.moe_ctx_profile_read(self.h, ms, n), "moe_ctx_profile_read")
         return {k: (ms[i], int(n[i])) for i, k in enumerate(self.PROF_KINDS)}
 
+    def stats(self, stream=None) -> dict:
+        """The device cache counters (moe_ctx_stats), by name."""
+        out = (C.c_uint64 * MOE_STATS)()
+        _check(lib.moe_ctx_stats(self.h, _stream(stream), out), "moe_ctx_stats")
+        return {k: int(out[i]) for i, k in enumerate(STAT_NAMES)}
+
+    def stats_reset(self, stream=None):
+        _check(lib.moe_ctx_stats_reset(self.h, _stream(stream)), "moe_ctx_stats_reset")
+
     def state_words(self) -> int:
         return int(lib.moe_cache_state_words(C.byref(self.dims)))
 
@@ -205,12 +220,18 @@ def router_topk(ctx: Ctx, x, wq, ws, bias, T, ids, gate_w, stream=None):
 
 
 def slot_cache(slots, slot_stride, state, store=None, store_stride=0, policy=MOE_POLICY_LFU,
-               decay_period=0, store_fd=None, store_file_offset=0) -> moe_slot_cache:
+               decay_period=0, store_fd=None, store_file_offset=0, direct=False) -> moe_slot_cache:
     """moe_slot_cache for torch tensors.  The struct keeps references to the
     tensors, so their memory lives at least as long as the struct.  With
     store_fd (an open file descriptor) the misses are read from that file at
-    store_file_offset + e * store_stride instead of the pinned `store`."""
+    store_file_offset + e * store_stride instead of the pinned `store`; with
+    direct=True one-token layers read missed experts from the pinned `store`
+    inside the layer kernel (MOE_SOURCE_HOST_DIRECT)."""
     src = MOE_SOURCE_HOST if store_fd is None else MOE_SOURCE_FILE
+    if direct:
+        if store_fd is not None:
+            raise ValueError("direct reads need the pinned host store, not a file")
+        src = MOE_SOURCE_HOST_DIRECT
     c = moe_slot_cache(slots.data_ptr(), slot_stride, state.data_ptr(),
                        None if store is None else store.data_ptr(), store_stride, policy, decay_period,
                        src, -1 if store_fd is None else store_fd, store_file_offset)

@@ -168,7 +168,14 @@ int moe_router_topk(moe_ctx *ctx, const uint16_t *x, const int8_t *wq, const uin
  *   policy        replacement rule (MOE_POLICY_*; 0 = LFU, the pages' rule)
  *   decay_period  MOE_POLICY_LFU_DECAY: counts are halved at the start of
  *                 every call whose step is a positive multiple of it (0: never)
- *   source        MOE_SOURCE_HOST (the pinned `store` above) or
+ *   source        MOE_SOURCE_HOST (the pinned `store` above, misses copied
+ *                 by the copy engine after the host has read the plan),
+ *                 MOE_SOURCE_HOST_DIRECT (the same pinned `store`, 16-byte
+ *                 aligned with store_stride % 16 == 0, but for one-token
+ *                 calls the layer kernel reads each missed expert straight
+ *                 from it over the bus and writes it into its slot as it
+ *                 computes with it: no host round trip; calls of two or more
+ *                 tokens copy as MOE_SOURCE_HOST does), or
  *                 MOE_SOURCE_FILE: expert e is read from file descriptor
  *                 store_fd at byte store_file_offset + e*store_stride with
  *                 positional reads, several in flight, into pinned staging
@@ -194,6 +201,7 @@ typedef struct moe_slot_cache {
 
 #define MOE_SOURCE_HOST 0
 #define MOE_SOURCE_FILE 1
+#define MOE_SOURCE_HOST_DIRECT 2
 
 /* Replacement rules of the slot cache ("El milagro ...", "Mas inteligente
  * que tu RAM": a miss replaces the least frequently used resident expert;
@@ -327,10 +335,14 @@ typedef struct moe_layer_weights {
  * cache == NULL: resident mode, expert e read from W->experts + e*stride.
  * cache != NULL: experts are served from cache->slots; misses are copied from
  * cache->store (host-synchronous on the plan, see moe_cache_plan).
- * T = 1 runs the dequantising GEMV kernels; T >= moe_gemm_min_tokens() (a
- * batched decode step or a prefill chunk) groups the tokens by expert and runs
- * the tcgen05 tensor-core grouped GEMM, one wave of at most n_slots experts at
- * a time.
+ * T = 1 with resident experts or a MOE_SOURCE_HOST_DIRECT cache runs the
+ * whole layer as one cooperative kernel (router, top-K, plan, shared and
+ * routed expert GEMVs, combine; all CTAs resident, two bounded grid-wide
+ * barriers; the plan reaches the host only when a trace is requested); other
+ * one-token calls run the router, plan and dequantising GEMV kernels;
+ * T >= moe_gemm_min_tokens() (a batched decode step or a prefill chunk) groups
+ * the tokens by expert and runs the tcgen05 tensor-core grouped GEMM, one wave
+ * of at most n_slots experts at a time.
  *   x dev bf16 [T][D]; bias dev fp32 [E] or NULL; y dev fp32 [T][D] out;
  *   y_bf16 dev bf16 [T][D] out or NULL; ids/gate_w dev [T][K] out or NULL;
  *   trace host, or NULL. */
@@ -440,7 +452,8 @@ size_t moe_attn_workspace_bytes(int n_heads_q, int head_dim);
 #define MOE_PROF_DOWN      4   /* expert down GEMV + combine kernel */
 #define MOE_PROF_HARNESS   5   /* harness kernels (residual/RMS, bf16 widening) */
 #define MOE_PROF_H2D       6   /* one batch of miss copies on the side stream */
-#define MOE_PROF_KINDS     7
+#define MOE_PROF_LAYER     7   /* one-token layer kernel (the whole layer) */
+#define MOE_PROF_KINDS     8
 
 /* Kernel timing for benchmarks.  While enabled, the context records a pair of
  * CUDA events on the launching stream around every kernel it launches (and
@@ -453,6 +466,28 @@ int moe_ctx_profile(moe_ctx *ctx, int enable);
  * the number of intervals since the previous read; then clears the records.
  * MOE_ERR_CUDA if an event could not be read. */
 int moe_ctx_profile_read(moe_ctx *ctx, double *total_ms, uint64_t *count);
+
+/* Cache counters kept on the device by the plan kernel and the one-token
+ * layer kernel, for every call with a slot cache: calls, hits and misses
+ * (distinct experts), bytes of missed experts, experts also chosen at the
+ * previous step of that cache (last_use == step) and at one of the two
+ * previous steps, and distinct experts planned (the denominator of the two
+ * repeat counts).  Reading them needs no host round trip per call. */
+#define MOE_STAT_CALLS        0
+#define MOE_STAT_HITS         1
+#define MOE_STAT_MISSES       2
+#define MOE_STAT_MISS_BYTES   3
+#define MOE_STAT_REPEAT_PREV  4
+#define MOE_STAT_REPEAT_PREV2 5
+#define MOE_STAT_PLANNED      6
+#define MOE_STATS             8
+
+/* Copies the counters (MOE_STATS words) into out (host) after the work
+ * already on `stream`; waits for it.  MOE_ERR_CUDA on a failed copy. */
+int moe_ctx_stats(moe_ctx *ctx, cudaStream_t stream, uint64_t *out);
+
+/* Zeroes the counters, enqueued on `stream`. */
+int moe_ctx_stats_reset(moe_ctx *ctx, cudaStream_t stream);
 
 /* ------------------------------------------------------ harness helpers
  * Not part of the method: the residual/RMS step a test or benchmark puts

@@ -1,5 +1,6 @@
-"""bench.py's argument rules, on CPU: the look-ahead default and the
-combinations it refuses, and the attention workload's layer mix and bytes."""
+"""bench.py's argument rules, on CPU: the miss-fill and look-ahead defaults
+and the combinations refused, and the attention workload's layer mix and
+bytes."""
 import os
 import sys
 
@@ -20,9 +21,12 @@ def _args(*argv):
         sys.argv = old
 
 
-def test_lookahead_default_only_for_one_token_streamed_decode():
-    assert _args().prefetch == 1
-    assert _args("--prefetch", "0").prefetch == 0
+def test_fill_and_lookahead_defaults():
+    """Misses are filled by the layer kernel by default; the look-ahead is off
+    unless asked for, and only the copy-engine fill can take it."""
+    a = _args()
+    assert a.fill == "direct" and a.prefetch == 0
+    assert _args("--fill", "copy", "--prefetch", "1").prefetch == 1
     assert _args("--workload", "prefill").prefetch == 0
     assert _args("--workload", "decode_resident", "--batch", "8").prefetch == 0
     assert _args("--store-file", "/tmp/x").prefetch == 0
@@ -31,7 +35,8 @@ def test_lookahead_default_only_for_one_token_streamed_decode():
 
 @pytest.mark.parametrize("argv", [("--workload", "prefill", "--prefetch", "1"),
                                   ("--store-file", "/tmp/x", "--prefetch", "2"),
-                                  ("--prefetch", "17")])
+                                  ("--prefetch", "1"),
+                                  ("--fill", "copy", "--prefetch", "17")])
 def test_lookahead_refused_where_it_does_not_apply(argv):
     with pytest.raises(SystemExit):
         _args(*argv)

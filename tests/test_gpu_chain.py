@@ -31,9 +31,10 @@ def O():
     return oracle.get()
 
 
-def _args(layers, slots, prefetch, seed=0):
+def _args(layers, slots, prefetch, fill, seed=0):
     return argparse.Namespace(layers=layers, slots=slots, seed=seed, zipf=1.1, zipf_lambda=synth.ZIPF_LAMBDA,
-                              policy="lfu", decay_period=0, store_file=None, direct=False, prefetch=prefetch)
+                              policy="lfu", decay_period=0, store_file=None, direct=False, prefetch=prefetch,
+                              fill=fill)
 
 
 def _bf16_ulp_diff(a, b):
@@ -44,8 +45,8 @@ def _bf16_ulp_diff(a, b):
     return np.abs(fa - fb) / ulp
 
 
-def _chain(O, d, layers, tokens, slots, prefetch, y_samples):
-    args = _args(layers, slots, prefetch)
+def _chain(O, d, layers, tokens, slots, prefetch, y_samples, fill="copy"):
+    args = _args(layers, slots, prefetch, fill)
     model = bench.Model(args, synth.Dims(**{**d.as_dict(), "L": layers, "S": slots}), max_tokens=1, streaming=True)
     moe = model.moe
     nb = model.nb
@@ -132,20 +133,22 @@ def _chain(O, d, layers, tokens, slots, prefetch, y_samples):
     return stats
 
 
-@pytest.mark.parametrize("prefetch", [0, 2], ids=["no-lookahead", "lookahead-2"])
-def test_chained_decode_tiny_30_layers(O, prefetch):
+@pytest.mark.parametrize("fill,prefetch", [("copy", 0), ("copy", 2), ("direct", 0)],
+                         ids=["copy", "copy-lookahead-2", "direct"])
+def test_chained_decode_tiny_30_layers(O, fill, prefetch):
     """30 chained layers of the scaled-down shape (6 slots), 24 tokens: every
     (token, layer) checked, outputs too."""
     d = synth.TINY
     samples = {(t, l) for t in range(24) for l in range(30)}
-    st = _chain(O, d, layers=30, tokens=24, slots=6, prefetch=prefetch, y_samples=samples)
+    st = _chain(O, d, layers=30, tokens=24, slots=6, prefetch=prefetch, y_samples=samples, fill=fill)
     assert st["misses"] > 0
     if prefetch:
         assert st["pf_used"] > 0
 
 
-@pytest.mark.parametrize("prefetch", [0, 1], ids=["no-lookahead", "lookahead-1"])
-def test_chained_decode_full_shape(O, prefetch):
+@pytest.mark.parametrize("fill,prefetch", [("copy", 0), ("copy", 1), ("direct", 0)],
+                         ids=["copy", "copy-lookahead-1", "direct"])
+def test_chained_decode_full_shape(O, fill, prefetch):
     """8 chained layers of the 26B-A4B shape, 16 slots, Zipf(1.1), 16 tokens:
     ids, gate weights, plans, chained inputs at every (token, layer), slot
     contents every 4th token, outputs on a sample spread over tokens and
@@ -153,7 +156,7 @@ def test_chained_decode_full_shape(O, prefetch):
     d = synth.GEMMA4_26B
     samples = {(0, 0), (0, 7), (1, 3), (3, 1), (5, 6), (7, 2), (8, 5), (10, 0), (11, 4), (13, 7), (15, 1),
                (15, 6)}
-    st = _chain(O, d, layers=8, tokens=16, slots=16, prefetch=prefetch, y_samples=samples)
+    st = _chain(O, d, layers=8, tokens=16, slots=16, prefetch=prefetch, y_samples=samples, fill=fill)
     assert st["misses"] > 0
     if prefetch:
         assert st["pf_issued"] > 0

@@ -36,9 +36,12 @@ def _check_token(O, L, xb, ids, gw, y):
     return err
 
 
+@pytest.mark.parametrize("kernel", ["layer", "split"])
 @pytest.mark.parametrize("d", [TINY, FULL], ids=["tiny", "full"])
-def test_decode_resident_single_layer(O, d):
-    """One layer, all experts resident, 16 sequential decode tokens."""
+def test_decode_resident_single_layer(O, d, kernel, monkeypatch):
+    """One layer, all experts resident, 16 sequential decode tokens: through the
+    one-launch layer kernel and through the separate router / GEMV kernels."""
+    monkeypatch.setenv("MOE_LAYER_KERNEL", "1" if kernel == "layer" else "0")
     L = Layer(d, layer=0, seed=0, zipf_s=None)
     ctx = moe.Ctx.from_dims(d, max_tokens=1)
     W = L.weights()
@@ -71,7 +74,7 @@ def test_batched_decode_resident(O, d, T):
 
 
 def _streaming(O, d, layers, tokens, S, check_y_every=1, T=1, policy=0, period=0, file_dir=None, prefetch=0,
-               same_x=False, stats=None):
+               same_x=False, stats=None, direct=False, counters=None):
     Ls = [Layer(d, layer=l, seed=1, zipf_s=1.1, resident=False, pinned=True) for l in range(layers)]
     ctx = moe.Ctx.from_dims(d, max_tokens=T, S=S)
     caches, states, slotbufs = [], [], []
@@ -92,7 +95,8 @@ def _streaming(O, d, layers, tokens, S, check_y_every=1, T=1, policy=0, period=0
             c = moe.slot_cache(slots, L.stride, state, None, fstride, policy=policy, decay_period=period,
                                store_fd=fd, store_file_offset=4096)
         else:
-            c = moe.slot_cache(slots, L.stride, state, L.store_t, L.stride, policy=policy, decay_period=period)
+            c = moe.slot_cache(slots, L.stride, state, L.store_t, L.stride, policy=policy, decay_period=period,
+                               direct=direct)
         moe.cache_reset(ctx, c)
         caches.append(c)
         states.append(state)
@@ -103,6 +107,9 @@ def _streaming(O, d, layers, tokens, S, check_y_every=1, T=1, policy=0, period=0
     gw = torch.empty((T, d.K), dtype=torch.float32, device="cuda")
     tr = moe.Trace(d.E)
     hits = misses = 0
+    rep1 = rep2 = 0
+    last_use = [np.zeros(d.E, dtype=np.int64) for _ in Ls]  # host copy, for the repeat counters
+    ctx.stats_reset()
     if prefetch:
         moe.prefetch_configure(ctx, prefetch)
         nexts = [moe.next_layer(Ls[l + 1].weights(resident=False), caches[l + 1], Ls[l + 1].bias_t)
@@ -132,6 +139,11 @@ def _streaming(O, d, layers, tokens, S, check_y_every=1, T=1, policy=0, period=0
             assert got["misses"] == nmiss and got["h2d_bytes"] == nmiss * L.nb
             hits += int(want["hit"].sum())
             misses += nmiss
+            for e in want["expert"]:
+                lu = last_use[l][e]
+                rep1 += int(lu != 0 and lu == step)
+                rep2 += int(lu != 0 and lu + 1 >= step)
+            last_use[l][want["expert"]] = step + 1
             if prefetch and l > 0:
                 later_misses += nmiss
             if step % check_y_every == 0:
@@ -145,6 +157,14 @@ def _streaming(O, d, layers, tokens, S, check_y_every=1, T=1, policy=0, period=0
                         assert np.array_equal(sl[s_, :L.nb], L.blobs[e_]), (step, l, s_, e_)
     for fd in fds:
         os.close(fd)
+    # the device counters agree with the oracle's plans
+    st = ctx.stats()
+    assert st["calls"] == layers * tokens
+    assert (st["hits"], st["misses"]) == (hits, misses)
+    assert st["miss_bytes"] == misses * Ls[0].nb
+    assert (st["repeat_prev"], st["repeat_prev2"], st["planned"]) == (rep1, rep2, hits + misses)
+    if counters is not None:
+        counters.update(st)
     if prefetch and stats is not None:
         stats["issued"], stats["used"] = moe.prefetch_stats(ctx)
         stats["later_misses"], stats["nb"] = later_misses, Ls[0].nb
@@ -305,3 +325,63 @@ def test_prefill_resident_tensor_core(O, d, T):
     for t in sample:
         _check_token(O, L, xb[t], ids_h[t], gw_h[t], y_h[t])
     assert np.array_equal(yb.cpu().numpy().view(np.uint16), synth.to_bf16_bits(y_h))
+
+
+@pytest.mark.parametrize("d,layers,tokens,S,every", [(TINY, 3, 40, 6, 1), (FULL, 3, 24, 16, 4)], ids=["tiny", "full"])
+def test_streaming_decode_direct_fill(O, d, layers, tokens, S, every):
+    """Misses read by the layer kernel straight from the pinned host store and
+    written into their slots as it computes: traces, slot contents (the write
+    back) and outputs against the oracle, and the device counters."""
+    cnt = {}
+    h, m = _streaming(O, d, layers=layers, tokens=tokens, S=S, check_y_every=every, direct=True, counters=cnt)
+    assert m > 0 and h > 0
+    assert h + m == layers * tokens * d.K
+
+
+@pytest.mark.parametrize("policy,period", [(moe.MOE_POLICY_LRU, 0), (moe.MOE_POLICY_LFU_DECAY, 5),
+                                           (moe.MOE_POLICY_LFU_IN_CACHE, 0)], ids=["lru", "decay5", "in-cache"])
+def test_streaming_direct_fill_policies(O, policy, period):
+    _streaming(O, TINY, layers=2, tokens=30, S=6, policy=policy, period=period, direct=True)
+
+
+def test_direct_fill_with_batches_copies(O):
+    """A direct-source cache given a 4-token batch: the plan runs in waves and
+    the copy engine fills the slots, as for the pinned store."""
+    _streaming(O, TINY, layers=1, tokens=3, S=6, T=4, direct=True)
+
+
+def test_layer_kernel_nan_logits(O):
+    """A NaN router logit: no order exists; the one-launch layer reports
+    MOE_ERR_NAN and uses experts 0..K-1 with equal weights, like the router."""
+    d = TINY
+    L = Layer(d, layer=0, seed=3, zipf_s=None)
+    ctx = moe.Ctx.from_dims(d, max_tokens=1)
+    bias = np.zeros(d.E, dtype=np.float32)
+    bias[5] = np.nan
+    y = torch.empty((1, d.D), dtype=torch.float32, device="cuda")
+    ids = torch.empty((1, d.K), dtype=torch.int32, device="cuda")
+    gw = torch.empty((1, d.K), dtype=torch.float32, device="cuda")
+    moe.layer_forward(ctx, L.weights(), None, bf16_tensor(synth.hidden(3, 0, 0, d.D)[None]), 1, 0,
+                      torch.from_numpy(bias).cuda(), y, ids=ids, gate_w=gw)
+    assert ctx.sync_status() == moe.MOE_ERR_NAN
+    assert np.array_equal(ids.cpu().numpy()[0], np.arange(d.K))
+    assert np.allclose(gw.cpu().numpy()[0], 1.0 / d.K)
+    ctx.close()
+
+
+def test_direct_fill_rejects_unpinned_store():
+    d = TINY
+    L = Layer(d, layer=0, seed=1, zipf_s=1.1, resident=False, pinned=False)
+    ctx = moe.Ctx.from_dims(d, max_tokens=1, S=6)
+    state = torch.empty(ctx.state_words(), dtype=torch.int32, device="cuda")
+    slots = torch.empty((6, L.stride), dtype=torch.uint8, device="cuda")
+    pageable = torch.from_numpy(L.host)  # not pinned: the kernel cannot read it
+    c = moe.slot_cache(slots, L.stride, state, pageable, L.stride, direct=True)
+    moe.cache_reset(ctx, c)
+    y = torch.empty((1, d.D), dtype=torch.float32, device="cuda")
+    with pytest.raises(moe.MoeError) as ei:
+        moe.layer_forward(ctx, L.weights(resident=False), c, bf16_tensor(synth.hidden(1, 0, 0, d.D)[None]), 1, 0,
+                          L.bias_t, y)
+    assert ei.value.code == moe.MOE_ERR_ARG
+    ctx.sync()
+    ctx.close()
