@@ -108,7 +108,7 @@ struct moe_ctx {
     bool layer_pdl = true;
     int layer_hvals = 0;
     float* layer_logits = nullptr;
-    float* layer_partials = nullptr;  // [4 * G][32]: gate/up then down
+    float* layer_partials = nullptr;  // [6 * G][32]: gate/up (two pools) then down
     unsigned* layer_bar = nullptr;    // [4]
     uint64_t* stats = nullptr;        // [MOE_STATS] device counters
     std::unordered_map<const void*, const uint8_t*> direct_store;  // host store -> device-accessible address
@@ -571,7 +571,7 @@ int moe_ctx_create(const moe_dims* dims, int device, moe_ctx** out) {
         if (const char* v = std::getenv("MOE_LAYER_KERNEL")) c->layer_on = !(v[0] == '0');
     }
     ok = ok && dalloc(&c->layer_logits, size_t(d.n_experts)) == cudaSuccess;
-    ok = ok && dalloc(&c->layer_partials, size_t(4) * c->layer_G * 32) == cudaSuccess;
+    ok = ok && dalloc(&c->layer_partials, size_t(6) * c->layer_G * 32) == cudaSuccess;
     ok = ok && dalloc(&c->layer_bar, 4) == cudaSuccess;
     ok = ok && dalloc(&c->stats, MOE_STATS) == cudaSuccess;
     ok = ok && cudaMemset(c->layer_bar, 0, 4 * sizeof(unsigned)) == cudaSuccess;
@@ -796,7 +796,7 @@ static int run_layer_kernel(moe_ctx* c, const moe_layer_weights* W, moe_slot_cac
     a.logits = c->layer_logits;
     a.h = c->h;
     a.partials_gu = c->layer_partials;
-    a.partials_dn = c->layer_partials + size_t(2) * c->layer_G * 32;
+    a.partials_dn = c->layer_partials + size_t(4) * c->layer_G * 32;
     a.counters_gu = c->counters_gu;
     a.counters_dn = c->counters_dn;
     a.bar = c->layer_bar;
@@ -812,6 +812,8 @@ static int run_layer_kernel(moe_ctx* c, const moe_layer_weights* W, moe_slot_cac
     prof_mark(c, MOE_PROF_LAYER, false, s);
     c->launches += 1;
     if (e != cudaSuccess) return MOE_ERR_CUDA;
+    // the mailbox wait watches this event to tell a failed kernel from a slow one
+    if (cudaEventRecord(c->ev_plan, s) != cudaSuccess) return MOE_ERR_CUDA;
     if (cache && trace) {
         const int r = wait_mailbox(c, a.seq, 10000);
         if (r != MOE_OK) return r;

@@ -21,18 +21,19 @@
 //   * K runs in groups of 64 (one quantisation group).  Per group eight math
 //     warps dequantise the 128 x 64 weight tile from the ring (w = s*q + b
 //     rounded to fp16, two weights per half2 instruction) and write it, with
-//     the N x 64 activation tile (loaded into registers one group ahead), in
+//     the N x 64 activation tile (loaded into registers four groups ahead: x
+//     as bf16, h as the fp16 the gate/up epilogue stored), in
 //     the no-swizzle K-major core-matrix layout (8 rows x 16 bytes per core
 //     matrix; K-direction core stride 128 B, 8-row stride 1024 B).  An MMA
 //     warp issues 4 MMAs of K = 16 per group and commits them to an mbarrier;
 //     two fp16 buffer sets let the math warps run a group ahead of the tensor
 //     core, and the raw-weight ring holds 12 groups per CTA.
 //   * gate/up epilogue: TMEM lanes 32w..32w+31 hold one 32-row blob tile (16
-//     gate rows then the 16 matching up rows): h = gelu(g) * u with one shuffle.
+//     gate rows then the 16 matching up rows): h = gelu(g) * u with one
+//     shuffle, stored as fp16 (the down GEMM's operand type; the rounding is
+//     the one the down GEMM applied to fp32 h before).
 //   * down epilogue: y[token][row] += w * D, fp32 atomics (entries of different
 //     experts add into the same output rows).
-#include <type_traits>
-
 #include "common.cuh"
 #include "ffn.cuh"
 #include "launch.cuh"
@@ -114,6 +115,7 @@ constexpr int kProducerWarp = kMathWarps;   // bulk copies of raw weights
 constexpr int kMmaWarp = kMathWarps + 1;    // issues the tensor-core MMAs
 constexpr int kGemmWarps = kMathWarps + 2;
 constexpr int kBTasks = kGemmMaxRows * 8 / kMathThreads;  // (row, 8-input block) tasks of the B tile per thread
+constexpr int kAhead = 4;  // groups whose activations are in flight (registers) ahead of their use
 
 // Inside every 8-input block the fp16 tiles hold the inputs in the order
 // 0,4,1,5,2,6,3,7 (A and B alike, so the contraction is unchanged): that is
@@ -295,17 +297,19 @@ __global__ void __launch_bounds__(kGemmWarps * 32, 2) grouped_gemm_kernel(GemmAr
     // core matrix (no bank conflicts) and its loads still fill whole sectors.
     // Rows M..N-1 are zero padding.  Raw loads are kept in registers, two
     // groups ahead (two register sets, alternating), and converted when used.
+    // MODE 0 reads x (bf16), MODE 1 the h rows the gate/up GEMM stored as fp16
+    // (at the same element offsets); both are 8 x 16-bit values per task
     const int ntasks = 8 * N;
-    using Raw = typename std::conditional<MODE == 0, uint4, float4[2]>::type;
-    const void* bsrc[kBTasks];  // row base of each task (nullptr: padding row)
+    using Raw = uint4;
+    const uint16_t* bsrc[kBTasks];  // row base of each task (nullptr: padding row)
 #pragma unroll
     for (int i = 0; i < kBTasks; ++i) {
         const int idx = tid + kMathThreads * i;
         const int j = 8 * (idx >> 6) + (idx & 7);
         bsrc[i] = nullptr;
         if (idx < ntasks && j < M)
-            bsrc[i] = MODE == 0 ? static_cast<const void*>(A.x + size_t(s_rows[j].x_row) * D)
-                                : static_cast<const void*>(A.h + s_rows[j].h_off);
+            bsrc[i] = MODE == 0 ? A.x + size_t(s_rows[j].x_row) * D
+                                : reinterpret_cast<const uint16_t*>(A.h) + s_rows[j].h_off;
     }
     auto load_b = [&](int g, Raw (&braw)[kBTasks]) {
 #pragma unroll
@@ -313,21 +317,7 @@ __global__ void __launch_bounds__(kGemmWarps * 32, 2) grouped_gemm_kernel(GemmAr
             const int idx = tid + kMathThreads * i;
             if (idx >= ntasks) break;
             const int k0 = g * kGroup + 8 * ((idx >> 3) & 7);
-            if (MODE == 0) {
-                uint4& q = reinterpret_cast<uint4&>(braw[i]);
-                q = bsrc[i] ? *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(bsrc[i]) + k0)
-                            : make_uint4(0, 0, 0, 0);
-            } else {
-                float4* f = reinterpret_cast<float4*>(&braw[i]);
-                if (bsrc[i]) {
-                    const float* hp = static_cast<const float*>(bsrc[i]) + k0;
-                    f[0] = *reinterpret_cast<const float4*>(hp);
-                    f[1] = *reinterpret_cast<const float4*>(hp + 4);
-                } else {
-                    f[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-                    f[1] = f[0];
-                }
-            }
+            braw[i] = bsrc[i] ? *reinterpret_cast<const uint4*>(bsrc[i] + k0) : make_uint4(0, 0, 0, 0);
         }
     };
     // this thread's weights: row r of the 128 (blob tile 4*tile + r/32, row r%32), inputs 32*hk .. +31 of each group
@@ -347,27 +337,30 @@ __global__ void __launch_bounds__(kGemmWarps * 32, 2) grouped_gemm_kernel(GemmAr
         for (int i = 0; i < kBTasks; ++i) {
             const int idx = tid + kMathThreads * i;
             if (idx >= ntasks) break;
-            float v[8];
+            const uint4 q = braw[i];
+            uint4 out;
             if (MODE == 0) {
-                const uint4 q = reinterpret_cast<const uint4&>(braw[i]);
+                float v[8];
                 const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
                 for (int t = 0; t < 4; ++t) {
                     v[2 * t] = __uint_as_float(w4[t] << 16);
                     v[2 * t + 1] = __uint_as_float(w4[t] & 0xFFFF0000u);
                 }
-            } else {
-                const float4* f = reinterpret_cast<const float4*>(&braw[i]);
-                v[0] = f[0].x; v[1] = f[0].y; v[2] = f[0].z; v[3] = f[0].w;
-                v[4] = f[1].x; v[5] = f[1].y; v[6] = f[1].z; v[7] = f[1].w;
-            }
 #pragma unroll
-            for (int t = 0; t < 8; ++t)
-                if (!(fabsf(v[t]) <= 65504.f)) { s_bad = 1; v[t] = 0.f; }  // beyond fp16 (or NaN)
+                for (int t = 0; t < 8; ++t)
+                    if (!(fabsf(v[t]) <= 65504.f)) { s_bad = 1; v[t] = 0.f; }  // beyond fp16 (or NaN)
+                out = pack_block_perm(v);
+            } else {
+                // already fp16 (range checked when written): reorder (0,1)(2,3)(4,5)(6,7)
+                // into the block order (0,4)(1,5)(2,6)(3,7)
+                out = make_uint4(__byte_perm(q.x, q.z, 0x5410), __byte_perm(q.x, q.z, 0x7632),
+                                 __byte_perm(q.y, q.w, 0x5410), __byte_perm(q.y, q.w, 0x7632));
+            }
             const int j = 8 * (idx >> 6) + (idx & 7);
-            *reinterpret_cast<uint4*>(bt + core_off(j, 8 * ((idx >> 3) & 7))) = pack_block_perm(v);
+            *reinterpret_cast<uint4*>(bt + core_off(j, 8 * ((idx >> 3) & 7))) = out;
         }
-        if (g + 2 < ngroups) load_b(g + 2, braw);
+        if (g + kAhead < ngroups) load_b(g + kAhead, braw);
         // A: dequantise this thread's 32 weights of the group from the raw stage
         {
             const uint8_t* raw = ring + size_t(st) * ST_BYTES + bt_row * BT_BYTES;
@@ -387,20 +380,22 @@ __global__ void __launch_bounds__(kGemmWarps * 32, 2) grouped_gemm_kernel(GemmAr
         }
         return true;
     };
-    Raw braw0[kBTasks], braw1[kBTasks];
+    Raw braw0[kBTasks], braw1[kBTasks], braw2[kBTasks], braw3[kBTasks];
     load_b(0, braw0);
     if (ngroups > 1) load_b(1, braw1);
+    if (ngroups > 2) load_b(2, braw2);
+    if (ngroups > 3) load_b(3, braw3);
     bool ok = true;
-    for (int g = 0; g < ngroups && ok; g += 2) {
+    for (int g = 0; g < ngroups && ok; g += kAhead) {
         ok = step(g, braw0);
         if (ok && g + 1 < ngroups) ok = step(g + 1, braw1);
+        if (ok && g + 2 < ngroups) ok = step(g + 2, braw2);
+        if (ok && g + 3 < ngroups) ok = step(g + 3, braw3);
     }
     // every MMA the MMA warp issued has completed
     if (ok) ok = ring_wait_gemm(&done, 0, A.status, &s_abort);
     ok = __all_sync(0xffffffffu, ok);  // the tensor-memory loads below are warp-collective
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    if (s_bad && tid == 0) set_status(A.status, MOE_ERR_RANGE);
-
     if (ok) {
         // warp w reads TMEM lanes 32*(w%4) ..; warps 0-3 take column blocks 0, 32, warps 4-7 blocks 16, 48
         const int q4 = warp & 3;
@@ -422,8 +417,14 @@ __global__ void __launch_bounds__(kGemmWarps * 32, 2) grouped_gemm_kernel(GemmAr
                 if (MODE == 0) {
                     // lanes of blob tile 4*tile + q4: 0..15 gate, 16..31 up of outputs 16*bt + lane
                     const float up = __shfl_down_sync(0xffffffffu, d, 16);
-                    if (lane < 16 && j < M)
-                        A.h[s_rows[j].h_off + 16 * (4 * tile + q4) + lane] = gelu_tanh(d) * up;
+                    if (lane < 16 && j < M) {
+                        // h as fp16, the type the down GEMM's B tile needs (same rounding)
+                        const float hv = gelu_tanh(d) * up;
+                        const bool in_range = fabsf(hv) <= 65504.f;
+                        if (!in_range) s_bad = 1;
+                        reinterpret_cast<__half*>(A.h)[s_rows[j].h_off + 16 * (4 * tile + q4) + lane] =
+                            __float2half_rn(in_range ? hv : 0.f);
+                    }
                 } else if (j < M) {
                     atomicAdd(&A.y[size_t(s_rows[j].y_row) * D + 128 * tile + 32 * q4 + lane], s_rows[j].w * d);
                 }
@@ -432,6 +433,7 @@ __global__ void __launch_bounds__(kGemmWarps * 32, 2) grouped_gemm_kernel(GemmAr
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     named_sync(1, kMathThreads);
+    if (s_bad && tid == 0) set_status(A.status, MOE_ERR_RANGE);  // an input or h beyond fp16
     if (warp == 0)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(ncols) : "memory");
 }

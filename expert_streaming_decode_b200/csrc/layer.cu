@@ -50,7 +50,7 @@ namespace {
 constexpr int kLNW = 12;                      // consumer warps
 constexpr int kLNC = kLNW * 32;               // consumer threads
 constexpr int kLThreads = kLNC + 32;          // + producer warp
-constexpr int kLGuStages = 8;
+constexpr int kLGuStages = 12;
 constexpr int kLDnStages = 8;
 constexpr int kLGuStage = 18 * kGuSlice;      // 4608 B
 constexpr int kLDnStage = 18 * kDownSliceMax; // 12672 B
@@ -149,6 +149,9 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
 __device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
     asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// waits until every cp.async this thread issued has landed
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 __device__ __forceinline__ bool lwait(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag) {
     if (*abort_flag) return false;
@@ -290,7 +293,15 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_decode_kernel(LayerArgs A)
     const int ns_sh = nsh ? FS / ks_sh : 0, ns_rt = F / ks_rt;
     const int upt = ns_sh + K * ns_rt, tiles_dn = D / kChunkRows;
     const int Udn = tiles_dn * upt;
-    const int g0 = range_start(c, Ugu, G), g1 = range_start(c + 1, Ugu, G);
+    // gate/up: the shared expert's units and the routed units are two pools,
+    // each split evenly over all CTAs, so every CTA streams shared weights
+    // during the router phase and routed weights after the plan
+    // (whole 16-output tiles per CTA: no tile is split between CTAs, so the
+    // gate/up results need no cross-CTA reduction)
+    const int Urt = Ugu - ush;
+    const int TS = nsh ? FS / 16 : 0, TR = K * (F / 16);
+    const int sh0 = range_start(c, TS, G) * NSg, sh1 = range_start(c + 1, TS, G) * NSg;
+    const int r0 = ush + range_start(c, TR, G) * NSg, r1 = ush + range_start(c + 1, TR, G) * NSg;
     const int d0 = range_start(c, Udn, G), d1 = range_start(c + 1, Udn, G);
     const int n_rows = c < E ? (E - 1 - c) / G + 1 : 0;  // experts c, c+G, ...
     auto gu_entry = [&](int u) { return u < ush ? 0 : nsh + (u - ush) / urt; };
@@ -352,6 +363,7 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_decode_kernel(LayerArgs A)
             uint8_t* dst = ring + size_t(st) * stage_bytes;
             if (host) {
                 for (uint32_t o = uint32_t(lane) * 16u; o < bytes; o += 32u * 16u) cp_async16(dst + o, src + o);
+                cp_async_commit();
                 cp_async_arrive(&full[st]);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&full[st]);
@@ -363,20 +375,44 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_decode_kernel(LayerArgs A)
             ++issued;
             return true;
         };
+        // a chunk source must lie inside the blob its entry names: the host
+        // store (host entries) or a slot, a resident expert or the shared blob
+        const size_t blob_rt = blob_bytes(D, F), blob_sh = nsh ? blob_bytes(D, FS) : 0;
+        auto src_ok = [&](const LEntry& en, const uint8_t* p, uint32_t bytes) {
+            if ((reinterpret_cast<uintptr_t>(p) & 15u) != 0 || (bytes & 15u) != 0) return false;
+            auto inside = [&](const uint8_t* base, size_t n) { return base && p >= base && p + bytes <= base + n; };
+            if (en.host) return inside(A.store, size_t(E) * A.store_stride);
+            return inside(A.shared_blob, blob_sh) ||
+                   (streaming ? inside(A.slots, size_t(S) * A.slot_stride)
+                              : inside(A.experts, size_t(E) * A.expert_stride));
+        };
+        auto issue_checked = [&](uint8_t* ring, int stage_bytes, uint64_t* full, uint64_t* empty, int nst,
+                                 int& issued, const LEntry& en, const uint8_t* src, uint32_t bytes) {
+            if (!src_ok(en, src, bytes) || (en.wb && en.host == 0)) {
+                // never copy from outside: report, stop, and complete nothing more
+                if (lane == 0) {
+                    set_status(A.status, MOE_ERR_RANGE);
+                    s_abort = 1;
+                }
+                __syncwarp();
+                return false;
+            }
+            return issue(ring, stage_bytes, full, empty, nst, issued, src, bytes, en.host != 0);
+        };
         auto issue_gu = [&](int u) {
             const int e = gu_entry(u);
             const LEntry& en = s_ent[e];
-            return issue(gu_ring, kLGuStage, full_gu, empty_gu, kLGuStages, issued_gu,
-                         en.src + size_t(u - gu_base(e)) * kLGuStage, kLGuStage, en.host != 0);
+            return issue_checked(gu_ring, kLGuStage, full_gu, empty_gu, kLGuStages, issued_gu, en,
+                                 en.src + size_t(u - gu_base(e)) * kLGuStage, kLGuStage);
         };
         auto issue_dn = [&](int u) {
             int e, tile, slice;
             dn_unit(u, e, tile, slice);
             const LEntry& en = s_ent[e];
             const int ks = down_ks(en.F);
-            return issue(dn_ring, kLDnStage, full_dn, empty_dn, kLDnStages, issued_dn,
-                         en.src + gu_section_bytes(D, en.F) + size_t(tile * (en.F / ks) + slice) * (18u * ks),
-                         uint32_t(18u * ks), en.host != 0);
+            return issue_checked(dn_ring, kLDnStage, full_dn, empty_dn, kLDnStages, issued_dn, en,
+                                 en.src + gu_section_bytes(D, en.F) + size_t(tile * (en.F / ks) + slice) * (18u * ks),
+                                 uint32_t(18u * ks));
         };
         // router rows of this CTA's experts and its shared-expert chunks:
         // immutable weights, fetched before the dependency wait
@@ -386,8 +422,7 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_decode_kernel(LayerArgs A)
             for (int r = 0; r < n_rows; ++r)
                 bulk_g2s(rrow + size_t(r) * D, A.wq + size_t(c + r * G) * D, uint32_t(D), rt_bar, keep);
         }
-        int u = g0;
-        for (; ok && u < g1 && u < ush; ++u) ok = issue_gu(u);
+        for (int u = sh0; ok && u < sh1; ++u) ok = issue_gu(u);
         // the plan (entries) is ready
         if (ok) {
             bool w = true;
@@ -400,9 +435,12 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_decode_kernel(LayerArgs A)
         // the rest of the down chunks as the ring frees up
         int v = d0;
         for (; ok && v < d1 && v - d0 < kLDnStages; ++v) ok = issue_dn(v);
-        for (; ok && u < g1; ++u) ok = issue_gu(u);
+        for (int u = r0; ok && u < r1; ++u) ok = issue_gu(u);
         for (; ok && v < d1; ++v) ok = issue_dn(v);
-        // every issued copy has landed before the CTA may exit
+        // every issued copy has landed before the CTA may exit: each lane's own
+        // asynchronous copies, then (lane 0) the last uses of every stage
+        cp_async_wait_all();
+        __syncwarp();
         if (lane == 0) {
             for (int i = issued_gu > kLGuStages ? issued_gu - kLGuStages : 0; i < issued_gu; ++i)
                 mbar_wait(&full_gu[i % kLGuStages], uint32_t(i / kLGuStages) & 1u, A.status);
@@ -484,10 +522,13 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_decode_kernel(LayerArgs A)
 
     // ---------------------------------------------- gate/up consumer loop
     float acc = 0.f;
-    int seg_start = g0;
-    auto gu_units = [&](int ua, int ub) {
+    int seg_start = 0;
+    // units [ua, ub) of pool `pool` (0 shared, 1 routed: base pb, size PU);
+    // i0 = ring position of unit ua
+    auto gu_units = [&](int ua, int ub, int pool, int pb, int PU, int i0) {
+        seg_start = ua;
         for (int u = ua; u < ub; ++u) {
-            const int i = u - g0, st = i % kLGuStages;
+            const int i = i0 + (u - ua), st = i % kLGuStages;
             const int e = gu_entry(u);
             const int ul = u - gu_base(e);
             const int tile = ul / NSg, slice = ul - tile * NSg;
@@ -506,7 +547,7 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_decode_kernel(LayerArgs A)
             }
             __syncwarp();
             if (mine && lane == 0) mbar_arrive(&empty_gu[st]);
-            const bool seg_end = (u + 1 == g1) || (u + 1 == key_u0 + NSg);
+            const bool seg_end = (u + 1 == ub) || (u + 1 == key_u0 + NSg);
             if (!seg_end) continue;
             named_sync(1, kLNC);
             red[warp * 32 + lane] = acc;
@@ -519,8 +560,8 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_decode_kernel(LayerArgs A)
                 bool lastc = whole;
                 const int cidx = key_u0 / NSg;
                 if (!whole) {
-                    const int sl = (seg_start == g0) ? 0 : 1;
-                    A.partials_gu[size_t(2 * c + sl) * 32 + lane] = tot;
+                    const int sl = (seg_start == ua) ? 0 : 1;
+                    A.partials_gu[size_t(4 * c + 2 * pool + sl) * 32 + lane] = tot;
                     __threadfence();
                     __syncwarp();
                     int old = 0;
@@ -530,11 +571,12 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_decode_kernel(LayerArgs A)
                     if (lastc) {
                         __threadfence();
                         tot = 0.f;
-                        const int c0 = cta_of(key_u0, Ugu, G), c1 = cta_of(key_u0 + NSg - 1, Ugu, G);
+                        const int kl = key_u0 - pb;  // the tile's first unit inside its pool
+                        const int c0 = cta_of(kl, PU, G), c1 = cta_of(kl + NSg - 1, PU, G);
                         for (int cc = c0; cc <= c1; ++cc) {
-                            const int rs = range_start(cc, Ugu, G);
-                            if (rs >= range_start(cc + 1, Ugu, G)) continue;
-                            tot += __ldcg(A.partials_gu + size_t(2 * cc + (rs >= key_u0 ? 0 : 1)) * 32 + lane);
+                            const int rs = range_start(cc, PU, G);
+                            if (rs >= range_start(cc + 1, PU, G)) continue;
+                            tot += __ldcg(A.partials_gu + size_t(4 * cc + 2 * pool + (rs >= kl ? 0 : 1)) * 32 + lane);
                         }
                         if (lane == 0) A.counters_gu[cidx] = 0;
                     }
@@ -548,8 +590,7 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_decode_kernel(LayerArgs A)
             seg_start = u + 1;
         }
     };
-    const int g_sh_end = g1 < ush ? g1 : (g0 > ush ? g0 : ush);
-    gu_units(g0, g_sh_end);  // shared-expert chunks (known before the plan)
+    gu_units(sh0, sh1, 0, 0, ush, 0);  // shared-expert chunks (known before the plan)
 
     // ------------------------------------------------- phase 2: top-K + plan
     bool ok_a = true;
@@ -752,7 +793,7 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_decode_kernel(LayerArgs A)
     named_sync(1, kLNC);
 
     // ------------------------------------------- the routed gate/up chunks
-    gu_units(g_sh_end, g1);
+    gu_units(r0, r1, 1, ush, Urt, sh1 - sh0);
 
     // ------------------------------------------------ phase 3: down + combine
     named_sync(1, kLNC);

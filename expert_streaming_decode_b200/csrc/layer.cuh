@@ -38,7 +38,7 @@ struct LayerArgs {
     // scratch
     float* logits;               // [E]
     float* h;                    // [FS + K*F]
-    float* partials_gu;          // [2*G][32]
+    float* partials_gu;          // [4*G][32]: two per CTA and pool (shared, routed)
     int* counters_gu;            // [FS/16 + K*F/16], zero between launches
     float* partials_dn;          // [2*G][32]
     int* counters_dn;            // [D/32], zero between launches
