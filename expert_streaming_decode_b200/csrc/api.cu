@@ -77,6 +77,7 @@ struct moe_ctx {
     float* gate_w = nullptr;
     int32_t* pair_slot = nullptr;
     int32_t* pair_wave = nullptr;
+    uint16_t* x16 = nullptr;  // [max_tokens][D] fp16 copy of a multi-token call's hidden states (GEMM operand)
     GemvShapes shapes{};
     uint64_t launches = 0;
     size_t blob_routed = 0;
@@ -184,6 +185,7 @@ void free_ctx(moe_ctx* c) {
     cudaFree(c->gate_w);
     cudaFree(c->pair_slot);
     cudaFree(c->pair_wave);
+    cudaFree(c->x16);
     if (c->mbox_host) cudaFreeHost(c->mbox_host);
     if (c->ev_plan) cudaEventDestroy(c->ev_plan);
     if (c->ev_fill) cudaEventDestroy(c->ev_fill);
@@ -290,7 +292,8 @@ int run_ffn(moe_ctx* c, const WorkListArgs& wa, const uint16_t* x, int T, const 
 // Batches and prefill chunks: builds a GEMM-mode work list (entries of up to
 // kGemmMaxRows rows) and runs the tensor-core grouped GEMM; adds into y, which
 // the caller zeroed before the first call of the layer.
-int run_gemm(moe_ctx* c, WorkListArgs wa, const uint16_t* x, int T, float* y, cudaStream_t s) {
+// x16: the call's hidden states as fp16 (to_f16 below)
+int run_gemm(moe_ctx* c, WorkListArgs wa, const uint16_t* x16, int T, float* y, cudaStream_t s) {
     wa.gemm = 1;
     prof_mark(c, MOE_PROF_WORKLIST, true, s);
     cudaError_t e = launch_build_worklist(wa, c->pdl, s);
@@ -304,7 +307,7 @@ int run_gemm(moe_ctx* c, WorkListArgs wa, const uint16_t* x, int T, float* y, cu
     L.wl = c->wl;
     L.entries = c->entries;
     L.rows = c->rows;
-    L.x = x;
+    L.x = x16;
     L.h = c->h;
     L.y = y;
     L.D = c->d.d_model;
@@ -317,6 +320,12 @@ int run_gemm(moe_ctx* c, WorkListArgs wa, const uint16_t* x, int T, float* y, cu
     e = launch_gemm(L, s, c->prof ? ffn_hook : nullptr, &ha);
     c->launches += 2;
     return cuda_status(e);
+}
+
+// The hidden states of a multi-token call as fp16 (the grouped GEMM's B operand).
+int to_f16(moe_ctx* c, const uint16_t* x, int T, cudaStream_t s) {
+    c->launches += 1;
+    return cuda_status(launch_bf16_to_f16(x, c->x16, size_t(T) * c->d.d_model, c->status, c->pdl, s));
 }
 
 DecodeWLTarget decode_target(moe_ctx* c, WorkList* wl, FfnEntry* en, FfnRow* rows, const uint8_t* slot_base,
@@ -564,6 +573,7 @@ int moe_ctx_create(const moe_dims* dims, int device, moe_ctx** out) {
     ok = ok && dalloc(&c->gate_w, pairs) == cudaSuccess;
     ok = ok && dalloc(&c->pair_slot, pairs) == cudaSuccess;
     ok = ok && dalloc(&c->pair_wave, pairs) == cudaSuccess;
+    ok = ok && dalloc(&c->x16, size_t(T) * d.d_model) == cudaSuccess;
     ok = ok && layer_grid(device, &c->layer_G) == cudaSuccess;
     if (ok) {
         c->layer_ok = layer_supported(d.d_model, d.n_experts, d.top_k, d.d_ff, d.d_ff_shared, d.n_slots, c->layer_G);
@@ -878,7 +888,8 @@ static int layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache*
                                         W->shared_blob);
         if (!gemm) return run_ffn(c, wa, x, T, nullptr, y, y_bf16, s);
         if (cudaMemsetAsync(y, 0, sizeof(float) * size_t(T) * c->d.d_model, s) != cudaSuccess) return MOE_ERR_CUDA;
-        r = run_gemm(c, wa, x, T, y, s);
+        r = to_f16(c, x, T, s);
+        if (r == MOE_OK) r = run_gemm(c, wa, c->x16, T, y, s);
         if (r != MOE_OK) return r;
         if (y_bf16) {
             c->launches += 1;
@@ -920,10 +931,12 @@ static int layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache*
     } else if (gemm) {
         // prefill chunk: every contribution is added into y
         if (cudaMemsetAsync(y, 0, sizeof(float) * size_t(T) * c->d.d_model, s) != cudaSuccess) return MOE_ERR_CUDA;
+        r = to_f16(c, x, T, s);
+        if (r != MOE_OK) return r;
         if (W->shared_blob) {
             WorkListArgs wa = worklist_args(c, T, 0, c->pair_slot, gw, cache->slots, cache->slot_stride, c->d.n_slots,
                                             c->d.d_ff, W->shared_blob);
-            r = run_gemm(c, wa, x, T, y, s);
+            r = run_gemm(c, wa, c->x16, T, y, s);
             if (r != MOE_OK) return r;
         }
         have_y = true;
@@ -962,7 +975,7 @@ static int layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache*
                                             c->d.n_slots, c->d.d_ff, nullptr);
             wa.pair_wave = c->pair_wave;
             wa.wave = w;
-            r = run_gemm(c, wa, x, T, y, s);
+            r = run_gemm(c, wa, c->x16, T, y, s);
         } else {
             WorkListArgs wa = worklist_args(c, T, K, c->pair_slot, gw, cache->slots, cache->slot_stride,
                                             c->d.n_slots, c->d.d_ff, nullptr);

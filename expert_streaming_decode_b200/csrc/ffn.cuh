@@ -69,7 +69,7 @@ struct GemmLaunch {
     const WorkList* wl;
     const FfnEntry* entries;
     const FfnRow* rows;
-    const uint16_t* x;
+    const uint16_t* x;  // fp16 bits [T][D] (launch_bf16_to_f16 of the call's hidden states)
     float* h;
     float* y;          // accumulated with atomics: zero it before the first launch
     int D;
@@ -81,6 +81,8 @@ struct GemmLaunch {
 cudaError_t gemm_prepare();
 cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, void (*hook)(void*, int), void* hook_arg);
 cudaError_t launch_f32_to_bf16(const float* y, uint16_t* out, size_t n, bool pdl, cudaStream_t s);
+// bf16 [n] -> fp16 [n] (n % 8 == 0, 16-byte aligned); out-of-range values -> 0, MOE_ERR_RANGE
+cudaError_t launch_bf16_to_f16(const uint16_t* x, uint16_t* out, size_t n, int* status, bool pdl, cudaStream_t s);
 
 cudaError_t ffn_prepare(int D, int F, int FS, int K, int T, int sms, GemvShapes* shapes);
 // Launch shapes of the one-token kernels (shapes->gu[0], dn[0]) for inputs up

@@ -45,7 +45,7 @@ struct GemmArgs {
     const WorkList* wl;
     const FfnEntry* entries;
     const FfnRow* rows;
-    const uint16_t* x;   // bf16 [T][D]
+    const uint16_t* x;   // fp16 bits [T][D] (the call's hidden states, converted once per call)
     float* h;            // activations
     float* y;            // [T][D], accumulated
     int D;
@@ -120,10 +120,6 @@ constexpr int kAhead = 4;  // groups whose activations are in flight (registers)
 // Inside every 8-input block the fp16 tiles hold the inputs in the order
 // 0,4,1,5,2,6,3,7 (A and B alike, so the contraction is unchanged): that is
 // the order in which two nibbles at a time come out of a 32-bit word below.
-__device__ __forceinline__ uint4 pack_block_perm(const float v[8]) {
-    return make_uint4(pack_half2(v[0], v[4]), pack_half2(v[1], v[5]), pack_half2(v[2], v[6]),
-                      pack_half2(v[3], v[7]));
-}
 
 // 8 weights w = s*q + b of one 32-bit word (nibble i = input i) as fp16, in the
 // block order above.  A nibble placed in the low mantissa bits of the binary16
@@ -297,8 +293,8 @@ __global__ void __launch_bounds__(kGemmWarps * 32, 2) grouped_gemm_kernel(GemmAr
     // core matrix (no bank conflicts) and its loads still fill whole sectors.
     // Rows M..N-1 are zero padding.  Raw loads are kept in registers, two
     // groups ahead (two register sets, alternating), and converted when used.
-    // MODE 0 reads x (bf16), MODE 1 the h rows the gate/up GEMM stored as fp16
-    // (at the same element offsets); both are 8 x 16-bit values per task
+    // MODE 0 reads x (as fp16, converted once per call), MODE 1 the h rows the
+    // gate/up GEMM stored as fp16 (at the same element offsets): 8 fp16 per task
     const int ntasks = 8 * N;
     using Raw = uint4;
     const uint16_t* bsrc[kBTasks];  // row base of each task (nullptr: padding row)
@@ -338,25 +334,10 @@ __global__ void __launch_bounds__(kGemmWarps * 32, 2) grouped_gemm_kernel(GemmAr
             const int idx = tid + kMathThreads * i;
             if (idx >= ntasks) break;
             const uint4 q = braw[i];
-            uint4 out;
-            if (MODE == 0) {
-                float v[8];
-                const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    v[2 * t] = __uint_as_float(w4[t] << 16);
-                    v[2 * t + 1] = __uint_as_float(w4[t] & 0xFFFF0000u);
-                }
-#pragma unroll
-                for (int t = 0; t < 8; ++t)
-                    if (!(fabsf(v[t]) <= 65504.f)) { s_bad = 1; v[t] = 0.f; }  // beyond fp16 (or NaN)
-                out = pack_block_perm(v);
-            } else {
-                // already fp16 (range checked when written): reorder (0,1)(2,3)(4,5)(6,7)
-                // into the block order (0,4)(1,5)(2,6)(3,7)
-                out = make_uint4(__byte_perm(q.x, q.z, 0x5410), __byte_perm(q.x, q.z, 0x7632),
-                                 __byte_perm(q.y, q.w, 0x5410), __byte_perm(q.y, q.w, 0x7632));
-            }
+            // fp16 already (range checked when written): reorder (0,1)(2,3)(4,5)(6,7)
+            // into the block order (0,4)(1,5)(2,6)(3,7)
+            const uint4 out = make_uint4(__byte_perm(q.x, q.z, 0x5410), __byte_perm(q.x, q.z, 0x7632),
+                                         __byte_perm(q.y, q.w, 0x5410), __byte_perm(q.y, q.w, 0x7632));
             const int j = 8 * (idx >> 6) + (idx & 7);
             *reinterpret_cast<uint4*>(bt + core_off(j, 8 * ((idx >> 3) & 7))) = out;
         }
@@ -465,6 +446,36 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, void (*hook)(void*,
                       1, a);
     if (hook) hook(hook_arg, 2);
     return e;
+}
+
+// The call's hidden states bf16 -> fp16, the operand type of the tensor-core
+// tiles, once per layer call (every expert a token is routed to reads it);
+// values beyond the fp16 range become 0 and are reported (MOE_ERR_RANGE).
+__global__ void bf16_to_f16_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ out, size_t n8,
+                                   int* status) {
+    pdl_wait();
+    pdl_trigger();
+    bool bad = false;
+    for (size_t i = blockIdx.x * size_t(blockDim.x) + threadIdx.x; i < n8; i += size_t(gridDim.x) * blockDim.x) {
+        const uint4 q = reinterpret_cast<const uint4*>(x)[i];
+        const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            float a = __uint_as_float(w4[t] << 16), b = __uint_as_float(w4[t] & 0xFFFF0000u);
+            if (!(fabsf(a) <= 65504.f)) { bad = true; a = 0.f; }
+            if (!(fabsf(b) <= 65504.f)) { bad = true; b = 0.f; }
+            o[t] = pack_half2(a, b);
+        }
+        reinterpret_cast<uint4*>(out)[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    if (bad) set_status(status, MOE_ERR_RANGE);
+}
+
+cudaError_t launch_bf16_to_f16(const uint16_t* x, uint16_t* out, size_t n, int* status, bool pdl, cudaStream_t s) {
+    const size_t n8 = n / 8;
+    const int blocks = int(n8 / 256 + 1 < 592 ? n8 / 256 + 1 : 592);
+    return launch_kernel(bf16_to_f16_kernel, dim3(blocks), dim3(256), 0, s, pdl, 1, x, out, n8, status);
 }
 
 // y (fp32) -> bf16, for the prefill path's optional bf16 output
