@@ -60,13 +60,13 @@ def parse_args():
                    help="streamed workloads: write each layer's experts to DIR/layerNN.experts and read misses "
                         "from those files with positional reads (the file-backed store)")
     p.add_argument("--direct", action="store_true", help="--store-file: open the files with O_DIRECT")
-    p.add_argument("--fill", choices=["direct", "copy"], default="direct",
+    p.add_argument("--fill", choices=["direct", "copy"], default="copy",
                    help="streamed workloads with the pinned store: how one-token misses reach their slots -- "
-                        "'direct': the layer kernel reads them from pinned host memory as it computes (default); "
-                        "'copy': the host reads the plan and the copy engine copies them")
+                        "'copy': the host reads the plan and the copy engine copies them (default); "
+                        "'direct': the one-launch layer kernel reads them from pinned host memory as it computes")
     p.add_argument("--prefetch", type=int, default=None, metavar="P",
                    help="decode_stream with --fill copy: stage up to P of the next layer's predicted misses "
-                        "(look-ahead; 0 = off, the default)")
+                        "(look-ahead; 0 = off; default 1 for the one-token streamed decode from the pinned store)")
     p.add_argument("--zipf", type=float, default=None,
                    help="Zipf exponent of the router popularity bias (default 1.1; 0 = uniform router, "
                         "the default for decode_resident)")
@@ -82,7 +82,8 @@ def parse_args():
     if a.zipf is None:
         a.zipf = 0.0 if a.workload == "decode_resident" else 1.1
     if a.prefetch is None:
-        a.prefetch = 0
+        a.prefetch = 1 if (a.workload == "decode_stream" and a.batch == 1 and not a.store_file
+                           and a.fill == "copy") else 0
     if a.prefetch and (a.workload != "decode_stream" or a.batch != 1 or a.store_file or a.fill != "copy"):
         p.error("--prefetch needs the one-token decode_stream workload with the pinned host store and --fill copy")
     if not 0 <= a.prefetch <= 16:

@@ -105,7 +105,8 @@ struct moe_ctx {
     // one-token layer kernel (layer.cu): grid, support for the dims, scratch
     int layer_G = 0;
     bool layer_ok = false;
-    bool layer_on = true;
+    bool layer_on = true;         // MOE_LAYER_KERNEL=0: never (direct sources then copy)
+    bool layer_resident = false;  // MOE_LAYER_KERNEL=1: resident one-token layers too
     bool layer_pdl = true;
     int layer_hvals = 0;
     float* layer_logits = nullptr;
@@ -578,7 +579,10 @@ int moe_ctx_create(const moe_dims* dims, int device, moe_ctx** out) {
     if (ok) {
         c->layer_ok = layer_supported(d.d_model, d.n_experts, d.top_k, d.d_ff, d.d_ff_shared, d.n_slots, c->layer_G);
         c->layer_hvals = layer_hvals(d.d_model, d.top_k, d.d_ff, d.d_ff_shared, c->layer_G);
-        if (const char* v = std::getenv("MOE_LAYER_KERNEL")) c->layer_on = !(v[0] == '0');
+        if (const char* v = std::getenv("MOE_LAYER_KERNEL")) {
+            c->layer_on = v[0] != '0';
+            c->layer_resident = v[0] == '1';
+        }
     }
     ok = ok && dalloc(&c->layer_logits, size_t(d.n_experts)) == cudaSuccess;
     ok = ok && dalloc(&c->layer_partials, size_t(6) * c->layer_G * 32) == cudaSuccess;
@@ -856,7 +860,11 @@ static int layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache*
     // stream, while this layer runs (one token, host stores, buffers configured)
     const bool prefetch = next && T == 1 && c->pf_n > 0 && next->W && next->W->router_q && next->W->router_s &&
                           next->cache && next->cache->source == MOE_SOURCE_HOST && next->cache->store;
-    if (T == 1 && c->layer_ok && c->layer_on && !prefetch && (!cache || cache->source == MOE_SOURCE_HOST_DIRECT))
+    // the one-launch layer kernel: always for direct-fill caches (the kernel
+    // reads the misses), for resident experts when asked (MOE_LAYER_KERNEL=1;
+    // the separate router / GEMV kernels are faster there today)
+    if (T == 1 && c->layer_ok && c->layer_on && !prefetch &&
+        ((cache && cache->source == MOE_SOURCE_HOST_DIRECT) || (!cache && c->layer_resident)))
         return run_layer_kernel(c, W, cache, x, step, bias, y, y_bf16, id, gw, trace, s);
     if (T == 1 && !cache) {
         // one token, resident: the router writes the work list itself

@@ -54,16 +54,25 @@ struct GemvCfg<1> {  // down: KS <= 704, up to 11 groups per chunk, one per warp
 // group of every unit, warps 4-7 (when NW = 8) alternate units with them.
 template <int MODE>
 struct DecodeCfg;
+// Gate/up stages hold up to CPS consecutive chunks of one tile (contiguous in
+// the blob): one bulk request per stage.  A CTA's bulk requests are served at
+// a roughly fixed rate whatever their size (measured on B200: 4.6 KB requests
+// stream at ~12 GB/s per CTA, 18-37 KB requests at 45+ GB/s), so larger
+// requests raise the CTA's share of HBM bandwidth.
 template <>
 struct DecodeCfg<0> {
     static constexpr int NW = 4;  // a multiple of 4 (groups per 256-input unit)
-    static constexpr int NSTAGES = 8;
+    static constexpr int CPS = 4;  // chunks per stage
+    static constexpr int NSTAGES = 3;
+    static constexpr int STAGE = CPS * 18 * kGuSlice;
     static constexpr int kTilesPerCta = 1;
 };
 template <>
 struct DecodeCfg<1> {
     static constexpr int NW = 11;
+    static constexpr int CPS = 1;
     static constexpr int NSTAGES = 6;
+    static constexpr int STAGE = 18 * kDownSliceMax;
 };
 
 constexpr int kCtaEntries = 24;  // work-list entries a CTA keeps in shared memory
@@ -544,7 +553,8 @@ __device__ __forceinline__ void stage_task(const float (&v)[8], bool ok, int chu
 template <int MODE>
 __global__ void __launch_bounds__((DecodeCfg<MODE>::NW + 1) * 32) gemv_decode_kernel(GemvArgs A) {
     constexpr int NW = DecodeCfg<MODE>::NW;
-    constexpr int STAGE = GemvCfg<MODE>::STAGE;
+    constexpr int STAGE = DecodeCfg<MODE>::STAGE;
+    constexpr int CPS = DecodeCfg<MODE>::CPS;
     constexpr int kStages = DecodeCfg<MODE>::NSTAGES;
     constexpr int NCONS = NW * 32;
     // gate/up: the work list is the previous launch's output, so wait before
@@ -707,13 +717,16 @@ __global__ void __launch_bounds__((DecodeCfg<MODE>::NW + 1) * 32) gemv_decode_ke
             const uint64_t pol = l2_evict_first();
             int issued = 0;
             bool ok = true;
-            for (int u = u_begin; u < u_end && ok; ++u, ++issued) {
+            for (int u = u_begin, n = 1; u < u_end && ok; u += n, ++issued) {
                 const uint8_t* src;
                 uint32_t bytes;
                 if (MODE == 0) {
+                    // up to CPS chunks, never past the end of the tile
                     const int e = M.gu_entry(u);
-                    src = s_ent[e].blob + size_t(u - M.gu_base(e)) * (18 * kGuSlice);
-                    bytes = 18 * kGuSlice;
+                    const int ul = u - M.gu_base(e), slice = ul % NSg;
+                    n = min(min(CPS - slice % CPS, NSg - slice), u_end - u);
+                    src = s_ent[e].blob + size_t(ul) * (18 * kGuSlice);
+                    bytes = uint32_t(n) * (18 * kGuSlice);
                 } else {
                     int e, tile, slice;
                     M.dn_unit(u, e, tile, slice);
@@ -767,8 +780,10 @@ __global__ void __launch_bounds__((DecodeCfg<MODE>::NW + 1) * 32) gemv_decode_ke
     // -------------------------------------------------- consumers: the units
     float acc = 0.f;
     int seg_start = u_begin;
+    int q = -1;            // stage sequence number of the current unit
+    bool have_q = false;   // whether that stage's copy has landed
+    int st_first = 0;      // first slice of the current stage
     for (int u = u_begin; u < u_end; ++u) {
-        const int i = u - u_begin, st = i % kStages;
         int e, tile, slice, key_u0, key_len;
         if (MODE == 0) {
             e = M.gu_entry(u);
@@ -786,12 +801,22 @@ __global__ void __launch_bounds__((DecodeCfg<MODE>::NW + 1) * 32) gemv_decode_ke
         const int g_in0 = MODE == 0 ? slice * (kGuSlice / kGroup) : M.stage_chunk0(e) / 8 + slice * (ks / kGroup);
         const float w = MODE == 0 ? 1.f : s_row[e].w;
 
-        // gate/up: warps 4j .. 4j+3 read units i = j (mod NW / 4) of the
-        // range, one group each; down: every warp reads every unit
-        const bool mine = MODE == 1 || (i % (NW / 4)) == (warp >> 2);
+        // stages: gate/up, up to CPS chunks of one tile; down, one unit
+        const int in_st = MODE == 0 ? slice % CPS : 0;
+        const bool stage_start = MODE == 1 || in_st == 0 || u == u_begin;
+        const bool stage_end = MODE == 1 || in_st == CPS - 1 || slice == NSg - 1 || u + 1 == u_end;
+        if (stage_start) {
+            ++q;
+            st_first = slice;
+            have_q = ring_wait(&full[q % kStages], (q / kStages) & 1, A.status, &s_abort);
+        }
+        const int st = q % kStages;
+        // gate/up: all four warps read every chunk, one group each; down:
+        // every warp reads every unit
+        const bool mine = true;
         const int gw = MODE == 0 ? (warp & 3) : warp, gstep = MODE == 0 ? 4 : NW;
-        const bool have = mine && ring_wait(&full[st], (i / kStages) & 1, A.status, &s_abort);
-        const uint8_t* chunk = ring + size_t(st) * STAGE;
+        const bool have = mine && have_q;
+        const uint8_t* chunk = ring + size_t(st) * STAGE + size_t(MODE == 0 ? slice - st_first : 0) * (18 * kGuSlice);
         for (int g = gw; have && g < ks / kGroup; g += gstep) {
             const uint4 qa = lds128(chunk + ((2 * g) * 32 + lane) * 16);
             const uint4 qb = lds128(chunk + ((2 * g + 1) * 32 + lane) * 16);
@@ -816,7 +841,7 @@ __global__ void __launch_bounds__((DecodeCfg<MODE>::NW + 1) * 32) gemv_decode_ke
             acc = fmaf(w, part, acc);
         }
         __syncwarp();
-        if (mine && lane == 0) mbar_arrive(&empty[st]);
+        if (stage_end && lane == 0) mbar_arrive(&empty[st]);
 
         const bool seg_end = (u + 1 == u_end) || (u + 1 == key_u0 + key_len);
         if (!seg_end) continue;
@@ -887,7 +912,7 @@ static size_t gemv_smem(int vstride, int T) {
 template <int MODE>
 static size_t decode_smem(int vstride) {
     constexpr int NW = DecodeCfg<MODE>::NW;
-    size_t b = size_t(DecodeCfg<MODE>::NSTAGES) * GemvCfg<MODE>::STAGE + 2 * DecodeCfg<MODE>::NSTAGES * sizeof(uint64_t);
+    size_t b = size_t(DecodeCfg<MODE>::NSTAGES) * DecodeCfg<MODE>::STAGE + 2 * DecodeCfg<MODE>::NSTAGES * sizeof(uint64_t);
     b += (sizeof(FfnEntry) + sizeof(FfnRow)) * kCtaEntries;
     b += size_t(NW) * 32 * 4;
     b += size_t(((vstride / kGroup) + 3) & ~3) * 4 * 2;

@@ -50,9 +50,16 @@ namespace {
 constexpr int kLNW = 12;                      // consumer warps
 constexpr int kLNC = kLNW * 32;               // consumer threads
 constexpr int kLThreads = kLNC + 32;          // + producer warp
-constexpr int kLGuStages = 12;
-constexpr int kLDnStages = 8;
-constexpr int kLGuStage = 18 * kGuSlice;      // 4608 B
+// Gate/up stages hold up to kLChunksPerStage consecutive chunks of one tile (a
+// tile's chunks are contiguous in the blob): one bulk request per stage.  Each
+// bulk request costs a CTA a roughly fixed time whatever its size (measured:
+// 4.6 KB requests stream at ~12 GB/s per CTA, 18-37 KB requests at 45+), so
+// few large requests keep the CTA's share of HBM bandwidth.
+constexpr int kLChunk = 18 * kGuSlice;        // 4608 B: 32 rows x 256 inputs
+constexpr int kLChunksPerStage = 4;
+constexpr int kLGuStages = 6;
+constexpr int kLDnStages = 5;
+constexpr int kLGuStage = kLChunksPerStage * kLChunk;  // 18432 B
 constexpr int kLDnStage = 18 * kDownSliceMax; // 12672 B
 constexpr int kLMaxK = 16;
 constexpr unsigned long long kGridWaitNs = 1000000000ull;  // 1 s
@@ -316,7 +323,7 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_decode_kernel(LayerArgs A)
     if (threadIdx.x == 0) {
         for (int i = 0; i < kLGuStages; ++i) {
             mbar_init(&full_gu[i], 1);
-            mbar_init(&empty_gu[i], 4);  // the four warps that read a gate/up chunk
+            mbar_init(&empty_gu[i], kLNW);  // every consumer warp, once per stage
         }
         for (int i = 0; i < kLDnStages; ++i) {
             mbar_init(&full_dn[i], 1);
@@ -399,11 +406,20 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_decode_kernel(LayerArgs A)
             }
             return issue(ring, stage_bytes, full, empty, nst, issued, src, bytes, en.host != 0);
         };
-        auto issue_gu = [&](int u) {
+        // the stage of units [u, u + n) (consecutive chunks of one tile)
+        auto issue_gu = [&](int u, int n) {
             const int e = gu_entry(u);
             const LEntry& en = s_ent[e];
             return issue_checked(gu_ring, kLGuStage, full_gu, empty_gu, kLGuStages, issued_gu, en,
-                                 en.src + size_t(u - gu_base(e)) * kLGuStage, kLGuStage);
+                                 en.src + size_t(u - gu_base(e)) * kLChunk, uint32_t(n) * kLChunk);
+        };
+        // a pool range [a, b) of whole tiles, stage by stage
+        auto issue_gu_range = [&](int a, int b) {
+            bool good = true;
+            for (int t0 = a; good && t0 < b; t0 += NSg)
+                for (int j = 0; good && j < NSg; j += kLChunksPerStage)
+                    good = issue_gu(t0 + j, min(kLChunksPerStage, NSg - j));
+            return good;
         };
         auto issue_dn = [&](int u) {
             int e, tile, slice;
@@ -422,7 +438,7 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_decode_kernel(LayerArgs A)
             for (int r = 0; r < n_rows; ++r)
                 bulk_g2s(rrow + size_t(r) * D, A.wq + size_t(c + r * G) * D, uint32_t(D), rt_bar, keep);
         }
-        for (int u = sh0; ok && u < sh1; ++u) ok = issue_gu(u);
+        ok = ok && issue_gu_range(sh0, sh1);
         // the plan (entries) is ready
         if (ok) {
             bool w = true;
@@ -435,7 +451,7 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_decode_kernel(LayerArgs A)
         // the rest of the down chunks as the ring frees up
         int v = d0;
         for (; ok && v < d1 && v - d0 < kLDnStages; ++v) ok = issue_dn(v);
-        for (int u = r0; ok && u < r1; ++u) ok = issue_gu(u);
+        ok = ok && issue_gu_range(r0, r1);
         for (; ok && v < d1; ++v) ok = issue_dn(v);
         // every issued copy has landed before the CTA may exit: each lane's own
         // asynchronous copies, then (lane 0) the last uses of every stage
@@ -523,30 +539,36 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_decode_kernel(LayerArgs A)
     // ---------------------------------------------- gate/up consumer loop
     float acc = 0.f;
     int seg_start = 0;
-    // units [ua, ub) of pool `pool` (0 shared, 1 routed: base pb, size PU);
-    // i0 = ring position of unit ua
-    auto gu_units = [&](int ua, int ub, int pool, int pb, int PU, int i0) {
+    // units [ua, ub) of pool `pool` (0 shared, 1 routed: base pb, size PU),
+    // whole tiles; q0 = ring position (stage count) of the range's first stage
+    const int SPT = (NSg + kLChunksPerStage - 1) / kLChunksPerStage;  // stages per tile
+    bool have_stage = false;
+    auto gu_units = [&](int ua, int ub, int pool, int pb, int PU, int q0) {
         seg_start = ua;
         for (int u = ua; u < ub; ++u) {
-            const int i = i0 + (u - ua), st = i % kLGuStages;
             const int e = gu_entry(u);
             const int ul = u - gu_base(e);
             const int tile = ul / NSg, slice = ul - tile * NSg;
             const int key_u0 = gu_base(e) + tile * NSg;
+            const int q = q0 + ((u - ua) / NSg) * SPT + slice / kLChunksPerStage;  // stage sequence number
+            const int st = q % kLGuStages, in_st = slice % kLChunksPerStage;
+            if (in_st == 0) have_stage = lwait(&full_gu[st], uint32_t(q / kLGuStages) & 1u, A.status, &s_abort);
+            const int i = u - ua;
             const bool mine = (i % (kLNW / 4)) == (warp >> 2);
             const int gw = warp & 3;
-            const bool have = mine && lwait(&full_gu[st], uint32_t(i / kLGuStages) & 1u, A.status, &s_abort);
+            const bool have = mine && have_stage;
             if (have) {
-                const uint8_t* chunk = gu_ring + size_t(st) * kLGuStage;
+                const uint8_t* chunk = gu_ring + size_t(st) * kLGuStage + size_t(in_st) * kLChunk;
                 const int gi = slice * (kGuSlice / kGroup) + gw;  // input group
                 uint4 qa, qb;
                 uint32_t sbw;
                 acc += group_dot(chunk, kGuSlice, gw, lane, xq + gi * 8, xsx[gi], xX[gi], &qa, &qb, &sbw);
                 const LEntry& en = s_ent[e];
-                if (en.wb) group_writeback(en.wb + size_t(ul) * kLGuStage, kGuSlice, gw, lane, qa, qb, sbw);
+                if (en.wb) group_writeback(en.wb + size_t(ul) * kLChunk, kGuSlice, gw, lane, qa, qb, sbw);
             }
             __syncwarp();
-            if (mine && lane == 0) mbar_arrive(&empty_gu[st]);
+            // every warp leaves the stage after its last chunk
+            if ((in_st == kLChunksPerStage - 1 || slice == NSg - 1) && lane == 0) mbar_arrive(&empty_gu[st]);
             const bool seg_end = (u + 1 == ub) || (u + 1 == key_u0 + NSg);
             if (!seg_end) continue;
             named_sync(1, kLNC);
@@ -793,7 +815,7 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_decode_kernel(LayerArgs A)
     named_sync(1, kLNC);
 
     // ------------------------------------------- the routed gate/up chunks
-    gu_units(r0, r1, 1, ush, Urt, sh1 - sh0);
+    gu_units(r0, r1, 1, ush, Urt, ((sh1 - sh0) / NSg) * SPT);
 
     // ------------------------------------------------ phase 3: down + combine
     named_sync(1, kLNC);

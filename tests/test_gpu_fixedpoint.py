@@ -111,10 +111,14 @@ def test_expert_ffn_fixed_point_edges(O, layer, case):
     ctx.close()
 
 
+@pytest.mark.parametrize("kernel", ["split", "layer"])
 @pytest.mark.parametrize("case", CASES)
-def test_layer_forward_fixed_point_edges(O, layer, case):
-    """The whole one-token resident layer on the same inputs; the activation
-    outlier case biases the router towards expert 9 so it is selected."""
+def test_layer_forward_fixed_point_edges(O, layer, case, kernel, monkeypatch):
+    """The whole one-token resident layer on the same inputs, through the
+    separate router / GEMV kernels and through the one-launch layer kernel;
+    the activation outlier case biases the router towards expert 9 so it is
+    selected."""
+    monkeypatch.setenv("MOE_LAYER_KERNEL", "1" if kernel == "layer" else "0")
     L = layer
     rng = np.random.default_rng(1001 if case == "activation_outlier" else 100 + CASES.index(case))
     xb = _inputs(case, rng)
