@@ -744,7 +744,9 @@ def run_sweep(args, dims, dist):
     def plan_point(S, zs, policy=moe.MOE_POLICY_LFU, period=0):
         """Router + cache plan over Tn tokens x all layers: hit rate and H2D bytes per token."""
         ctx = moe.Ctx.from_dims(d, max_tokens=1, S=S)
-        bias = [torch.from_numpy(synth.zipf_bias(args.seed, l, d.E, s=zs)).cuda() for l in range(args.layers)]
+        # independent states per (token, layer): the unchained bias strength
+        bias = [torch.from_numpy(synth.zipf_bias(args.seed, l, d.E, s=zs, lam=synth.ZIPF_LAMBDA_UNCHAINED)).cuda()
+                for l in range(args.layers)]
         states = [torch.empty(ctx.state_words(), dtype=torch.int32, device="cuda") for _ in range(args.layers)]
         slots = torch.empty((S, 256), dtype=torch.uint8, device="cuda")  # plan only: never read
         caches = []
@@ -800,9 +802,15 @@ def run_sweep(args, dims, dist):
         line = {"metric": "MoE decode cache sweep: hit rate, H2D bytes/token, tokens/s (30 layers, 4-bit g64)",
                 "value": base["tokens_per_s"], "unit": "tokens/s", "n_gpus": dist.world, "steps": 64, "warmup": 16,
                 "ms_per_step": 1e3 / base["tokens_per_s"], "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "vs_baseline": None,
+                "dtype": "int4 weights x 16-bit fixed-point activations (dp4a), fp32 accumulation",
+                "data": "synthetic",
                 "config": {"workload": "sweep", "layers": args.layers, "sweep_tokens": Tn,
-                           "value_point": "slots 16, zipf 1.1, LFU", "hidden_state_generation_s": gen_s},
+                           "value_point": "slots 16, zipf 1.1, LFU", "hidden_state_generation_s": gen_s,
+                           "hit_rate_inputs": "independent hidden states per (token, layer), bias strength "
+                                              f"{synth.ZIPF_LAMBDA_UNCHAINED}",
+                           "tokens_per_s_inputs": "chained decode (residual stream), bias strength "
+                                                  f"{args.zipf_lambda}"},
                 "sweep": results, "policies": policies}
         print(json.dumps(line), flush=True)
     return 0

@@ -39,6 +39,11 @@ cudaError_t launch_bf16_to_f32(const uint16_t* x, float* out, size_t n, bool pdl
 
 using namespace moe;
 
+// cuStreamWriteValue32 (driver API), resolved at run time through the runtime's
+// entry-point query so the library links against the runtime only.
+typedef int (*StreamWriteValue32)(cudaStream_t stream, unsigned long long addr, unsigned int value,
+                                  unsigned int flags);
+
 // Calls of at least this many tokens run the experts as the tcgen05 grouped
 // GEMM (tokens grouped per expert); one token runs the streamed GEMV kernels.
 // Measured on B200 with the 26B-A4B layer, 30 layers resident: 2 tokens 567
@@ -53,6 +58,15 @@ struct moe_ctx {
     int sms = 0;
     cudaStream_t side = nullptr;
     cudaEvent_t ev_plan = nullptr, ev_fill = nullptr, ev_wave = nullptr;
+    // per-miss completion (optional): after each one-token miss copy the side
+    // stream writes the call's sequence number into ready[slot] (a stream
+    // memory write, executed by the stream itself, not by a kernel); the
+    // routed experts' kernel then waits for it per expert instead of for all
+    // copies
+    uint32_t* ready = nullptr;                // [n_slots] (device)
+    StreamWriteValue32 write_value = nullptr;  // driver entry point, or null: event join
+    bool per_miss = false;                    // MOE_PER_MISS=1 (measured slower on B200: off by default)
+    bool inject_skip_ready = false;           // MOE_INJECT_SKIP_READY=1: omit the first write of a call
     PlanMailbox* mbox_host = nullptr;
     PlanMailbox* mbox_dev = nullptr;
     uint32_t seq = 0;
@@ -167,6 +181,7 @@ void free_ctx(moe_ctx* c) {
     }
     for (auto e : c->pool) cudaEventDestroy(e);
     cudaFree(c->status);
+    cudaFree(c->ready);
     cudaFree(c->layer_logits);
     cudaFree(c->layer_partials);
     cudaFree(c->layer_bar);
@@ -343,6 +358,8 @@ DecodeWLTarget decode_target(moe_ctx* c, WorkList* wl, FfnEntry* en, FfnRow* row
     t.D = c->d.d_model;
     t.h_shared_off = c->h_shared_off;
     t.blob_bytes = c->blob_routed;
+    t.ready = nullptr;
+    t.ready_val = 0;
     return t;
 }
 
@@ -415,7 +432,8 @@ void copy_trace(const PlanMailbox* mb, moe_plan_trace* tr, size_t blob, uint64_t
 
 // Issues the copies of wave `w`'s misses on the side stream after `after`
 // (an event on the compute stream), then makes `s` wait for them.
-int fill_wave(moe_ctx* c, const moe_slot_cache* cache, int w, cudaEvent_t after, cudaStream_t s, uint64_t* bytes) {
+int fill_wave(moe_ctx* c, const moe_slot_cache* cache, int w, cudaEvent_t after, cudaStream_t s, uint64_t* bytes,
+              uint32_t ready_seq = 0) {
     const PlanMailbox* mb = c->mbox_host;
     const size_t nb = c->blob_routed;
     if (cudaStreamWaitEvent(c->side, after, 0) != cudaSuccess) return MOE_ERR_CUDA;
@@ -440,25 +458,54 @@ int fill_wave(moe_ctx* c, const moe_slot_cache* cache, int w, cudaEvent_t after,
         if (cudaStreamWaitEvent(s, c->ev_fill, 0) != cudaSuccess) return MOE_ERR_CUDA;
         return MOE_OK;
     }
-    for (int i = 0; i < mb->n_distinct; ++i) {
-        if (mb->wave[i] != w || mb->hit[i]) continue;
-        const int e = mb->expert[i], sl = mb->slot[i];
-        if (e < 0 || e >= c->d.n_experts || sl < 0 || sl >= c->d.n_slots) return MOE_ERR_RANGE;
-        uint8_t* dst = cache->slots + size_t(sl) * cache->slot_stride;
-        // a blob prefetched for this cache is moved from its HBM buffer (the
-        // prefetch copy is earlier on the same side stream)
-        int pb = -1;
-        for (const auto& f : c->pf_table)
-            if (f.state == cache->state && f.store == cache->store && f.expert == e) pb = f.buf;
-        const cudaError_t ce =
-            pb >= 0 ? cudaMemcpyAsync(dst, c->pf_buf + size_t(pb) * c->pf_stride, nb, cudaMemcpyDeviceToDevice, c->side)
-                    : cudaMemcpyAsync(dst, cache->store + size_t(e) * cache->store_stride, nb, cudaMemcpyHostToDevice,
-                                      c->side);
-        if (ce != cudaSuccess) return MOE_ERR_CUDA;
-        if (pb >= 0) c->pf_used += nb;
-        *bytes += nb;
+    // Blobs prefetched for this cache are moved from their HBM buffers (the
+    // prefetch copies are earlier on the same side stream), the others copied
+    // from the host store.  With per-miss completion (ready_seq != 0) the
+    // staged blobs go first and the compute stream waits for them by event:
+    // a device-to-device copy may run as a kernel, which must not queue behind
+    // routed-expert kernels that wait on these blobs.  The host copies run on
+    // the copy engine and are announced one by one.
+    bool first_ready = true;
+    int n_staged = 0;
+    for (int pass = 0; pass < 2; ++pass) {
+        for (int i = 0; i < mb->n_distinct; ++i) {
+            if (mb->wave[i] != w || mb->hit[i]) continue;
+            const int e = mb->expert[i], sl = mb->slot[i];
+            if (e < 0 || e >= c->d.n_experts || sl < 0 || sl >= c->d.n_slots) return MOE_ERR_RANGE;
+            uint8_t* dst = cache->slots + size_t(sl) * cache->slot_stride;
+            int pb = -1;
+            for (const auto& f : c->pf_table)
+                if (f.state == cache->state && f.store == cache->store && f.expert == e) pb = f.buf;
+            if ((pb >= 0) != (pass == 0)) continue;
+            const cudaError_t ce =
+                pb >= 0 ? cudaMemcpyAsync(dst, c->pf_buf + size_t(pb) * c->pf_stride, nb, cudaMemcpyDeviceToDevice,
+                                          c->side)
+                        : cudaMemcpyAsync(dst, cache->store + size_t(e) * cache->store_stride, nb,
+                                          cudaMemcpyHostToDevice, c->side);
+            if (ce != cudaSuccess) return MOE_ERR_CUDA;
+            if (ready_seq) {
+                // this blob has landed once the stream reaches the write (the
+                // default flags fence the copy before it); the fault injection
+                // of the tests leaves the call's first write out
+                const bool skip = c->inject_skip_ready && first_ready;
+                first_ready = false;
+                if (!skip &&
+                    c->write_value(c->side, reinterpret_cast<unsigned long long>(c->ready + sl), ready_seq, 0) != 0)
+                    return MOE_ERR_CUDA;
+            }
+            if (pb >= 0) {
+                c->pf_used += nb;
+                ++n_staged;
+            }
+            *bytes += nb;
+        }
+        if (pass == 0 && ready_seq && n_staged > 0) {
+            if (cudaEventRecord(c->ev_fill, c->side) != cudaSuccess) return MOE_ERR_CUDA;
+            if (cudaStreamWaitEvent(s, c->ev_fill, 0) != cudaSuccess) return MOE_ERR_CUDA;
+        }
     }
     prof_mark(c, MOE_PROF_H2D, false, c->side);
+    if (ready_seq) return MOE_OK;  // the kernels wait per blob
     if (cudaEventRecord(c->ev_fill, c->side) != cudaSuccess) return MOE_ERR_CUDA;
     if (cudaStreamWaitEvent(s, c->ev_fill, 0) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
@@ -588,6 +635,21 @@ int moe_ctx_create(const moe_dims* dims, int device, moe_ctx** out) {
     ok = ok && dalloc(&c->layer_partials, size_t(6) * c->layer_G * 32) == cudaSuccess;
     ok = ok && dalloc(&c->layer_bar, 4) == cudaSuccess;
     ok = ok && dalloc(&c->stats, MOE_STATS) == cudaSuccess;
+    ok = ok && dalloc(&c->ready, size_t(d.n_slots)) == cudaSuccess;
+    ok = ok && cudaMemset(c->ready, 0, size_t(d.n_slots) * sizeof(uint32_t)) == cudaSuccess;
+    if (ok) {
+        // the stream memory write; without it the routed experts wait for all
+        // of a call's copies through an event, as multi-token calls do
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPointByVersion("cuStreamWriteValue32", &fn, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess && fn)
+            c->write_value = reinterpret_cast<StreamWriteValue32>(fn);
+        cudaGetLastError();
+        if (const char* v = std::getenv("MOE_PER_MISS")) c->per_miss = v[0] == '1';
+        if (const char* v = std::getenv("MOE_INJECT_SKIP_READY")) c->inject_skip_ready = v[0] == '1';
+    }
     ok = ok && cudaMemset(c->layer_bar, 0, 4 * sizeof(unsigned)) == cudaSuccess;
     ok = ok && cudaMemset(c->stats, 0, MOE_STATS * sizeof(uint64_t)) == cudaSuccess;
     ok = ok && cudaMemset(c->status, 0, sizeof(int)) == cudaSuccess;
@@ -914,9 +976,20 @@ static int layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache*
     const DecodeWLTarget t_sh = one ? decode_target(c, c->wl, c->entries, c->rows, cache->slots, cache->slot_stride,
                                                     W->shared_blob)
                                     : DecodeWLTarget{};
-    const DecodeWLTarget t_rt = one ? decode_target(c, c->wl2, c->entries2, c->rows2, cache->slots,
-                                                    cache->slot_stride, nullptr)
-                                    : DecodeWLTarget{};
+    DecodeWLTarget t_rt = one ? decode_target(c, c->wl2, c->entries2, c->rows2, cache->slots, cache->slot_stride,
+                                              nullptr)
+                              : DecodeWLTarget{};
+    // one token from host memory, when enabled: list B waits per missed blob.
+    // Measured on B200 (30 layers, 16 slots): the stream memory write after
+    // each copy leaves the link idle for a few microseconds, more than the
+    // overlap gains (143.7 vs 152.4 tokens/s), so the default joins all of a
+    // call's copies with one event before list B
+    const bool per_miss = one && c->per_miss && c->write_value && cache->source == MOE_SOURCE_HOST && cache->store &&
+                          seq != 0u;
+    if (per_miss) {
+        t_rt.ready = c->ready;
+        t_rt.ready_val = seq;
+    }
     prof_mark(c, MOE_PROF_PLAN, true, s);
     cudaError_t e = launch_plan(id, T * K, c->d.n_experts, c->d.n_slots, cache->policy, cache->decay_period,
                                 cache->state, step, c->pair_slot,
@@ -971,7 +1044,7 @@ static int layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache*
                 if (cudaEventRecord(c->ev_wave, s) != cudaSuccess) return MOE_ERR_CUDA;
                 after = c->ev_wave;
             }
-            r = fill_wave(c, cache, w, after, s, &bytes);
+            r = fill_wave(c, cache, w, after, s, &bytes, per_miss ? seq : 0u);
             if (r != MOE_OK) return r;
         }
         if (one) {

@@ -167,6 +167,10 @@ __device__ __forceinline__ float gelu_tanh(float v) {
 // token rows that use it.
 struct FfnEntry {
     const uint8_t* blob;   // expert blob (device, 256-byte aligned)
+    // null, or a word that holds ready_val once the blob has landed (a miss
+    // copied in by the copy engine while this list already runs)
+    const uint32_t* ready;
+    uint32_t ready_val;
     int F;                 // FFN width of this expert
     int n_rows;            // 1..kMaxRows
     int row0;              // first row in FfnRow[]
@@ -208,6 +212,9 @@ struct DecodeWLTarget {
     int F, FS, D;
     int h_shared_off;           // float offset of the shared row's activation
     size_t blob_bytes;          // routed blob size (for L2 prefetch)
+    // routed entries of slot s wait until ready[s] == ready_val (null: no wait)
+    const uint32_t* ready;
+    uint32_t ready_val;
 };
 
 }  // namespace moe

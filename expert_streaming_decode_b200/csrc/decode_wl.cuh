@@ -25,6 +25,8 @@ __device__ __forceinline__ void write_decode_worklist(const DecodeWLTarget& t, i
         const int e = nsh + j;
         FfnEntry en;
         en.blob = t.slot_base + size_t(slot) * t.slot_stride;
+        en.ready = t.ready ? t.ready + slot : nullptr;
+        en.ready_val = t.ready_val;
         en.F = t.F;
         en.n_rows = 1;
         en.row0 = e;
@@ -42,6 +44,8 @@ __device__ __forceinline__ void write_decode_worklist(const DecodeWLTarget& t, i
         if (nsh) {
             FfnEntry en;
             en.blob = t.shared_blob;
+            en.ready = nullptr;
+            en.ready_val = 0;
             en.F = t.FS;
             en.n_rows = 1;
             en.row0 = 0;

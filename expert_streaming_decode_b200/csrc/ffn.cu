@@ -55,17 +55,26 @@ struct GemvCfg<1> {  // down: KS <= 704, up to 11 groups per chunk, one per warp
 template <int MODE>
 struct DecodeCfg;
 // Gate/up stages hold up to CPS consecutive chunks of one tile (contiguous in
-// the blob): one bulk request per stage.  A CTA's bulk requests are served at
-// a roughly fixed rate whatever their size (measured on B200: 4.6 KB requests
-// stream at ~12 GB/s per CTA, 18-37 KB requests at 45+ GB/s), so larger
-// requests raise the CTA's share of HBM bandwidth.
+// the blob): one bulk request per stage.  Larger requests raise one CTA's
+// share of HBM bandwidth, but the ring's shared memory sets how many of the
+// layer's tile CTAs (484 for the 26B-A4B shapes) are resident at once; on
+// B200 one-chunk stages (8 x 4.6 KB, five CTAs per SM: every tile in one
+// wave) measured faster than 3 x 18 KB (three CTAs per SM).  The two values
+// can be set at compile time for tuning.
+#ifndef MOE_DECODE_GU_CPS
+#define MOE_DECODE_GU_CPS 1
+#endif
+#ifndef MOE_DECODE_GU_STAGES
+#define MOE_DECODE_GU_STAGES 8
+#endif
 template <>
 struct DecodeCfg<0> {
     static constexpr int NW = 4;  // a multiple of 4 (groups per 256-input unit)
-    static constexpr int CPS = 4;  // chunks per stage
-    static constexpr int NSTAGES = 3;
+    static constexpr int CPS = MOE_DECODE_GU_CPS;  // chunks per stage
+    static constexpr int NSTAGES = MOE_DECODE_GU_STAGES;
     static constexpr int STAGE = CPS * 18 * kGuSlice;
     static constexpr int kTilesPerCta = 1;
+    static_assert(CPS >= 1 && NSTAGES >= 1, "gate/up ring");
 };
 template <>
 struct DecodeCfg<1> {
@@ -76,6 +85,7 @@ struct DecodeCfg<1> {
 };
 
 constexpr int kCtaEntries = 24;  // work-list entries a CTA keeps in shared memory
+static_assert(kCtaEntries <= 32, "the one-token producer keeps one bit per entry");
 
 struct GemvArgs {
     const WorkList* wl;
@@ -106,11 +116,45 @@ __device__ __forceinline__ int cta_of(int u, int U, int G) { return int(((long l
 
 __device__ __forceinline__ uint4 lds128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
 
-// Bounded wait that gives up at once after any warp of the CTA timed out, so
-// a failure costs one time-out, not one per stage.
+// Bounded wait that gives up at once after any warp of the CTA timed out or
+// the producer stopped (the flag is polled while waiting), so a failure costs
+// one time-out, not one per stage.
 __device__ __forceinline__ bool ring_wait(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag) {
     if (*abort_flag) return false;
-    if (mbar_wait(bar, parity, status)) return true;
+    unsigned long long t0 = 0;
+    for (uint32_t i = 0; i < kSpinLimit; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 255) == 255) {
+            if (*abort_flag) return false;
+            const unsigned long long t = global_ns();
+            if (t0 == 0) t0 = t;
+            else if (t - t0 > kWaitLimitNs) break;
+        }
+    }
+    set_status(status, MOE_ERR_TIMEOUT);
+    *abort_flag = 1;
+    return false;
+}
+
+// Bounded wait (producer lane) until an entry's blob has landed: *ready ==
+// want, written by the stream that copied it (after the copy, with a fence).
+// Gives up after kWaitLimitNs, records MOE_ERR_TIMEOUT and stops the CTA.
+__device__ __forceinline__ bool ready_wait(const uint32_t* ready, uint32_t want, int* status,
+                                           volatile int* abort_flag) {
+    unsigned long long t0 = 0;
+    for (uint32_t i = 0; i < kSpinLimit; ++i) {
+        uint32_t v;
+        asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(ready) : "memory");
+        if (v == want) return true;
+        if (*abort_flag) return false;
+        if ((i & 15) == 15) {
+            const unsigned long long t = global_ns();
+            if (t0 == 0) t0 = t;
+            else if (t - t0 > kWaitLimitNs) break;
+        }
+        __nanosleep(64);
+    }
+    set_status(status, MOE_ERR_TIMEOUT);
     *abort_flag = 1;
     return false;
 }
@@ -649,6 +693,8 @@ __global__ void __launch_bounds__((DecodeCfg<MODE>::NW + 1) * 32) gemv_decode_ke
         W.F = 64;
         W.FS = A.FS;
         my_en.blob = A.shared_blob;
+        my_en.ready = nullptr;
+        my_en.ready_val = 0;
         my_en.F = A.FS;
         my_en.n_rows = 1;
         my_en.row0 = 0;
@@ -717,22 +763,31 @@ __global__ void __launch_bounds__((DecodeCfg<MODE>::NW + 1) * 32) gemv_decode_ke
             const uint64_t pol = l2_evict_first();
             int issued = 0;
             bool ok = true;
+            uint32_t landed = 0;  // entries (bit e) whose blob is known to have landed
             for (int u = u_begin, n = 1; u < u_end && ok; u += n, ++issued) {
                 const uint8_t* src;
                 uint32_t bytes;
+                int e;
                 if (MODE == 0) {
                     // up to CPS chunks, never past the end of the tile
-                    const int e = M.gu_entry(u);
+                    e = M.gu_entry(u);
                     const int ul = u - M.gu_base(e), slice = ul % NSg;
                     n = min(min(CPS - slice % CPS, NSg - slice), u_end - u);
                     src = s_ent[e].blob + size_t(ul) * (18 * kGuSlice);
                     bytes = uint32_t(n) * (18 * kGuSlice);
                 } else {
-                    int e, tile, slice;
+                    int tile, slice;
                     M.dn_unit(u, e, tile, slice);
                     const int F = M.width(e), ks = down_ks(F);
                     src = s_ent[e].blob + gu_section_bytes(D, F) + size_t(tile * (F / ks) + slice) * (18u * ks);
                     bytes = 18u * ks;
+                }
+                // a miss still being copied in: wait for its ready word first
+                // (entries index s_ent, fewer than 32)
+                if (!((landed >> e) & 1u)) {
+                    if (s_ent[e].ready) ok = ready_wait(s_ent[e].ready, s_ent[e].ready_val, A.status, &s_abort);
+                    if (!ok) break;
+                    landed |= 1u << e;
                 }
                 const int st = issued % kStages;
                 if (issued >= kStages) ok = ring_wait(&empty[st], ((issued / kStages) - 1) & 1, A.status, &s_abort);
@@ -1216,6 +1271,8 @@ __global__ void __launch_bounds__(kWlThreads) build_worklist_kernel(WorkListArgs
     for (int j = threadIdx.x; j < nsh; j += blockDim.x) {
         FfnEntry en;
         en.blob = a.shared_blob;
+        en.ready = nullptr;
+        en.ready_val = 0;
         en.F = a.FS;
         en.row0 = j * mr;
         en.n_rows = min(mr, a.T - j * mr);
@@ -1228,6 +1285,8 @@ __global__ void __launch_bounds__(kWlThreads) build_worklist_kernel(WorkListArgs
             const int e = ebase[sl] + j;
             FfnEntry en;
             en.blob = a.slot_base + size_t(sl) * a.slot_stride;
+            en.ready = nullptr;
+            en.ready_val = 0;
             en.F = a.F;
             en.row0 = off[sl] + j * mr;
             en.n_rows = min(mr, cnt[sl] - j * mr);

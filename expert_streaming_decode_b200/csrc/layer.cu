@@ -56,10 +56,16 @@ constexpr int kLThreads = kLNC + 32;          // + producer warp
 // 4.6 KB requests stream at ~12 GB/s per CTA, 18-37 KB requests at 45+), so
 // few large requests keep the CTA's share of HBM bandwidth.
 constexpr int kLChunk = 18 * kGuSlice;        // 4608 B: 32 rows x 256 inputs
-constexpr int kLChunksPerStage = 4;
-constexpr int kLGuStages = 6;
+#ifndef MOE_LAYER_GU_CPS
+#define MOE_LAYER_GU_CPS 4
+#endif
+#ifndef MOE_LAYER_GU_STAGES
+#define MOE_LAYER_GU_STAGES 6
+#endif
+constexpr int kLChunksPerStage = MOE_LAYER_GU_CPS;  // compile-time tuning values
+constexpr int kLGuStages = MOE_LAYER_GU_STAGES;
 constexpr int kLDnStages = 5;
-constexpr int kLGuStage = kLChunksPerStage * kLChunk;  // 18432 B
+constexpr int kLGuStage = kLChunksPerStage * kLChunk;  // 18432 B at four chunks
 constexpr int kLDnStage = 18 * kDownSliceMax; // 12672 B
 constexpr int kLMaxK = 16;
 constexpr unsigned long long kGridWaitNs = 1000000000ull;  // 1 s

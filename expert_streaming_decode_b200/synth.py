@@ -197,6 +197,11 @@ def router_weights(seed, layer, E, D, G=64):
 # 0.55 keeps both the early tokens and the whole sequence in the pages' 60-70 %
 # band, with next-token / two-token repeats close to their 40 % / 57 %.
 ZIPF_LAMBDA = 0.55
+# The same band for independent hidden states per (token, layer) (no residual
+# stream, so consecutive tokens route less alike): the router + LFU plan over
+# such states give a 0.67 hit rate at 16 slots and Zipf 1.1 with lambda 0.75.
+# The cache sweep and the plan-only tests draw their states this way.
+ZIPF_LAMBDA_UNCHAINED = 0.75
 
 
 def zipf_bias(seed, layer, E, s=1.1, lam=None):

@@ -385,3 +385,51 @@ def test_direct_fill_rejects_unpinned_store():
     assert ei.value.code == moe.MOE_ERR_ARG
     ctx.sync()
     ctx.close()
+
+
+def test_missing_ready_word_times_out(O, monkeypatch):
+    """Per-miss completion (MOE_PER_MISS=1): a one-token miss copied from
+    pinned memory is announced by a stream memory write after its copy, and
+    the routed experts' kernel waits for that word (bounded).  With the first write of a call left
+    out on the host (MOE_INJECT_SKIP_READY=1) the wait runs out: the call
+    reports MOE_ERR_TIMEOUT within seconds and the context stays usable (a
+    resident call on it then matches the oracle)."""
+    import time
+
+    d = TINY
+    S = 6
+    monkeypatch.setenv("MOE_PER_MISS", "1")
+    monkeypatch.setenv("MOE_INJECT_SKIP_READY", "1")
+    L = Layer(d, layer=0, seed=1, zipf_s=1.1, resident=True, pinned=True)
+    ctx = moe.Ctx.from_dims(d, max_tokens=1, S=S)
+    monkeypatch.delenv("MOE_INJECT_SKIP_READY")
+    monkeypatch.delenv("MOE_PER_MISS")
+    state = torch.empty(ctx.state_words(), dtype=torch.int32, device="cuda")
+    slots = torch.empty((S, L.stride), dtype=torch.uint8, device="cuda")
+    c = moe.slot_cache(slots, L.stride, state, L.store_t, L.stride)
+    moe.cache_reset(ctx, c)
+    y = torch.empty((1, d.D), dtype=torch.float32, device="cuda")
+    xb = synth.hidden(1, 0, 0, d.D)
+    t0 = time.time()
+    moe.layer_forward(ctx, L.weights(resident=False), c, bf16_tensor(xb[None]), 1, 0, L.bias_t, y)
+    assert ctx.sync_status() == moe.MOE_ERR_TIMEOUT  # a cold cache: every selection misses
+    assert time.time() - t0 < 15.0
+    # the same context, resident experts (no copies): correct again
+    moe.layer_forward(ctx, L.weights(), None, bf16_tensor(xb[None]), 1, 0, L.bias_t, y)
+    assert ctx.sync_status() == 0
+    want = L.oracle_token(O, xb)[3]
+    assert rel_err(y.cpu().numpy()[0].astype(np.float64), want) <= TOL
+    ctx.close()
+
+
+@pytest.mark.parametrize("d,layers,tokens,S,every,prefetch", [(TINY, 3, 30, 6, 1, 0), (FULL, 2, 8, 16, 4, 0),
+                                                              (FULL, 3, 8, 16, 4, 8)],
+                         ids=["tiny", "full", "full-lookahead"])
+def test_streaming_decode_per_miss_ready(O, monkeypatch, d, layers, tokens, S, every, prefetch):
+    """Per-miss completion enabled (MOE_PER_MISS=1): list B starts before its
+    blobs have landed and waits per blob; staged look-ahead blobs (device to
+    device copies, which may run as kernels) are joined by event first.
+    Traces, slot contents and outputs are the oracle's."""
+    monkeypatch.setenv("MOE_PER_MISS", "1")
+    _streaming(O, d, layers=layers, tokens=tokens, S=S, check_y_every=every, prefetch=prefetch,
+               same_x=prefetch > 0)

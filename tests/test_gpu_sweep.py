@@ -23,7 +23,7 @@ def test_sweep_trace_bit_exact(S, zs):
     slots = torch.empty((S, 256), dtype=torch.uint8, device="cuda")  # plan only: never read
     for l in range(layers):
         q, s_ = synth.router_weights(3, l, d.E, d.D)
-        b = synth.zipf_bias(3, l, d.E, s=zs)
+        b = synth.zipf_bias(3, l, d.E, s=zs, lam=synth.ZIPF_LAMBDA_UNCHAINED)  # independent states per layer
         wq.append((q, torch.from_numpy(q).cuda()))
         ws.append((s_, torch.from_numpy(s_.view(np.int16)).cuda()))
         bias.append((b, torch.from_numpy(b).cuda()))

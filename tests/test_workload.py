@@ -5,7 +5,7 @@ HN: Motor de codigo abierto que ejecuta Gemma 4 26B en 2 GB de RAM", section
 popularity bias.
 
 This CPU check uses independent hidden states per token (no layer chain), for
-which a bias strength of 0.75 lands in the band.  The benchmark's decode
+which a bias strength of 0.75 (synth.ZIPF_LAMBDA_UNCHAINED) lands in the band.  The benchmark's decode
 chains the layers through a residual stream, which makes consecutive tokens
 route alike; there the strength is 0.55 (synth.ZIPF_LAMBDA, calibrated on the
 GPU over the chained 30-layer decode), checked by the benchmark's own
@@ -20,7 +20,7 @@ def test_zipf_hit_rate_band_unchained():
     O = oracle.get()
     d = synth.GEMMA4_26B
     wq, ws = synth.router_weights(0, 0, d.E, d.D)
-    bias = synth.zipf_bias(0, 0, d.E, s=1.1, lam=0.75)
+    bias = synth.zipf_bias(0, 0, d.E, s=1.1, lam=synth.ZIPF_LAMBDA_UNCHAINED)
     st = oracle.LfuState(d.E, 16)
     hits = total = 0
     for t in range(700):
