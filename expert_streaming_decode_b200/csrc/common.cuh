@@ -212,9 +212,10 @@ struct DecodeWLTarget {
     int F, FS, D;
     int h_shared_off;           // float offset of the shared row's activation
     size_t blob_bytes;          // routed blob size (for L2 prefetch)
-    // routed entries of slot s wait until ready[s] == ready_val (null: no wait)
-    const uint32_t* ready;
-    uint32_t ready_val;
+    // routed entries of slot s wait until ready[s] == ready_val (null: no wait;
+    // the default, so a target built field by field never waits on garbage)
+    const uint32_t* ready = nullptr;
+    uint32_t ready_val = 0;
 };
 
 }  // namespace moe

@@ -1172,6 +1172,8 @@ __global__ void __launch_bounds__(kWlThreads) build_worklist_kernel(WorkListArgs
             t.D = a.D;
             t.h_shared_off = a.h_shared_off;
             t.blob_bytes = 0;
+            t.ready = nullptr;  // every blob is in place before this list runs
+            t.ready_val = 0;
             write_decode_worklist(t, a.K, sl, w, take);
         }
         return;

@@ -293,6 +293,7 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_decode_kernel(LayerArgs A)
 
     __shared__ LEntry s_ent[kLMaxK + 1];
     __shared__ float red[kLNW * 32];
+    __shared__ float red2[2][kLNW * 32];
     __shared__ int s_sel_id[kLMaxK], s_ulist[kLMaxK], s_uslot[kLMaxK], s_uhit[kLMaxK], s_uvic[kLMaxK];
     __shared__ float s_sel_l[kLMaxK];
     __shared__ int s_nan, s_abort, s_unit_h[kLDnStages * 4 + 1];
@@ -301,7 +302,6 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_decode_kernel(LayerArgs A)
     // work ranges: gate/up units (shared tiles, then routed k = 0..K-1), down
     // units (tile-major: per 32-row tile the shared slices, then routed k)
     const int ush = nsh ? (FS / 16) * NSg : 0, urt = (F / 16) * NSg;
-    const int Ugu = ush + K * urt;
     const int ks_sh = nsh ? down_ks(FS) : 1, ks_rt = down_ks(F);
     const int ns_sh = nsh ? FS / ks_sh : 0, ns_rt = F / ks_rt;
     const int upt = ns_sh + K * ns_rt, tiles_dn = D / kChunkRows;
@@ -311,7 +311,6 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_decode_kernel(LayerArgs A)
     // during the router phase and routed weights after the plan
     // (whole 16-output tiles per CTA: no tile is split between CTAs, so the
     // gate/up results need no cross-CTA reduction)
-    const int Urt = Ugu - ush;
     const int TS = nsh ? FS / 16 : 0, TR = K * (F / 16);
     const int sh0 = range_start(c, TS, G) * NSg, sh1 = range_start(c + 1, TS, G) * NSg;
     const int r0 = ush + range_start(c, TR, G) * NSg, r1 = ush + range_start(c + 1, TR, G) * NSg;
@@ -543,82 +542,54 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_decode_kernel(LayerArgs A)
     if (threadIdx.x == 0) gen_a = grid_arrive(A.bar, unsigned(G));
 
     // ---------------------------------------------- gate/up consumer loop
-    float acc = 0.f;
-    int seg_start = 0;
-    // units [ua, ub) of pool `pool` (0 shared, 1 routed: base pb, size PU),
-    // whole tiles; q0 = ring position (stage count) of the range's first stage
-    const int SPT = (NSg + kLChunksPerStage - 1) / kLChunksPerStage;  // stages per tile
-    bool have_stage = false;
-    auto gu_units = [&](int ua, int ub, int pool, int pb, int PU, int q0) {
-        seg_start = ua;
-        for (int u = ua; u < ub; ++u) {
-            const int e = gu_entry(u);
-            const int ul = u - gu_base(e);
-            const int tile = ul / NSg, slice = ul - tile * NSg;
-            const int key_u0 = gu_base(e) + tile * NSg;
-            const int q = q0 + ((u - ua) / NSg) * SPT + slice / kLChunksPerStage;  // stage sequence number
-            const int st = q % kLGuStages, in_st = slice % kLChunksPerStage;
-            if (in_st == 0) have_stage = lwait(&full_gu[st], uint32_t(q / kLGuStages) & 1u, A.status, &s_abort);
-            const int i = u - ua;
-            const bool mine = (i % (kLNW / 4)) == (warp >> 2);
-            const int gw = warp & 3;
-            const bool have = mine && have_stage;
-            if (have) {
-                const uint8_t* chunk = gu_ring + size_t(st) * kLGuStage + size_t(in_st) * kLChunk;
-                const int gi = slice * (kGuSlice / kGroup) + gw;  // input group
-                uint4 qa, qb;
-                uint32_t sbw;
-                acc += group_dot(chunk, kGuSlice, gw, lane, xq + gi * 8, xsx[gi], xX[gi], &qa, &qb, &sbw);
-                const LEntry& en = s_ent[e];
-                if (en.wb) group_writeback(en.wb + size_t(ul) * kLChunk, kGuSlice, gw, lane, qa, qb, sbw);
-            }
-            __syncwarp();
-            // every warp leaves the stage after its last chunk
-            if ((in_st == kLChunksPerStage - 1 || slice == NSg - 1) && lane == 0) mbar_arrive(&empty_gu[st]);
-            const bool seg_end = (u + 1 == ub) || (u + 1 == key_u0 + NSg);
-            if (!seg_end) continue;
-            named_sync(1, kLNC);
-            red[warp * 32 + lane] = acc;
-            named_sync(1, kLNC);
-            acc = 0.f;
-            if (warp == 0) {
-                float tot = 0.f;
-                for (int w = 0; w < kLNW; ++w) tot += red[w * 32 + lane];
-                const bool whole = (seg_start == key_u0) && (u + 1 == key_u0 + NSg);
-                bool lastc = whole;
-                const int cidx = key_u0 / NSg;
-                if (!whole) {
-                    const int sl = (seg_start == ua) ? 0 : 1;
-                    A.partials_gu[size_t(4 * c + 2 * pool + sl) * 32 + lane] = tot;
-                    __threadfence();
-                    __syncwarp();
-                    int old = 0;
-                    if (lane == 0) old = atomicAdd(&A.counters_gu[cidx], u + 1 - seg_start);
-                    old = __shfl_sync(0xffffffffu, old, 0);
-                    lastc = (old + (u + 1 - seg_start) == NSg);
-                    if (lastc) {
-                        __threadfence();
-                        tot = 0.f;
-                        const int kl = key_u0 - pb;  // the tile's first unit inside its pool
-                        const int c0 = cta_of(kl, PU, G), c1 = cta_of(kl + NSg - 1, PU, G);
-                        for (int cc = c0; cc <= c1; ++cc) {
-                            const int rs = range_start(cc, PU, G);
-                            if (rs >= range_start(cc + 1, PU, G)) continue;
-                            tot += __ldcg(A.partials_gu + size_t(4 * cc + 2 * pool + (rs >= kl ? 0 : 1)) * 32 + lane);
-                        }
-                        if (lane == 0) A.counters_gu[cidx] = 0;
+    // Whole tiles (NSg chunks, 16 gate + 16 up rows) stage by stage: a stage
+    // holds up to kLChunksPerStage chunks (4 groups of 64 inputs each) and
+    // warp w takes the stage's groups w, w + 12, ...: one wait and one release
+    // per stage and warp.  At a tile's end the warps' partial sums (lane = row)
+    // are added in warp order by one warp (double-buffered by tile parity, so
+    // one barrier per tile suffices) and h = gelu(gate) * up is written.
+    int tiles_done = 0;
+    int q_gu = 0;  // ring position of the next gate/up stage
+    auto gu_tiles = [&](int ua, int ub) {
+        for (int t0 = ua; t0 < ub; t0 += NSg) {
+            const int e = gu_entry(t0);
+            const int ul0 = t0 - gu_base(e);  // the tile's first chunk inside its blob
+            const int tile = ul0 / NSg;
+            const LEntry& en = s_ent[e];
+            float a = 0.f;
+            for (int c0 = 0; c0 < NSg; c0 += kLChunksPerStage, ++q_gu) {
+                const int nc = min(kLChunksPerStage, NSg - c0);
+                const int st = q_gu % kLGuStages;
+                const bool have = lwait(&full_gu[st], uint32_t(q_gu / kLGuStages) & 1u, A.status, &s_abort);
+                if (have) {
+                    const uint8_t* stage = gu_ring + size_t(st) * kLGuStage;
+                    for (int g = warp; g < 4 * nc; g += kLNW) {
+                        const int ch = g >> 2, gw = g & 3;
+                        const int gi = 4 * c0 + g;  // input group: chunk c0 + ch, group gw
+                        uint4 qa, qb;
+                        uint32_t sbw;
+                        a += group_dot(stage + size_t(ch) * kLChunk, kGuSlice, gw, lane, xq + gi * 8, xsx[gi], xX[gi],
+                                       &qa, &qb, &sbw);
+                        if (en.wb) group_writeback(en.wb + size_t(ul0 + c0 + ch) * kLChunk, kGuSlice, gw, lane, qa, qb, sbw);
                     }
                 }
-                if (lastc) {
-                    // lanes 0..15 gate rows, 16..31 up rows of outputs 16*tile + lane
-                    const float upv = __shfl_down_sync(0xffffffffu, tot, 16);
-                    if (lane < 16) A.h[s_ent[e].h_off + 16 * tile + lane] = gelu_tanh(tot) * upv;
-                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty_gu[st]);
             }
-            seg_start = u + 1;
+            const int tb = tiles_done & 1;
+            red2[tb][warp * 32 + lane] = a;
+            named_sync(1, kLNC);
+            if (warp == tiles_done % kLNW) {
+                float tot = 0.f;
+                for (int w = 0; w < kLNW; ++w) tot += red2[tb][w * 32 + lane];
+                // lanes 0..15 gate rows, 16..31 up rows of outputs 16*tile + lane
+                const float upv = __shfl_down_sync(0xffffffffu, tot, 16);
+                if (lane < 16) A.h[en.h_off + 16 * tile + lane] = gelu_tanh(tot) * upv;
+            }
+            ++tiles_done;
         }
     };
-    gu_units(sh0, sh1, 0, 0, ush, 0);  // shared-expert chunks (known before the plan)
+    gu_tiles(sh0, sh1);  // shared-expert tiles (known before the plan)
 
     // ------------------------------------------------- phase 2: top-K + plan
     bool ok_a = true;
@@ -821,7 +792,7 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_decode_kernel(LayerArgs A)
     named_sync(1, kLNC);
 
     // ------------------------------------------- the routed gate/up chunks
-    gu_units(r0, r1, 1, ush, Urt, ((sh1 - sh0) / NSg) * SPT);
+    gu_tiles(r0, r1);
 
     // ------------------------------------------------ phase 3: down + combine
     named_sync(1, kLNC);
@@ -876,8 +847,8 @@ __global__ void __launch_bounds__(kLThreads, 1) layer_decode_kernel(LayerArgs A)
         }
         named_sync(1, kLNC);
     }
-    acc = 0.f;
-    seg_start = d0;
+    float acc = 0.f;
+    int seg_start = d0;
     for (int u = d0; u < d1; ++u) {
         const int i = u - d0, st = i % kLDnStages;
         int e, tile, slice;
