@@ -125,7 +125,7 @@ struct moe_ctx {
     int layer_hvals = 0;
     float* layer_logits = nullptr;
     float* layer_partials = nullptr;  // [6 * G][32]: gate/up (two pools) then down
-    unsigned* layer_bar = nullptr;    // [4]
+    unsigned* layer_bar = nullptr;    // [128]
     uint64_t* stats = nullptr;        // [MOE_STATS] device counters
     std::unordered_map<const void*, const uint8_t*> direct_store;  // host store -> device-accessible address
     // instrumentation (moe_ctx_profile)
@@ -633,7 +633,7 @@ int moe_ctx_create(const moe_dims* dims, int device, moe_ctx** out) {
     }
     ok = ok && dalloc(&c->layer_logits, size_t(d.n_experts)) == cudaSuccess;
     ok = ok && dalloc(&c->layer_partials, size_t(6) * c->layer_G * 32) == cudaSuccess;
-    ok = ok && dalloc(&c->layer_bar, 4) == cudaSuccess;
+    ok = ok && dalloc(&c->layer_bar, 128) == cudaSuccess;
     ok = ok && dalloc(&c->stats, MOE_STATS) == cudaSuccess;
     ok = ok && dalloc(&c->ready, size_t(d.n_slots)) == cudaSuccess;
     ok = ok && cudaMemset(c->ready, 0, size_t(d.n_slots) * sizeof(uint32_t)) == cudaSuccess;
@@ -650,7 +650,7 @@ int moe_ctx_create(const moe_dims* dims, int device, moe_ctx** out) {
         if (const char* v = std::getenv("MOE_PER_MISS")) c->per_miss = v[0] == '1';
         if (const char* v = std::getenv("MOE_INJECT_SKIP_READY")) c->inject_skip_ready = v[0] == '1';
     }
-    ok = ok && cudaMemset(c->layer_bar, 0, 4 * sizeof(unsigned)) == cudaSuccess;
+    ok = ok && cudaMemset(c->layer_bar, 0, 128 * sizeof(unsigned)) == cudaSuccess;
     ok = ok && cudaMemset(c->stats, 0, MOE_STATS * sizeof(uint64_t)) == cudaSuccess;
     ok = ok && cudaMemset(c->status, 0, sizeof(int)) == cudaSuccess;
     ok = ok && cudaMemset(c->counters_gu, 0, tiles_gu * sizeof(int)) == cudaSuccess;

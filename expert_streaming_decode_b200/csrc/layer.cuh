@@ -42,7 +42,7 @@ struct LayerArgs {
     int* counters_gu;            // [FS/16 + K*F/16], zero between launches
     float* partials_dn;          // [2*G][32]
     int* counters_dn;            // [D/32], zero between launches
-    unsigned* bar;               // [4], zero-initialised
+    unsigned* bar;               // [128], zero-initialised (two grid barriers, counter and generation lines apart)
     int* status;
 };
 
