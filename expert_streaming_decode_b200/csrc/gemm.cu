@@ -122,16 +122,23 @@ constexpr int kAhead = 4;  // groups whose activations are in flight (registers)
 // the order in which two nibbles at a time come out of a 32-bit word below.
 
 // 8 weights w = s*q + b of one 32-bit word (nibble i = input i) as fp16, in the
-// block order above.  A nibble placed in the low mantissa bits of the binary16
-// 1024.0 (0x6400) reads as 1024 + q exactly; subtracting 1024 is exact; the
-// fused multiply-add rounds s*q + b once.
+// block order above.  A 4-bit field placed in a binary16 mantissa reads as an
+// exact integer offset from a power of two: in the low bits of 1024.0
+// (0x6400, unit 1) as 1024 + q, and in bits 4..7 of 64.0 (0x5400, unit 1/16)
+// as 64 + q.  So nibbles i and i+4 (bits 4i and 16+4i) come out of the word
+// with one logic operation each for i = 0, 1, and of the word shifted by 8 for
+// i = 2, 3; subtracting the power of two is exact, and the fused multiply-add
+// rounds s*q + b once.
 __device__ __forceinline__ uint4 dequant_word(uint32_t w, uint32_t s2, uint32_t b2) {
+    const uint32_t w8 = w >> 8;
+    const uint32_t m[4] = {(w & 0x000F000Fu) | 0x64006400u, (w & 0x00F000F0u) | 0x54005400u,
+                           (w8 & 0x000F000Fu) | 0x64006400u, (w8 & 0x00F000F0u) | 0x54005400u};
+    const uint32_t base[4] = {0x64006400u, 0x54005400u, 0x64006400u, 0x54005400u};
     uint32_t r[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const uint32_t m = ((w >> (4 * i)) & 0x000F000Fu) | 0x64006400u;  // nibbles i and i+4
         uint32_t q;
-        asm("sub.f16x2 %0, %1, %2;" : "=r"(q) : "r"(m), "r"(0x64006400u));
+        asm("sub.f16x2 %0, %1, %2;" : "=r"(q) : "r"(m[i]), "r"(base[i]));
         asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r[i]) : "r"(q), "r"(s2), "r"(b2));
     }
     return make_uint4(r[0], r[1], r[2], r[3]);
