@@ -64,6 +64,9 @@ def parse_args():
                    help="streamed workloads with the pinned store: how one-token misses reach their slots -- "
                         "'copy': the host reads the plan and the copy engine copies them (default); "
                         "'direct': the one-launch layer kernel reads them from pinned host memory as it computes")
+    p.add_argument("--lookahead", type=int, default=1, choices=[1, 2],
+                   help="layers ahead the look-ahead may stage for: 2 = also the layer after next when the next "
+                        "layer is predicted to miss nothing (measured: no gain, 178.6 vs 180.8 tokens/s)")
     p.add_argument("--prefetch", type=int, default=None, metavar="P",
                    help="decode_stream with --fill copy: stage up to P of the next layer's predicted misses "
                         "(look-ahead; 0 = off; default 1 for the one-token streamed decode from the pinned store)")
@@ -388,8 +391,13 @@ class Model:
             if getattr(args, "prefetch", 0) > 0:
                 # layer l stages layer l+1's predicted misses; the last layer has
                 # no successor within the token
+                # (and, with --lookahead 2, layer l+2's when layer l+1 is
+                # predicted to miss nothing)
                 moe.prefetch_configure(self.ctx, args.prefetch)
-                self.nexts = [moe.next_layer(self.W[l + 1], self.caches[l + 1], self.bias[l + 1])
+                deep = getattr(args, "lookahead", 1) >= 2
+                after = [moe.next_layer(self.W[l + 2], self.caches[l + 2], self.bias[l + 2])
+                         if deep and l + 2 < self.L else None for l in range(self.L)]
+                self.nexts = [moe.next_layer(self.W[l + 1], self.caches[l + 1], self.bias[l + 1], after=after[l])
                               for l in range(self.L - 1)] + [None]
         else:
             self.nexts = None
@@ -1115,6 +1123,7 @@ def main():
            "miss_fill": (("layer kernel reads pinned host memory" if args.fill == "direct" and T == 1
                           else "copy engine") if streaming and not args.store_file else None),
            "prefetch_buffers": args.prefetch if streaming else None,
+           "lookahead_layers": (args.lookahead if args.prefetch else None) if streaming else None,
            "store": (("file, O_DIRECT" if args.direct else "file, page cache") if args.store_file else "pinned host memory")
            if streaming else None,
            "zipf_s": args.zipf, "zipf_lambda": args.zipf_lambda if args.zipf > 0 else None,

@@ -922,6 +922,13 @@ static int layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache*
     // stream, while this layer runs (one token, host stores, buffers configured)
     const bool prefetch = next && T == 1 && c->pf_n > 0 && next->W && next->W->router_q && next->W->router_s &&
                           next->cache && next->cache->source == MOE_SOURCE_HOST && next->cache->store;
+    // the layer after next, staged for only when next has nothing to stage
+    const moe_next_layer* after = prefetch && next->after && next->after->W && next->after->W->router_q &&
+                                          next->after->W->router_s && next->after->cache &&
+                                          next->after->cache->source == MOE_SOURCE_HOST && next->after->cache->store &&
+                                          next->after->cache->state != next->cache->state
+                                      ? next->after
+                                      : nullptr;
     // the one-launch layer kernel: always for direct-fill caches (the kernel
     // reads the misses), for resident experts when asked (MOE_LAYER_KERNEL=1;
     // the separate router / GEMV kernels are faster there today)
@@ -943,10 +950,16 @@ static int layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache*
     if (prefetch) {
         if (cudaEventRecord(c->ev_x, s) != cudaSuccess || cudaStreamWaitEvent(c->pf_stream, c->ev_x, 0) != cudaSuccess)
             return MOE_ERR_CUDA;
-        const cudaError_t pe = launch_router(x, next->W->router_q, next->W->router_s, next->bias, c->d.n_experts,
-                                             c->d.d_model, K, 1, c->pf_ids_dev, c->pf_gw, c->status, DecodeWLTarget{},
-                                             false, c->pf_stream);
+        cudaError_t pe = launch_router(x, next->W->router_q, next->W->router_s, next->bias, c->d.n_experts,
+                                       c->d.d_model, K, 1, c->pf_ids_dev, c->pf_gw, c->status, DecodeWLTarget{},
+                                       false, c->pf_stream);
         c->launches += 1;
+        if (pe == cudaSuccess && after) {
+            pe = launch_router(x, after->W->router_q, after->W->router_s, after->bias, c->d.n_experts, c->d.d_model,
+                               K, 1, c->pf_ids_dev + K, c->pf_gw + K, c->status, DecodeWLTarget{}, false,
+                               c->pf_stream);
+            c->launches += 1;
+        }
         if (pe != cudaSuccess || cudaEventRecord(c->ev_pred, c->pf_stream) != cudaSuccess) return MOE_ERR_CUDA;
     }
     r = moe_router_topk(c, x, W->router_q, W->router_s, bias, T, id, gw, s);
@@ -1072,22 +1085,60 @@ static int layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache*
         if (launch_f32_to_bf16(y, y_bf16, size_t(T) * c->d.d_model, c->pdl, s) != cudaSuccess) return MOE_ERR_CUDA;
     }
     if (prefetch) {
-        // the next layer's predicted experts its cache does not hold, in
-        // logit order, after this layer's own copies on the side stream; the
-        // blobs the buffers held before are no longer wanted
+        // The next layer's predicted experts its cache does not hold, in logit
+        // order, after this layer's own copies on the side stream.  Blobs
+        // staged for this layer are used or stale now, and blobs for layers
+        // other than the next two are not wanted; blobs staged earlier for the
+        // next layer (as its "after") stay.  When nothing of the next layer is
+        // worth staging, a free buffer takes the top predicted miss of the
+        // layer after it.
         if (cudaEventSynchronize(c->ev_pred) != cudaSuccess) return MOE_ERR_CUDA;
-        c->pf_table.clear();
-        const auto& m = mirror_of(c, next->cache->state);
-        for (int k = 0; k < K && int(c->pf_table.size()) < c->pf_n; ++k) {
-            const int e = c->pf_ids_host[k];
-            if (e < 0 || e >= c->d.n_experts || m[size_t(e)] >= 0) continue;
-            const int b = int(c->pf_table.size());
-            if (cudaMemcpyAsync(c->pf_buf + size_t(b) * c->pf_stride,
-                                next->cache->store + size_t(e) * next->cache->store_stride, c->blob_routed,
-                                cudaMemcpyHostToDevice, c->side) != cudaSuccess)
-                return MOE_ERR_CUDA;
-            c->pf_table.push_back({next->cache->state, next->cache->store, e, b});
-            c->pf_issued += c->blob_routed;
+        const int32_t* keep_a = next->cache->state;
+        const int32_t* keep_b = after ? after->cache->state : nullptr;
+        for (size_t i = 0; i < c->pf_table.size();)
+            if (c->pf_table[i].state != keep_a && (!keep_b || c->pf_table[i].state != keep_b))
+                c->pf_table.erase(c->pf_table.begin() + long(i));
+            else
+                ++i;
+        auto staged = [&](const int32_t* state, int e) {
+            for (const auto& f : c->pf_table)
+                if (f.state == state && f.expert == e) return true;
+            return false;
+        };
+        auto free_buf = [&]() {
+            for (int b = 0; b < c->pf_n; ++b) {
+                bool used = false;
+                for (const auto& f : c->pf_table) used = used || f.buf == b;
+                if (!used) return b;
+            }
+            return -1;
+        };
+        // stage up to `limit` predicted misses of layer L (ids at pred); returns
+        // how many of its predicted misses are missing from its cache and the buffers
+        auto stage = [&](const moe_next_layer* L, const int32_t* pred, int limit, int* n_stage) -> int {
+            const auto& m = mirror_of(c, L->cache->state);
+            int wanted = 0;
+            for (int k = 0; k < K; ++k) {
+                const int e = pred[k];
+                if (e < 0 || e >= c->d.n_experts || m[size_t(e)] >= 0 || staged(L->cache->state, e)) continue;
+                ++wanted;
+                const int b = *n_stage < limit ? free_buf() : -1;
+                if (b < 0) continue;
+                if (cudaMemcpyAsync(c->pf_buf + size_t(b) * c->pf_stride, L->cache->store + size_t(e) * L->cache->store_stride,
+                                    c->blob_routed, cudaMemcpyHostToDevice, c->side) != cudaSuccess)
+                    return -1;
+                c->pf_table.push_back({L->cache->state, L->cache->store, e, b});
+                c->pf_issued += c->blob_routed;
+                ++*n_stage;
+            }
+            return wanted;
+        };
+        int n_stage = 0;
+        const int wanted = stage(next, c->pf_ids_host, c->pf_n, &n_stage);
+        if (wanted < 0) return MOE_ERR_CUDA;
+        if (wanted == 0 && after) {
+            int n2 = 0;
+            if (stage(after, c->pf_ids_host + K, 1, &n2) < 0) return MOE_ERR_CUDA;
         }
     }
     copy_trace(c->mbox_host, trace, c->blob_routed, bytes);
@@ -1128,10 +1179,11 @@ int moe_prefetch_configure(moe_ctx* c, int n_buffers) {
         ok = ok && cudaStreamCreateWithFlags(&c->pf_stream, cudaStreamNonBlocking) == cudaSuccess;
         ok = ok && cudaEventCreateWithFlags(&c->ev_x, cudaEventDisableTiming) == cudaSuccess;
         ok = ok && cudaEventCreateWithFlags(&c->ev_pred, cudaEventDisableTiming) == cudaSuccess;
-        ok = ok && cudaHostAlloc(reinterpret_cast<void**>(&c->pf_ids_host), sizeof(int32_t) * size_t(c->d.top_k),
+        // the predicted ids of the next layer, then of the layer after it
+        ok = ok && cudaHostAlloc(reinterpret_cast<void**>(&c->pf_ids_host), sizeof(int32_t) * size_t(2 * c->d.top_k),
                                  cudaHostAllocMapped) == cudaSuccess;
         ok = ok && cudaHostGetDevicePointer(reinterpret_cast<void**>(&c->pf_ids_dev), c->pf_ids_host, 0) == cudaSuccess;
-        ok = ok && dalloc(&c->pf_gw, size_t(c->d.top_k)) == cudaSuccess;
+        ok = ok && dalloc(&c->pf_gw, size_t(2 * c->d.top_k)) == cudaSuccess;
     }
     c->pf_stride = (c->blob_routed + 255) / 256 * 256;
     ok = ok && cudaMalloc(reinterpret_cast<void**>(&c->pf_buf), c->pf_stride * size_t(n_buffers)) == cudaSuccess;

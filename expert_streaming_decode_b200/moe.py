@@ -59,7 +59,11 @@ _I32P = C.POINTER(C.c_int32)
 
 
 class moe_next_layer(C.Structure):
-    _fields_ = [("W", C.POINTER(moe_layer_weights)), ("cache", C.POINTER(moe_slot_cache)), ("bias", C.c_void_p)]
+    pass
+
+
+moe_next_layer._fields_ = [("W", C.POINTER(moe_layer_weights)), ("cache", C.POINTER(moe_slot_cache)),
+                           ("bias", C.c_void_p), ("after", C.POINTER(moe_next_layer))]
 
 
 class moe_plan_trace(C.Structure):
@@ -300,11 +304,11 @@ def layer_forward(ctx: Ctx, W: moe_layer_weights, cache: moe_slot_cache | None, 
            "moe_layer_forward")
 
 
-def next_layer(W: moe_layer_weights, cache: moe_slot_cache, bias=None):
+def next_layer(W: moe_layer_weights, cache: moe_slot_cache, bias=None, after: "moe_next_layer | None" = None):
     """The layer after the one being run, for moe_layer_forward_next (keeps its
-    structures alive with it)."""
-    n = moe_next_layer(C.pointer(W), C.pointer(cache), _ptr(bias))
-    n._keep = (W, cache, bias)
+    structures alive with it); `after` is the layer after that, or None."""
+    n = moe_next_layer(C.pointer(W), C.pointer(cache), _ptr(bias), C.pointer(after) if after is not None else None)
+    n._keep = (W, cache, bias, after)
     return n
 
 

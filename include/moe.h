@@ -335,11 +335,17 @@ typedef struct moe_layer_weights {
  * cache == NULL: resident mode, expert e read from W->experts + e*stride.
  * cache != NULL: experts are served from cache->slots; misses are copied from
  * cache->store (host-synchronous on the plan, see moe_cache_plan).
- * T = 1 with resident experts or a MOE_SOURCE_HOST_DIRECT cache runs the
- * whole layer as one cooperative kernel (router, top-K, plan, shared and
- * routed expert GEMVs, combine; all CTAs resident, two bounded grid-wide
- * barriers; the plan reaches the host only when a trace is requested); other
- * one-token calls run the router, plan and dequantising GEMV kernels;
+ * T = 1 with a MOE_SOURCE_HOST_DIRECT cache runs the whole layer as one
+ * cooperative kernel (router, top-K, plan, shared and routed expert GEMVs,
+ * combine; all CTAs resident, two bounded grid-wide barriers; the plan reaches
+ * the host only when a trace is requested); so does T = 1 with resident
+ * experts when the environment sets MOE_LAYER_KERNEL=1 (MOE_LAYER_KERNEL=0
+ * never uses it).  Other one-token calls run the router, plan and dequantising
+ * GEMV kernels; with a MOE_SOURCE_HOST cache the routed experts' kernels wait
+ * for all of the call's copies through one event, or, when the environment
+ * sets MOE_PER_MISS=1 at context creation, start at once and wait per expert
+ * for a completion word written after that expert's copy (bounded:
+ * MOE_ERR_TIMEOUT);
  * T >= moe_gemm_min_tokens() (a batched decode step or a prefill chunk) groups
  * the tokens by expert and runs the tcgen05 tensor-core grouped GEMM, one wave
  * of at most n_slots experts at a time.
@@ -391,13 +397,19 @@ typedef struct moe_next_layer {
     const moe_layer_weights *W;
     moe_slot_cache *cache;
     const float *bias;
+    /* the layer after this one, or NULL: when none of this layer's predicted
+     * experts is missing from its cache (nothing to stage for it), a free
+     * buffer stages the top predicted miss of `after` instead (its router is
+     * also evaluated on the current input); after->after is ignored */
+    const struct moe_next_layer *after;
 } moe_next_layer;
 
 /* moe_layer_forward, plus the look-ahead prefetch of `next` when T = 1, buffers
  * are configured and next->cache has a host store; otherwise (next NULL or any
  * of these missing) exactly moe_layer_forward.  The staged blobs are matched to
- * a later miss by (cache state, store, expert); a later call that issues new
- * prefetches drops the old ones.  The host waits for the prediction router
+ * a later miss by (cache state, store, expert); a blob is kept until the
+ * layer it was staged for has run (or its cache is reset), and blobs for any
+ * layer other than next and next->after are dropped.  The host waits for the prediction router
  * (issued before this layer's own router) after queueing this layer's copies.
  * Errors: those of moe_layer_forward, and next->cache is checked as any cache. */
 int moe_layer_forward_next(moe_ctx *ctx, const moe_layer_weights *W, moe_slot_cache *cache,

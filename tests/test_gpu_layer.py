@@ -74,7 +74,7 @@ def test_batched_decode_resident(O, d, T):
 
 
 def _streaming(O, d, layers, tokens, S, check_y_every=1, T=1, policy=0, period=0, file_dir=None, prefetch=0,
-               same_x=False, stats=None, direct=False, counters=None):
+               same_x=False, stats=None, direct=False, counters=None, deep=False):
     Ls = [Layer(d, layer=l, seed=1, zipf_s=1.1, resident=False, pinned=True) for l in range(layers)]
     ctx = moe.Ctx.from_dims(d, max_tokens=T, S=S)
     caches, states, slotbufs = [], [], []
@@ -112,7 +112,10 @@ def _streaming(O, d, layers, tokens, S, check_y_every=1, T=1, policy=0, period=0
     ctx.stats_reset()
     if prefetch:
         moe.prefetch_configure(ctx, prefetch)
-        nexts = [moe.next_layer(Ls[l + 1].weights(resident=False), caches[l + 1], Ls[l + 1].bias_t)
+        # deep: layer l may also stage for layer l+2 when layer l+1 has nothing to stage
+        after = [moe.next_layer(Ls[l + 2].weights(resident=False), caches[l + 2], Ls[l + 2].bias_t)
+                 if deep and l + 2 < layers else None for l in range(layers)]
+        nexts = [moe.next_layer(Ls[l + 1].weights(resident=False), caches[l + 1], Ls[l + 1].bias_t, after=after[l])
                  for l in range(layers - 1)] + [None]
         later_misses = 0  # misses of layers 1.. (the ones a prefetch can serve)
     for step in range(tokens):
@@ -252,6 +255,19 @@ def test_streaming_decode_lookahead_exact(O, d, layers, tokens, S, every):
     _streaming(O, d, layers=layers, tokens=tokens, S=S, check_y_every=every, prefetch=d.K, same_x=True, stats=st)
     assert st["later_misses"] > 0
     assert st["issued"] == st["used"] == st["later_misses"] * st["nb"]
+
+
+@pytest.mark.parametrize("d,layers,tokens,S,every", [(TINY, 4, 40, 6, 1), (FULL, 4, 10, 16, 3)], ids=["tiny", "full"])
+def test_streaming_decode_lookahead_two_layers(O, d, layers, tokens, S, every):
+    """One look-ahead buffer that may stage for the layer after next when the
+    next layer is predicted to miss nothing (exact predictions: one input per
+    token for every layer).  Traces, slots and outputs are the oracle's; every
+    staged blob is used."""
+    st = {}
+    _streaming(O, d, layers=layers, tokens=tokens, S=S, check_y_every=every, prefetch=1, same_x=True, stats=st,
+               deep=True)
+    assert st["later_misses"] > 0 and st["issued"] > 0
+    assert st["used"] == st["issued"]
 
 
 def test_streaming_decode_lookahead_mispredicted(O):
