@@ -1177,8 +1177,9 @@ def main():
         tf = flop_layer * n_layer_tok / (gemm_ms * 1e-3) / 1e12
         pk = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["bf16_tflops"] if peak_kind == "measured" else 1590.0
         line["tensor"] = {"achieved_tflops": tf, "peak_tflops": pk, "frac": tf / pk,
-                          "note": "fp16 tcgen05 MMAs (peak: measured bf16 dense, same rate as fp16); "
-                                  "per-expert rows average ~11, so the GEMM is weight-bandwidth bound"}
+                          "note": "fp16 tcgen05 MMAs (peak: bf16 dense, same rate as fp16); per-expert rows "
+                                  f"average {T * dims.K / distinct:.1f} ({T} tokens over ~{distinct:.0f} experts), so "
+                                  "the tensor pipe idles: the GEMM is bound by the weights' dequantisation and bytes"}
     line["kernels"] = kern
     line["kernels_note"] = (f"per-kernel times from a separate pass of {kp} steps with an event pair around every "
                             "kernel (serialised: no overlap between kernels)")
