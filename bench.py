@@ -388,6 +388,7 @@ class Model:
                                for l in range(self.L)]
             self.W = [moe.layer_weights(self.wq[l], self.ws[l], self.shared[l]) for l in range(self.L)]
             self.nexts = None
+            self.lookahead = bool(getattr(args, "prefetch", 0))
             if getattr(args, "prefetch", 0) > 0:
                 # layer l stages layer l+1's predicted misses; the last layer has
                 # no successor within the token
@@ -400,12 +401,13 @@ class Model:
                 self.nexts = [moe.next_layer(self.W[l + 1], self.caches[l + 1], self.bias[l + 1], after=after[l])
                               for l in range(self.L - 1)] + [None]
         else:
-            self.nexts = None
+            self.lookahead = False
             self.experts = store.to(dev)
             del store
             self.caches = [None] * self.L
             self.W = [moe.layer_weights(self.wq[l], self.ws[l], self.shared[l], self.experts[l], self.stride)
                       for l in range(self.L)]
+            self.nexts = None
 
     def close_files(self):
         """Closes and deletes the expert files this run wrote (--store-file)."""
@@ -436,7 +438,7 @@ class Model:
 
 def moe_prefetch_stats(model):
     """(issued, used) look-ahead bytes so far; zeros when prefetch is off."""
-    return model.moe.prefetch_stats(model.ctx) if model.nexts is not None else (0, 0)
+    return model.moe.prefetch_stats(model.ctx) if model.lookahead else (0, 0)
 
 
 def decode_token(model, x0, r, x, y, T, tok, tr=None, trace_acc=None, on_layer=None, ids=None, gate_w=None):
@@ -1231,7 +1233,7 @@ def main():
                                                 "4 threads" + (", O_DIRECT" if args.direct else ", page cache"),
                                  "note": "misses are read from the expert files (positional reads into pinned "
                                          "staging, 4 in flight) and then copied"}
-        if model.nexts is not None:
+        if model.lookahead:
             line["prefetch"] = {"buffers": args.prefetch, "issued_bytes_per_token": pf_iss / (K * T),
                                 "used_bytes_per_token": pf_used / (K * T),
                                 "wasted_bytes_per_token": (pf_iss - pf_used) / (K * T),
@@ -1251,7 +1253,7 @@ def main():
         ms2, _ = timed(dist, model, lambda: runner.run(None, K, W, host_io=(xh, yh)))
         line["e2e"] = {"value": dist.sum(K * T) / (ms2 * 1e-3), "unit": "tokens/s",
                        "h2d_bytes_per_step": T * dims.D * 2, "d2h_bytes_per_step": T * dims.D * 4,
-                       "api": ("moe_layer_forward_next" if model.nexts is not None else "moe_layer_forward")
+                       "api": ("moe_layer_forward_next" if model.nexts is not None and T == 1 else "moe_layer_forward")
                               + f" x {args.layers} per step, input bf16 copied from pinned host, output fp32 copied back"}
 
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu and not args.profile and args.workload == "decode_stream":

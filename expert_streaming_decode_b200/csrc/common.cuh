@@ -96,7 +96,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
 // ------------------------------------------------------- 1-D bulk copies
 // Global -> shared bulk copy on the TMA engine, completion counted on `bar`
 // (complete_tx).  Source and destination 16-byte aligned, bytes % 16 == 0.
-// No multicast: the copy lands in this CTA's shared memory only.
+// The copy lands in this CTA's own shared memory only.
 __device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar,
                                          uint64_t policy) {
     asm volatile(

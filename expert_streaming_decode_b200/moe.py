@@ -304,18 +304,21 @@ def layer_forward(ctx: Ctx, W: moe_layer_weights, cache: moe_slot_cache | None, 
            "moe_layer_forward")
 
 
-def next_layer(W: moe_layer_weights, cache: moe_slot_cache, bias=None, after: "moe_next_layer | None" = None):
+def next_layer(W: moe_layer_weights, cache: "moe_slot_cache | None", bias=None, after: "moe_next_layer | None" = None):
     """The layer after the one being run, for moe_layer_forward_next (keeps its
-    structures alive with it); `after` is the layer after that, or None."""
-    n = moe_next_layer(C.pointer(W), C.pointer(cache), _ptr(bias), C.pointer(after) if after is not None else None)
+    structures alive with it); `after` is the layer after that, or None.  A
+    next layer without a cache (resident experts) stages nothing."""
+    n = moe_next_layer(C.pointer(W), C.pointer(cache) if cache is not None else None, _ptr(bias),
+                       C.pointer(after) if after is not None else None)
     n._keep = (W, cache, bias, after)
     return n
 
 
-def layer_forward_next(ctx: Ctx, W: moe_layer_weights, cache: moe_slot_cache, x, T, step, bias, y,
+def layer_forward_next(ctx: Ctx, W: moe_layer_weights, cache: "moe_slot_cache | None", x, T, step, bias, y,
                        next: moe_next_layer | None, y_bf16=None, ids=None, gate_w=None, trace: Trace | None = None,
                        stream=None):
-    _check(lib.moe_layer_forward_next(ctx.h, C.byref(W), C.byref(cache), _ptr(x), T, step, _ptr(bias), _ptr(y),
+    _check(lib.moe_layer_forward_next(ctx.h, C.byref(W), None if cache is None else C.byref(cache), _ptr(x), T, step,
+                                      _ptr(bias), _ptr(y),
                                       _ptr(y_bf16), _ptr(ids), _ptr(gate_w),
                                       None if trace is None else C.byref(trace.c),
                                       None if next is None else C.byref(next), _stream(stream)),

@@ -55,6 +55,32 @@ def test_decode_resident_single_layer(O, d, kernel, monkeypatch):
         _check_token(O, L, xb, ids.cpu().numpy()[0], gw.cpu().numpy()[0], y.cpu().numpy()[0])
 
 
+@pytest.mark.parametrize("kernel", ["layer", "split"])
+@pytest.mark.parametrize("d", [TINY, FULL], ids=["tiny", "full"])
+def test_decode_resident_with_next_layer(O, d, kernel, monkeypatch):
+    """Two resident layers, the first called with the next layer named
+    (moe_layer_forward_next, no cache: nothing to stage, exactly
+    moe_layer_forward): results are the oracle's through either kernel path."""
+    monkeypatch.setenv("MOE_LAYER_KERNEL", "1" if kernel == "layer" else "0")
+    Ls = [Layer(d, layer=l, seed=4, zipf_s=None) for l in range(2)]
+    ctx = moe.Ctx.from_dims(d, max_tokens=1)
+    Ws = [L.weights() for L in Ls]
+    nxt = moe.next_layer(Ws[1], None, Ls[1].bias_t)
+    y = torch.empty((1, d.D), dtype=torch.float32, device="cuda")
+    ids = torch.empty((1, d.K), dtype=torch.int32, device="cuda")
+    gw = torch.empty((1, d.K), dtype=torch.float32, device="cuda")
+    for t in range(6):
+        for l, L in enumerate(Ls):
+            xb = synth.hidden(4, t, l, d.D)
+            if l == 0:
+                moe.layer_forward_next(ctx, Ws[0], None, bf16_tensor(xb[None]), 1, t, None, y, nxt, ids=ids,
+                                       gate_w=gw)
+            else:
+                moe.layer_forward(ctx, Ws[1], None, bf16_tensor(xb[None]), 1, t, None, y, ids=ids, gate_w=gw)
+            ctx.sync()
+            _check_token(O, L, xb, ids.cpu().numpy()[0], gw.cpu().numpy()[0], y.cpu().numpy()[0])
+
+
 @pytest.mark.parametrize("d,T", [(TINY, 8), (FULL, 8), (FULL, 32)], ids=["tiny-8", "full-8", "full-32"])
 def test_batched_decode_resident(O, d, T):
     L = Layer(d, layer=1, seed=2, zipf_s=None)
