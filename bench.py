@@ -275,7 +275,12 @@ class HostStore:
                                f"{avail / 1e9:.2f} GB available")
         self._path = os.path.join(self.SHM_DIR, f"{tag}_{os.environ.get('MASTER_PORT', '0')}")
         if dist.local == 0:
-            fd = os.open(self._path, os.O_CREAT | os.O_EXCL | os.O_RDWR, 0o600)
+            try:
+                fd = os.open(self._path, os.O_CREAT | os.O_EXCL | os.O_RDWR, 0o600)
+            except FileExistsError:
+                # left behind by an earlier run on this port that did not finish
+                os.unlink(self._path)
+                fd = os.open(self._path, os.O_CREAT | os.O_EXCL | os.O_RDWR, 0o600)
             try:
                 os.ftruncate(fd, self.nbytes)
                 self._mm = mmap.mmap(fd, self.nbytes)
