@@ -1084,6 +1084,11 @@ static int layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache*
         c->launches += 1;
         if (launch_f32_to_bf16(y, y_bf16, size_t(T) * c->d.d_model, c->pdl, s) != cudaSuccess) return MOE_ERR_CUDA;
     }
+    // this layer has run: the blobs staged for its cache were used or are
+    // stale (also when this call stages nothing, e.g. the last layer)
+    for (size_t i = 0; i < c->pf_table.size();)
+        if (c->pf_table[i].state == cache->state) c->pf_table.erase(c->pf_table.begin() + long(i));
+        else ++i;
     if (prefetch) {
         // The next layer's predicted experts its cache does not hold, in logit
         // order, after this layer's own copies on the side stream.  Blobs
