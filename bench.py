@@ -453,15 +453,16 @@ def decode_token(model, x0, r, x, y, T, tok, tr=None, trace_acc=None, on_layer=N
     use it to read each layer's input and output); ids / gate_w receive the
     layer's routing when given."""
     moe, d, ctx = model.moe, model.d, model.ctx
-    moe.bf16_to_f32(ctx, x0, r, T * d.D)
+    st = model.torch.cuda.current_stream()  # once per token: the library calls all go to it
+    moe.bf16_to_f32(ctx, x0, r, T * d.D, stream=st)
     cur = x0
     for l in range(model.L):
         if model.nexts is not None and T == 1:
             moe.layer_forward_next(ctx, model.W[l], model.caches[l], cur, T, tok, model.bias[l], y, model.nexts[l],
-                                   ids=ids, gate_w=gate_w, trace=tr)
+                                   ids=ids, gate_w=gate_w, trace=tr, stream=st)
         else:
             moe.layer_forward(ctx, model.W[l], model.caches[l], cur, T, tok, model.bias[l], y, ids=ids,
-                              gate_w=gate_w, trace=tr)
+                              gate_w=gate_w, trace=tr, stream=st)
         if tr is not None:
             res = tr.c
             trace_acc["misses"] += res.n_misses
@@ -480,7 +481,7 @@ def decode_token(model, x0, r, x, y, T, tok, tr=None, trace_acc=None, on_layer=N
         if on_layer is not None:
             on_layer(l, cur, y, r)
         if l + 1 < model.L:
-            moe.residual_rmsnorm(ctx, r, y, x, T)
+            moe.residual_rmsnorm(ctx, r, y, x, T, stream=st)
             cur = x
 
 
