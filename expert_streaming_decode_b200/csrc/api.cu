@@ -329,6 +329,7 @@ int run_gemm(moe_ctx* c, WorkListArgs wa, const uint16_t* x16, int T, float* y, 
     L.D = c->d.d_model;
     L.max_tiles_gu = (wa.K > 0 ? routed * (c->d.d_ff / 64) : 0) + shared * (c->d.d_ff_shared / 64);
     L.max_tiles_dn = ((wa.K > 0 ? routed : 0) + shared) * (c->d.d_model / 128);
+    L.row_cap = T;  // an entry carries one expert's rows: at most one per token
     L.status = c->status;
     L.pdl = c->pdl;
     if (L.max_tiles_gu <= 0 || L.max_tiles_dn <= 0) return MOE_OK;

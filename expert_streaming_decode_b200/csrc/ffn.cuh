@@ -75,6 +75,7 @@ struct GemmLaunch {
     int D;
     int max_tiles_gu;  // grid bounds (CTAs past the work list's tile count exit)
     int max_tiles_dn;
+    int row_cap = 0;   // most token rows any entry carries (the call's T, at most kGemmMaxRows); 0: kGemmMaxRows
     int* status;
     bool pdl = true;
 };

@@ -49,6 +49,7 @@ struct GemmArgs {
     float* h;            // activations
     float* y;            // [T][D], accumulated
     int D;
+    int b_bytes;         // bytes of one B (activation) tile buffer: the call's row cap (<= 64, a multiple of 16) x 128
     int* status;
 };
 
@@ -86,15 +87,18 @@ __device__ __forceinline__ bool ring_wait_gemm(uint64_t* bar, uint32_t parity, i
 // Ring layout: [NST stages][4 blob tiles][GPS KB nibbles | GPS x 128 B s,b].
 template <int MODE>
 struct GemmRing;
+#ifndef MOE_GEMM_GU_STAGES
+#define MOE_GEMM_GU_STAGES 3
+#endif
 template <>
 struct GemmRing<0> {  // gate/up: 4 groups per 256-input chunk, take 2 at a time
     static constexpr int kGroupsPerStage = 2;
-    static constexpr int kStages = 6;
+    static constexpr int kStages = MOE_GEMM_GU_STAGES;
 };
 template <>
 struct GemmRing<1> {  // down: chunk widths need not be even in groups
     static constexpr int kGroupsPerStage = 1;
-    static constexpr int kStages = 12;
+    static constexpr int kStages = 2 * MOE_GEMM_GU_STAGES;
 };
 template <int MODE>
 __host__ __device__ constexpr int ring_bt_bytes() { return GemmRing<MODE>::kGroupsPerStage * 1152; }
@@ -104,9 +108,12 @@ __host__ __device__ constexpr int ring_stage_bytes() { return 4 * ring_bt_bytes<
 constexpr int kOpBufs = 2;                          // fp16 operand buffer sets (A and B tiles of one group)
 constexpr int kABytes = 128 * 64 * 2;               // A: 128 weight rows x 64 inputs
 constexpr int kBBytes = kGemmMaxRows * 64 * 2;      // B: up to kGemmMaxRows token rows x 64 inputs
+// Shared memory of one CTA when the B buffers hold b_bytes each (sized by the
+// call's row cap, so that small batches fit three CTAs per SM).
 template <int MODE>
-constexpr size_t gemm_smem() {
-    return size_t(kOpBufs) * (kABytes + kBBytes) + size_t(GemmRing<MODE>::kStages) * ring_stage_bytes<MODE>() + 128;
+constexpr size_t gemm_smem(int b_bytes = kBBytes) {
+    return size_t(kOpBufs) * (kABytes + size_t(b_bytes)) + size_t(GemmRing<MODE>::kStages) * ring_stage_bytes<MODE>() +
+           128;
 }
 
 constexpr int kMathWarps = 8;               // thread = (weight row, half of the group's 64 inputs)
@@ -153,15 +160,15 @@ __device__ __forceinline__ uint4 dequant_word(uint32_t w, uint32_t s2, uint32_t 
 // a last commit on `done` releases the epilogue.  No CTA-wide barrier runs
 // per group.
 template <int MODE>
-__global__ void __launch_bounds__(kGemmWarps * 32, 2) grouped_gemm_kernel(GemmArgs A) {
+__global__ void __launch_bounds__(kGemmWarps * 32, 3) grouped_gemm_kernel(GemmArgs A) {
     constexpr int GPS = GemmRing<MODE>::kGroupsPerStage;
     constexpr int NST = GemmRing<MODE>::kStages;
     constexpr int BT_BYTES = ring_bt_bytes<MODE>();
     constexpr int ST_BYTES = ring_stage_bytes<MODE>();
     extern __shared__ __align__(128) uint8_t gsm[];
     uint8_t* sA = gsm;                                   // [kOpBufs][128 x 64 fp16]
-    uint8_t* sB = gsm + kOpBufs * kABytes;               // [kOpBufs][kGemmMaxRows x 64 fp16]
-    uint8_t* ring = sB + kOpBufs * kBBytes;              // [NST][ST_BYTES]
+    uint8_t* sB = gsm + kOpBufs * kABytes;               // [kOpBufs][b_bytes: row cap x 64 fp16]
+    uint8_t* ring = sB + kOpBufs * A.b_bytes;            // [NST][ST_BYTES]
     __shared__ __align__(8) uint64_t full[NST], empty[NST];
     __shared__ __align__(8) uint64_t ready[kOpBufs], freed[kOpBufs], done;
     __shared__ uint32_t tbase;
@@ -208,6 +215,10 @@ __global__ void __launch_bounds__(kGemmWarps * 32, 2) grouped_gemm_kernel(GemmAr
     const int tile = s_tile;
     const int M = min(en.n_rows, kGemmMaxRows);
     const int N = (M + 15) & ~15;
+    if (N * 128 > A.b_bytes) {  // more rows than the launch's B buffers hold: report, touch nothing
+        if (tid == 0) set_status(A.status, MOE_ERR_RANGE);
+        return;
+    }
     const int F = en.F;
     const int Kin = MODE == 0 ? D : F;
     const int ngroups = Kin / kGroup;
@@ -265,7 +276,7 @@ __global__ void __launch_bounds__(kGemmWarps * 32, 2) grouped_gemm_kernel(GemmAr
                 const int b = g % kOpBufs;
                 if (!ring_wait_gemm(&ready[b], (g / kOpBufs) & 1, A.status, &s_abort)) break;
                 asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-                const uint32_t a_addr = smem_u32(sA + b * kABytes), b_addr = smem_u32(sB + b * kBBytes);
+                const uint32_t a_addr = smem_u32(sA + b * kABytes), b_addr = smem_u32(sB + b * A.b_bytes);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                     const uint64_t ad = umma_desc(a_addr + kk * 256);
@@ -335,7 +346,7 @@ __global__ void __launch_bounds__(kGemmWarps * 32, 2) grouped_gemm_kernel(GemmAr
         if (g >= kOpBufs && !ring_wait_gemm(&freed[b], ((g / kOpBufs) - 1) & 1, A.status, &s_abort)) return false;
         if (gl == 0 && !ring_wait_gemm(&full[st], (si / NST) & 1, A.status, &s_abort)) return false;
         uint8_t* a = sA + b * kABytes;
-        uint8_t* bt = sB + b * kBBytes;
+        uint8_t* bt = sB + b * A.b_bytes;
 #pragma unroll
         for (int i = 0; i < kBTasks; ++i) {
             const int idx = tid + kMathThreads * i;
@@ -444,13 +455,15 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t s, void (*hook)(void*,
     a.y = L.y;
     a.D = L.D;
     a.status = L.status;
+    const int n_cap = L.row_cap < 1 ? kGemmMaxRows : (L.row_cap > kGemmMaxRows ? kGemmMaxRows : L.row_cap);
+    a.b_bytes = ((n_cap + 15) & ~15) * 128;
     if (hook) hook(hook_arg, 0);
     cudaError_t e = launch_kernel(grouped_gemm_kernel<0>, dim3(L.max_tiles_gu), dim3(kGemmWarps * 32),
-                                  gemm_smem<0>(), s, L.pdl, 1, a);
+                                  gemm_smem<0>(a.b_bytes), s, L.pdl, 1, a);
     if (e != cudaSuccess) return e;
     if (hook) hook(hook_arg, 1);
-    e = launch_kernel(grouped_gemm_kernel<1>, dim3(L.max_tiles_dn), dim3(kGemmWarps * 32), gemm_smem<1>(), s, L.pdl,
-                      1, a);
+    e = launch_kernel(grouped_gemm_kernel<1>, dim3(L.max_tiles_dn), dim3(kGemmWarps * 32), gemm_smem<1>(a.b_bytes),
+                      s, L.pdl, 1, a);
     if (hook) hook(hook_arg, 2);
     return e;
 }
