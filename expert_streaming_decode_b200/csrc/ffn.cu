@@ -76,11 +76,14 @@ struct DecodeCfg<0> {
     static constexpr int kTilesPerCta = 1;
     static_assert(CPS >= 1 && NSTAGES >= 1, "gate/up ring");
 };
+#ifndef MOE_DECODE_DN_STAGES
+#define MOE_DECODE_DN_STAGES 6
+#endif
 template <>
 struct DecodeCfg<1> {
     static constexpr int NW = 11;
     static constexpr int CPS = 1;
-    static constexpr int NSTAGES = 6;
+    static constexpr int NSTAGES = MOE_DECODE_DN_STAGES;
     static constexpr int STAGE = 18 * kDownSliceMax;
 };
 
