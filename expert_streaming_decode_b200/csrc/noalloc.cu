@@ -2,7 +2,7 @@
 // one token, for callers that are not allowed to allocate device memory.
 //
 // Who needs this: code that runs inside another program's memory budget (a
-// serving engine or graph runtime that hands each plugin a fixed workspace and
+// serving engine or inference runtime that hands each plugin a fixed workspace and
 // owns every device allocation itself), and code on a latency-critical path,
 // where cudaMalloc/cudaFree may synchronise the whole device and take an
 // unbounded time.  Such callers cannot create a moe_ctx (it allocates its

@@ -305,10 +305,9 @@ int moe_expert_ffn(moe_ctx *ctx, const uint16_t *x, int T, int top_k, const int3
  * Scratch: a 4 MiB file-scope device array inside libmoe.so, present on every
  * GPU that loads the library until the process exits.  The FIRST call on each
  * device sets up that device (looks up the array's device address and the
- * kernels' launch shapes, with the device current); make that first call
- * before any stream capture.  Every call shares the array and it keeps the
- * last call's contents: calls whose work overlaps on the GPU race, so issue
- * them on one stream (or order them).  Errors: MOE_ERR_ARG (sizes, pointers),
+ * kernels' launch shapes, with the device current).  Every call shares the
+ * array and it keeps the last call's contents: calls whose work overlaps on
+ * the GPU race, so issue them on one stream (or order them).  Errors: MOE_ERR_ARG (sizes, pointers),
  * MOE_ERR_CUDA (a launch or the set-up failed), MOE_ERR_STATE (the GPU has
  * more SMs than the scratch covers).  Slot indices out of range are clamped;
  * there is no status word to read back. */
