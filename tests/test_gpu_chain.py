@@ -13,6 +13,7 @@ weights, plan traces and slot contents bit for bit (gate weights within 1e-5);
 outputs within max|y - r| <= 2e-3 max|r|; the chained bf16 input within one
 bf16 unit in the last place of the oracle's rounding of the fp64 value."""
 import argparse
+import gc
 
 import numpy as np
 import pytest
@@ -176,3 +177,114 @@ def test_chained_decode_headline_workload(O):
     # the early tokens of the default workload miss in the pages' band
     hit = 1.0 - st["misses"] / (25 * 30 * d.K)
     assert 0.5 < hit < 0.8, hit
+
+
+def _chain_batch(O, d, layers, T, slots, streaming, y_samples, seed=0, zipf=1.1):
+    """One step of the benchmark's multi-token loop (a batched decode step on
+    resident experts, or a prefill chunk through cold slot caches), with the
+    oracle teacher-forced on every layer's bf16 input rows."""
+    args = _args(layers, slots, 0, "copy", seed=seed)
+    args.zipf = zipf  # 0: no popularity bias (the resident workload's uniform router)
+    model = bench.Model(args, synth.Dims(**{**d.as_dict(), "L": layers, "S": slots}), max_tokens=T,
+                        streaming=streaming)
+    moe = model.moe
+    nb = model.nb
+    routers = [synth.router_weights(args.seed, l, d.E, d.D) for l in range(layers)]
+    biases = [synth.zipf_bias(args.seed, l, d.E, s=args.zipf, lam=args.zipf_lambda) if zipf > 0 else None
+              for l in range(layers)]
+    shared = [synth.expert_blob(args.seed, l, 0, d.D, d.FS, shared=True) for l in range(layers)]
+    dev = torch.device("cuda")
+    x0 = torch.empty((T, d.D), dtype=torch.int16, device=dev)
+    x = torch.empty((T, d.D), dtype=torch.int16, device=dev)
+    r = torch.empty((T, d.D), dtype=torch.float32, device=dev)
+    y = torch.empty((T, d.D), dtype=torch.float32, device=dev)
+    ids = torch.empty((T, d.K), dtype=torch.int32, device=dev)
+    gw = torch.empty((T, d.K), dtype=torch.float32, device=dev)
+    tr = moe.Trace(d.E) if streaming else None
+    acc = {"misses": 0, "distinct": 0, "h2d": 0}
+    model.reset()
+    xb0 = synth.hidden_batch(args.seed + 17, range(T), 0, d.D)
+    x0.copy_(torch.from_numpy(xb0.view(np.int16).copy()))
+    stats = {"layers": 0, "outputs": 0, "waves": 0, "misses": 0}
+    prev = {}
+
+    def blobs(l):
+        if streaming:
+            return [model.store.numpy()[l, e, :nb] for e in range(d.E)]
+        return [model.experts[l, e, :nb].cpu().numpy() for e in range(d.E)]
+
+    def on_layer(l, cur, y_t, r_t):
+        torch.cuda.synchronize()
+        model.ctx.sync()
+        xl = cur.cpu().numpy().view(np.uint16).copy()
+        yl = y_t.cpu().numpy().astype(np.float64)
+        rl = r_t.cpu().numpy().astype(np.float64)
+        got_ids, got_w = ids.cpu().numpy(), gw.cpu().numpy()
+        if l == 0:
+            assert np.array_equal(xl, xb0)
+        else:
+            for t in range(T):
+                r_want, x_want = O.residual_rmsnorm(prev["r"][t], prev["y"][t])
+                assert np.all(np.abs(rl[t] - r_want) <= np.abs(r_want) * 2.0 ** -24 + 1e-30), (t, l)
+                assert _bf16_ulp_diff(xl[t], x_want).max() <= 1.0, (t, l)
+        wq, ws = routers[l]
+        lgs = [O.router_logits(xl[t], wq, ws, biases[l], d.E, d.D, d.G) for t in range(T)]
+        want_ids = np.stack([O.topk(lg, d.K) for lg in lgs])
+        assert np.array_equal(got_ids, want_ids), l
+        for t in range(T):
+            assert np.max(np.abs(got_w[t] - O.gate_weights(lgs[t], want_ids[t]))) <= GATE_TOL, (t, l)
+        if streaming:
+            plan = tr.result()
+            want = O.lfu_plan(oracle.LfuState(d.E, slots), want_ids, 0)  # every chunk starts cold
+            for key in ("expert", "slot", "hit", "victim", "wave"):
+                assert np.array_equal(plan[key], want[key]), (l, key)
+            assert plan["waves"] == want["waves"]
+            stats["waves"] += plan["waves"]
+            stats["misses"] += plan["misses"]
+        rows = [t for (t, ll) in y_samples if ll == l]
+        if rows:
+            bl = blobs(l)
+            for t in rows:
+                _, _, _, want_y = O.moe_token(d.as_dict(), xl[t], wq, ws, biases[l], shared[l], bl)
+                err = rel_err(yl[t], want_y)
+                assert err <= TOL, (t, l, err)
+                stats["outputs"] += 1
+        stats["layers"] += 1
+        prev["r"], prev["y"] = rl, yl
+
+    bench.decode_token(model, x0, r, x, y, T, 0, tr=tr, trace_acc=acc if streaming else None, on_layer=on_layer,
+                       ids=ids, gate_w=gw)
+    torch.cuda.synchronize()
+    model.ctx.sync()
+    model.ctx.close()
+    assert stats["layers"] == layers and stats["outputs"] == len(y_samples)
+    return stats
+
+
+@pytest.mark.parametrize("T", [8, 32])
+def test_chained_batched_decode_resident_30_layers(O, T):
+    """The resident batched-decode workload at full size: 30 chained layers
+    of the 26B-A4B shape with every expert in HBM, a step of T tokens through
+    the tensor-core grouped GEMM (uniform router, as the benchmark runs it).
+    Ids and gate weights of every token at every layer, the chained inputs,
+    and outputs on a sample of (token, layer)."""
+    d = synth.GEMMA4_26B
+    samples = {(0, 0), (T - 1, 4), (T // 2, 11), (1, 19), (T - 2, 25), (T // 3, 29)}
+    torch.cuda.empty_cache()
+    _chain_batch(O, d, layers=30, T=T, slots=16, streaming=False, y_samples=samples, zipf=0.0)
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
+def test_chained_prefill_chunk_30_layers(O):
+    """The prefill workload at full size: a 128-token chunk through 30 chained
+    layers of the 26B-A4B shape, every layer's 16-slot cache cold, the plan in
+    waves, misses copied from the pinned host store; ids, gate weights, plans
+    and chained inputs at every layer, outputs on a sample."""
+    d = synth.GEMMA4_26B
+    samples = {(0, 0), (127, 3), (64, 9), (5, 16), (100, 23), (31, 29)}
+    torch.cuda.empty_cache()
+    st = _chain_batch(O, d, layers=30, T=128, slots=16, streaming=True, y_samples=samples)
+    assert st["waves"] > 30 and st["misses"] > 0
+    gc.collect()
+    torch.cuda.empty_cache()

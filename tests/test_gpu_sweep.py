@@ -12,13 +12,15 @@ from gpu_data import bf16_tensor
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("S,zs", [(8, 0.8), (16, 1.1), (32, 1.4), (64, 0.8)])
-def test_sweep_trace_bit_exact(S, zs):
+@pytest.mark.parametrize("S,zs,tokens", [(8, 0.8, 500), (16, 1.1, 500), (32, 1.4, 500), (64, 0.8, 500),
+                                         (16, 1.1, 4096)])
+def test_sweep_trace_bit_exact(S, zs, tokens):
+    """Two layers; the last case runs the sweep's full 4096-token length."""
     d = synth.GEMMA4_26B
     O = oracle.get()
     ctx = moe.Ctx.from_dims(d, max_tokens=1, S=S)
     nb = synth.blob_bytes(d.D, d.F)
-    layers, tokens = 2, 500
+    layers = 2
     wq, ws, bias, caches, ost = [], [], [], [], []
     slots = torch.empty((S, 256), dtype=torch.uint8, device="cuda")  # plan only: never read
     for l in range(layers):
