@@ -106,6 +106,9 @@ struct moe_ctx {
     float* pf_gw = nullptr;                // device scratch: their gate weights
     cudaStream_t pf_stream = nullptr;
     cudaEvent_t ev_x = nullptr, ev_pred = nullptr;
+    // side stream: after the last staging copies; look-ahead stream: after
+    // the last moves of staged blobs into their slots
+    cudaEvent_t ev_staged = nullptr, ev_moved = nullptr;
     struct Prefetched {
         const int32_t* state;  // the cache the blob was fetched for
         const uint8_t* store;  // and the store it was copied from
@@ -174,6 +177,8 @@ void free_ctx(moe_ctx* c) {
     if (c->pf_ids_host) cudaFreeHost(c->pf_ids_host);
     if (c->ev_x) cudaEventDestroy(c->ev_x);
     if (c->ev_pred) cudaEventDestroy(c->ev_pred);
+    if (c->ev_staged) cudaEventDestroy(c->ev_staged);
+    if (c->ev_moved) cudaEventDestroy(c->ev_moved);
     if (c->pf_stream) cudaStreamDestroy(c->pf_stream);
     for (auto& r : c->recs) {
         cudaEventDestroy(r.a);
@@ -459,13 +464,18 @@ int fill_wave(moe_ctx* c, const moe_slot_cache* cache, int w, cudaEvent_t after,
         if (cudaStreamWaitEvent(s, c->ev_fill, 0) != cudaSuccess) return MOE_ERR_CUDA;
         return MOE_OK;
     }
-    // Blobs prefetched for this cache are moved from their HBM buffers (the
-    // prefetch copies are earlier on the same side stream), the others copied
-    // from the host store.  With per-miss completion (ready_seq != 0) the
-    // staged blobs go first and the compute stream waits for them by event:
-    // a device-to-device copy may run as a kernel, which must not queue behind
-    // routed-expert kernels that wait on these blobs.  The host copies run on
-    // the copy engine and are announced one by one.
+    // Blobs prefetched for this cache are moved from their HBM buffers, the
+    // others copied from the host store.  By default the moves run on the
+    // look-ahead stream, after the staging copies (event) and the wave's
+    // order point, so that the host link starts on the first missed blob at
+    // once; the compute stream waits for the moves by event.  With per-miss
+    // completion (ready_seq != 0) the staged blobs go first on the side stream
+    // and the compute stream waits for them by event: a device-to-device copy
+    // may run as a kernel, which must not queue behind routed-expert kernels
+    // that wait on these blobs.  The host copies run on the copy engine and are
+    // announced one by one.
+    const bool move_aside = ready_seq == 0u && c->pf_stream != nullptr;
+    bool moving = false;
     bool first_ready = true;
     int n_staged = 0;
     for (int pass = 0; pass < 2; ++pass) {
@@ -478,9 +488,15 @@ int fill_wave(moe_ctx* c, const moe_slot_cache* cache, int w, cudaEvent_t after,
             for (const auto& f : c->pf_table)
                 if (f.state == cache->state && f.store == cache->store && f.expert == e) pb = f.buf;
             if ((pb >= 0) != (pass == 0)) continue;
+            if (pb >= 0 && move_aside && !moving) {
+                if (cudaStreamWaitEvent(c->pf_stream, after, 0) != cudaSuccess ||
+                    cudaStreamWaitEvent(c->pf_stream, c->ev_staged, 0) != cudaSuccess)
+                    return MOE_ERR_CUDA;
+                moving = true;
+            }
             const cudaError_t ce =
                 pb >= 0 ? cudaMemcpyAsync(dst, c->pf_buf + size_t(pb) * c->pf_stride, nb, cudaMemcpyDeviceToDevice,
-                                          c->side)
+                                          move_aside ? c->pf_stream : c->side)
                         : cudaMemcpyAsync(dst, cache->store + size_t(e) * cache->store_stride, nb,
                                           cudaMemcpyHostToDevice, c->side);
             if (ce != cudaSuccess) return MOE_ERR_CUDA;
@@ -499,6 +515,13 @@ int fill_wave(moe_ctx* c, const moe_slot_cache* cache, int w, cudaEvent_t after,
                 ++n_staged;
             }
             *bytes += nb;
+        }
+        if (pass == 0 && moving) {
+            // the list that reads the moved blobs waits for the moves; the next
+            // staging copies wait for them too (they may reuse the buffers)
+            if (cudaEventRecord(c->ev_moved, c->pf_stream) != cudaSuccess ||
+                cudaStreamWaitEvent(s, c->ev_moved, 0) != cudaSuccess)
+                return MOE_ERR_CUDA;
         }
         if (pass == 0 && ready_seq && n_staged > 0) {
             if (cudaEventRecord(c->ev_fill, c->side) != cudaSuccess) return MOE_ERR_CUDA;
@@ -1119,6 +1142,7 @@ static int layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache*
             }
             return -1;
         };
+        bool waited = false;  // the side stream waits for the moves once, before the first staging copy
         // stage up to `limit` predicted misses of layer L (ids at pred); returns
         // how many of its predicted misses are missing from its cache and the buffers
         auto stage = [&](const moe_next_layer* L, const int32_t* pred, int limit, int* n_stage) -> int {
@@ -1130,6 +1154,9 @@ static int layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache*
                 ++wanted;
                 const int b = *n_stage < limit ? free_buf() : -1;
                 if (b < 0) continue;
+                // a buffer freed by this call may still be read by its move
+                if (!waited && cudaStreamWaitEvent(c->side, c->ev_moved, 0) != cudaSuccess) return -1;
+                waited = true;
                 if (cudaMemcpyAsync(c->pf_buf + size_t(b) * c->pf_stride, L->cache->store + size_t(e) * L->cache->store_stride,
                                     c->blob_routed, cudaMemcpyHostToDevice, c->side) != cudaSuccess)
                     return -1;
@@ -1146,6 +1173,8 @@ static int layer_forward(moe_ctx* c, const moe_layer_weights* W, moe_slot_cache*
             int n2 = 0;
             if (stage(after, c->pf_ids_host + K, 1, &n2) < 0) return MOE_ERR_CUDA;
         }
+        // the moves of staged blobs wait for this point of the side stream
+        if (waited && cudaEventRecord(c->ev_staged, c->side) != cudaSuccess) return MOE_ERR_CUDA;
     }
     copy_trace(c->mbox_host, trace, c->blob_routed, bytes);
     return MOE_OK;
@@ -1185,6 +1214,8 @@ int moe_prefetch_configure(moe_ctx* c, int n_buffers) {
         ok = ok && cudaStreamCreateWithFlags(&c->pf_stream, cudaStreamNonBlocking) == cudaSuccess;
         ok = ok && cudaEventCreateWithFlags(&c->ev_x, cudaEventDisableTiming) == cudaSuccess;
         ok = ok && cudaEventCreateWithFlags(&c->ev_pred, cudaEventDisableTiming) == cudaSuccess;
+        ok = ok && cudaEventCreateWithFlags(&c->ev_staged, cudaEventDisableTiming) == cudaSuccess;
+        ok = ok && cudaEventCreateWithFlags(&c->ev_moved, cudaEventDisableTiming) == cudaSuccess;
         // the predicted ids of the next layer, then of the layer after it
         ok = ok && cudaHostAlloc(reinterpret_cast<void**>(&c->pf_ids_host), sizeof(int32_t) * size_t(2 * c->d.top_k),
                                  cudaHostAllocMapped) == cudaSuccess;
