@@ -371,7 +371,9 @@ int moe_layer_forward(moe_ctx *ctx, const moe_layer_weights *W, moe_slot_cache *
  * predicted experts that layer l+1's cache does not hold (as far as the host
  * has seen from the plans it read) are copied from layer l+1's host store into
  * HBM staging buffers.  When layer l+1 runs, a miss whose blob is staged is
- * filled by a device-to-device copy instead of a host copy.  The cache plan,
+ * filled by a device-to-device copy instead of a host copy, issued on the
+ * look-ahead stream so that the host copies of its other misses start at once
+ * (the layer's routed experts wait for both by event).  The cache plan,
  * the trace and the outputs are exactly those of moe_layer_forward; only
  * where a missed blob is copied from changes.
  *
